@@ -1,0 +1,379 @@
+"""Benchmark of the fused sigmoid-gating GDN decode update on B200.
+
+One step = one call of the whole hot path (one fused kernel) over one batch
+of the Qwen3-Next per-rank decode shape: B = 512 sequences, T = 1, H = 4 key
+heads, HV = 8 value heads, K = V = 128, fp32 state pool of 1024 slots, 5 %
+padded (-1) slots.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...    (one replica per GPU)
+
+value      whole-job state-traffic throughput: algorithmic HBM bytes of all
+           ranks' steps / max-over-ranks device time (CUDA events), GB/s.
+           Inputs are resident in HBM; consecutive steps rotate over 4 copies
+           of the inputs (2.1 GB in all), so no step finds its data in L2.
+e2e        the same metric through the public API with pinned HOST buffers:
+           every step copies its inputs host -> device, runs the update and
+           reads the output back, synchronising on the result.
+roofline   the fused kernel against the measured HBM copy bandwidth.
+cpu_baseline  the CPU oracle (single thread, fp64) on a bounded sample of
+           the same workload (rank 0, N = 1 only).
+--impl reference  times the CPU oracle alone (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl  # noqa: E402
+
+METRIC = "µs/call and state GB/s (% of B200 HBM peak) at B=512, HV=8, K=V=128"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ROTATING_COPIES = 4
+
+# DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
+# ncu capture summarised in profiles/ (dram__bytes_read.sum +
+# dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
+NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_recurrent_sigmoid_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+CLOCK_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                "clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of this GPU's clocks while the timed region runs."""
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            import torch
+            ident = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            ident = str(device_index)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(REASON_NAMES, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_subset_seconds(w, seqs):
+    """Wall time of the oracle on a subset of sequences (its own inputs)."""
+    import oracle
+    lens = w.seq_lens
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    rows = np.concatenate([np.arange(starts[i], starts[i] + lens[i]) for i in seqs])
+    flat = lambda x, tail: x.reshape((-1,) + x.shape[-tail:])[rows]
+    slots = w.state_indices[seqs]
+    live = slots >= 0
+    idx = np.full(len(seqs), -1, np.int32)
+    idx[live] = np.arange(live.sum(), dtype=np.int32)
+    cu = np.zeros(len(seqs) + 1, np.int32)
+    cu[1:] = np.cumsum(lens[seqs])
+    args = (flat(w.q, 2), flat(w.k, 2), flat(w.v, 2), flat(w.a, 1), flat(w.b, 1), w.A_log, w.dt_bias,
+            np.ascontiguousarray(w.state_pool[slots[live]]), idx, cu)
+    t0 = time.perf_counter()
+    oracle.update(*args)
+    return time.perf_counter() - t0
+
+
+def subset_bytes(w, seqs):
+    s = w.spec
+    live = w.state_indices[seqs] >= 0
+    lens = w.seq_lens[seqs]
+    head = s.K * s.V * 4
+    nbytes = 2 * int(live.sum()) * s.HV * head
+    nbytes += int(lens[live].sum()) * (2 * s.H * s.K + s.HV * s.V + 2 * s.HV) * 2
+    nbytes += int(lens.sum()) * s.HV * s.V * 2 + 8 * s.HV + 4 * len(seqs)
+    return nbytes
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle as it stands, single-threaded, over the whole workload
+    repeated until about ``budget_s`` seconds of CPU work."""
+    seqs = np.arange(w.spec.N)
+    total_t, reps = 0.0, 0
+    while reps == 0 or total_t < budget_s:
+        total_t += oracle_subset_seconds(w, seqs)
+        reps += 1
+    per = total_t / reps
+    return {"value": round(wl.algorithmic_bytes(w) / per / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "us_per_call": round(per * 1e6, 1),
+            "sample": f"whole {w.spec.name} workload ({w.spec.N} sequences), {reps} repetitions, "
+                      f"{total_t:.1f} s single-threaded fp64 C loop nest"}
+
+
+def run_reference(args, w):
+    """Reference arm: the CPU oracle on bounded per-step samples."""
+    N = w.spec.N
+    rng = np.random.default_rng(0)
+    t1 = oracle_subset_seconds(w, np.arange(min(8, N))) / min(8, N)
+    budget = 120.0
+    per_step = max(1, min(N, int(budget / max(1, args.steps + args.warmup) / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_subset_seconds(w, rng.choice(N, per_step, replace=False))
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        seqs = np.sort(rng.choice(N, per_step, replace=False))
+        tot_t += oracle_subset_seconds(w, seqs)
+        tot_b += subset_bytes(w, seqs)
+    value = tot_b / tot_t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, 1),
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": round(value, 4), "unit": "GB/s",
+                             "sample": f"{per_step} random sequences of {w.spec.name} per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def workload_config(w, world):
+    s = w.spec
+    return {"workload": s.name, "B": s.N, "T": s.T if s.T is not None else "U{1..64}", "H": s.H, "HV": s.HV,
+            "K": s.K, "V": s.V, "num_slots": s.num_slots, "padded": int((w.state_indices < 0).sum()),
+            "state_dtype": "f32", "activation_dtype": "bf16",
+            "l2": f"inputs larger than L2: steps rotate over {ROTATING_COPIES} input copies",
+            "parallelism": "replicas" if world == 1 else f"dp{world}"}
+
+
+def device_copy(w, torch, device):
+    bf = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(device)
+    d = dict(q=bf(w.q), k=bf(w.k), v=bf(w.v), a=bf(w.a), b=bf(w.b),
+             A_log=torch.from_numpy(w.A_log).to(device), dt_bias=torch.from_numpy(w.dt_bias).to(device),
+             state_pool=torch.from_numpy(w.state_pool).to(device),
+             state_indices=torch.from_numpy(w.state_indices).to(device),
+             cu_seqlens=None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).to(device))
+    d["out"] = torch.empty(w.v.shape, dtype=torch.bfloat16, device=device)
+    if w.spec.intermediate:
+        d["inter"] = torch.empty((w.T_tot, w.spec.HV, w.spec.K, w.spec.V), device=device)
+    return d
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=wl.DECODE_B512.name, choices=sorted(wl.BY_NAME))
+    ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
+    ap.add_argument("--tile-v", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.generate(wl.BY_NAME[args.workload])
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from gated_deltanet_recurrent_sigmoid_b200 import binding, build
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if local_rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    binding.load()
+
+    stream = torch.cuda.Stream(device)
+    copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
+    flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
+    calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"], c["state_pool"],
+                                  c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
+                                  intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v)
+             for c in copies]
+    nbytes = wl.algorithmic_bytes(w)
+    torch.cuda.synchronize(device)
+
+    # warm-up
+    for s in range(args.warmup):
+        calls[s % len(calls)]()
+    stream.synchronize()
+
+    # timed region: K steps, one fused kernel each, events on the launch stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(local_rank)
+    time.sleep(0.2)
+    region0.record(stream)
+    for s in range(args.steps):
+        starts[s].record(stream)
+        calls[s % len(calls)]()
+        ends[s].record(stream)
+    region1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    region_ms = region0.elapsed_time(region1)
+    kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    avg_kernel_ms = sum(kernel_ms) / len(kernel_ms)
+
+    t = torch.tensor([region_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_region_ms = float(t.item())
+    ms_per_step = max_region_ms / args.steps
+    value = nbytes * world * args.steps / (max_region_ms * 1e-3) / 1e9
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.skip_e2e:
+        host = {n: copies[0][n].cpu().pin_memory() for n in ("q", "k", "v", "a", "b", "state_indices")}
+        if copies[0]["cu_seqlens"] is not None:
+            host["cu_seqlens"] = copies[0]["cu_seqlens"].cpu().pin_memory()
+        host["out"] = torch.empty(copies[0]["out"].shape, dtype=torch.bfloat16).pin_memory()
+        dev = dict(copies[0])
+        dev["intermediate_states"] = dev.pop("inter", None)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in host if n != "out")
+        d2h = host["out"].numel() * host["out"].element_size()
+        for _ in range(3):
+            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v)
+            stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v)
+            stream.synchronize()          # the step ends when the host holds the output
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / args.e2e_steps
+        e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank == 0:
+        peak, peak_src = hbm_peak()
+        achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
+        traffic = None
+        if NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash():
+            traffic = NCU_TRAFFIC["bytes_per_launch"]
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(w, world),
+            "us_per_call": round(avg_kernel_ms * 1e3, 3),
+            "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "peak_source": peak_src},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
+                         "kernel": "gdn::gdn_decode_kernel"},
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.skip_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+
+    del calls
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

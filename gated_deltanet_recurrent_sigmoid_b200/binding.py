@@ -1,0 +1,201 @@
+"""Thin ctypes binding of ``libgdn_decode.so`` (C ABI in include/gdn_decode.h).
+
+Argument marshalling only: torch tensors are described to the C ABI by
+their device pointer, dtype, shape and strides, and the current CUDA stream
+is passed along.  Every step of the update runs in the library's kernel.
+The library is loaded on first use; if it is missing this module raises --
+there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+L2NORM_QK = 1 << 0
+WRITE_INTERMEDIATE = 1 << 1
+NO_FINAL_WRITEBACK = 1 << 2
+CHECK_INDICES = 1 << 3
+
+DEV_BAD_SLOT = 1
+DEV_BAD_SEQLENS = 2
+
+OK = 0
+ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5
+ERR_UNSUPPORTED, ERR_ARG, ERR_INDICES, ERR_CUDA = -6, -7, -8, -9
+
+_DTYPE_CODES = {torch.bfloat16: 1, torch.float32: 2, torch.int32: 3}
+
+
+class GdnError(RuntimeError):
+    """A non-zero status from the C ABI."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class GdnTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class GdnExtra(ctypes.Structure):
+    _fields_ = [("stream", ctypes.c_void_p), ("intermediate_states", ctypes.POINTER(GdnTensor)),
+                ("device_status", ctypes.c_void_p), ("tile_v", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_LIB = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library; raise if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path):
+            raise GdnError(ERR_CUDA, f"{path} is missing: build it with "
+                                     "`python -m gated_deltanet_recurrent_sigmoid_b200.build`")
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER(GdnTensor)
+        lib.gdn_decode_update.restype = ctypes.c_int
+        lib.gdn_decode_update.argtypes = [P] * 11 + [ctypes.c_float, ctypes.c_uint32, ctypes.POINTER(GdnExtra)]
+        lib.gdn_status_string.restype = ctypes.c_char_p
+        lib.gdn_status_string.argtypes = [ctypes.c_int]
+        lib.gdn_version.restype = ctypes.c_int
+        lib.gdn_version.argtypes = []
+        _LIB = lib
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def describe(t: Optional[torch.Tensor]) -> Optional[GdnTensor]:
+    """gdn_tensor descriptor of a tensor (None stays None)."""
+    if t is None:
+        return None
+    if t.dim() < 1 or t.dim() > 4:
+        raise GdnError(ERR_SHAPE, f"rank {t.dim()} tensor cannot cross the C ABI")
+    d = GdnTensor()
+    d.data = t.data_ptr()
+    d.dtype = _DTYPE_CODES.get(t.dtype, 0)
+    d.ndim = t.dim()
+    for i, (n, s) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = n
+        d.stride[i] = s
+    return d
+
+
+def _ref(d: Optional[GdnTensor]):
+    return None if d is None else ctypes.byref(d)
+
+
+def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
+                  A_log: torch.Tensor, dt_bias: torch.Tensor, state_pool: torch.Tensor,
+                  state_indices: torch.Tensor, cu_seqlens: Optional[torch.Tensor], out: torch.Tensor,
+                  scale: Optional[float] = None, flags: int = L2NORM_QK,
+                  intermediate_states: Optional[torch.Tensor] = None,
+                  device_status: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0) -> torch.Tensor:
+    """Fused sigmoid-gating GDN decode update, in place on ``state_pool``.
+
+    Shapes, dtypes and semantics are those of ``gdn_decode_update`` in
+    include/gdn_decode.h.  ``scale`` defaults to 1/sqrt(K).  ``flags`` gets
+    WRITE_INTERMEDIATE added automatically when ``intermediate_states`` is
+    given.  Runs asynchronously on ``stream`` (default: the current torch
+    stream).  Returns ``out``.  Raises GdnError on a non-zero status.
+    """
+    lib = load()
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if intermediate_states is not None:
+        flags |= WRITE_INTERMEDIATE
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    descs = [describe(t) for t in (q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out)]
+    inter = describe(intermediate_states)
+    extra = GdnExtra()
+    extra.stream = stream.cuda_stream if stream is not None else None
+    extra.intermediate_states = ctypes.pointer(inter) if inter is not None else None
+    extra.device_status = device_status.data_ptr() if device_status is not None else None
+    extra.tile_v = int(tile_v)
+    extra.reserved = 0
+    status = lib.gdn_decode_update(*[_ref(d) for d in descs], ctypes.c_float(scale), ctypes.c_uint32(flags),
+                                   ctypes.byref(extra))
+    if status != OK:
+        raise GdnError(status, status_string(status))
+    return out
+
+
+def decode_update_host(host: dict, device: dict, *, scale: Optional[float] = None, flags: int = L2NORM_QK,
+                       stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0) -> None:
+    """End-to-end call from pinned host buffers.
+
+    ``host`` holds pinned CPU tensors q, k, v, a, b, state_indices,
+    cu_seqlens (optional) and out; ``device`` holds device tensors of the
+    same names plus A_log, dt_bias, state_pool (resident) and optionally
+    intermediate_states.  The call copies the per-step inputs host -> device,
+    runs the update and copies ``out`` device -> host, all on ``stream``
+    (asynchronous; synchronise the stream before reading host ``out``).
+    """
+    if stream is None:
+        stream = torch.cuda.current_stream(device["q"].device)
+    with torch.cuda.stream(stream):
+        for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
+            if host.get(name) is not None:
+                device[name].copy_(host[name], non_blocking=True)
+        decode_update(device["q"], device["k"], device["v"], device["a"], device["b"], device["A_log"],
+                      device["dt_bias"], device["state_pool"], device["state_indices"], device.get("cu_seqlens"),
+                      device["out"], scale=scale, flags=flags,
+                      intermediate_states=device.get("intermediate_states"), stream=stream, tile_v=tile_v)
+        host["out"].copy_(device["out"], non_blocking=True)
+
+
+class PreparedCall:
+    """A decode update whose descriptors are built once.
+
+    For a serving loop that calls the update on the same buffers every step
+    (the state pool, index and activation buffers are reused), this removes
+    the per-call descriptor marshalling; each ``__call__`` is one C-ABI call
+    that enqueues one kernel on ``stream``.  The tensors must stay alive and
+    keep their storage while the object is used.
+    """
+
+    def __init__(self, q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
+                 scale: Optional[float] = None, flags: int = L2NORM_QK, intermediate_states=None,
+                 device_status=None, stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0):
+        self._lib = load()
+        self._keep = (q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
+                      intermediate_states, device_status)
+        if scale is None:
+            scale = 1.0 / math.sqrt(q.shape[-1])
+        if intermediate_states is not None:
+            flags |= WRITE_INTERMEDIATE
+        self._descs = [describe(t) for t in self._keep[:11]]
+        self._inter = describe(intermediate_states)
+        self._extra = GdnExtra()
+        self.stream = stream if stream is not None else torch.cuda.current_stream(q.device)
+        self._extra.stream = self.stream.cuda_stream
+        self._extra.intermediate_states = ctypes.pointer(self._inter) if self._inter is not None else None
+        self._extra.device_status = device_status.data_ptr() if device_status is not None else None
+        self._extra.tile_v = int(tile_v)
+        self._args = [_ref(d) for d in self._descs] + [ctypes.c_float(scale), ctypes.c_uint32(flags),
+                                                       ctypes.byref(self._extra)]
+        self._fn = self._lib.gdn_decode_update
+
+    def __call__(self) -> None:
+        status = self._fn(*self._args)
+        if status != OK:
+            raise GdnError(status, status_string(status))

@@ -1,0 +1,414 @@
+// gdn_decode_api.cu -- host side of the C ABI declared in include/gdn_decode.h:
+// argument validation, parameter marshalling and the kernel launch.
+//
+// Every check runs on the host before anything is enqueued, and none of
+// them touches device memory or calls the CUDA runtime (only the optional
+// GDN_CHECK_INDICES copies the index arrays back).  This file holds no step
+// of the update's arithmetic; the kernel does all of it.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "gdn_decode.h"
+#include "gdn_decode_kernel.cuh"
+
+namespace {
+
+constexpr int kHeadK = 128;
+constexpr int kHeadV = 128;
+
+int64_t elem_size(int32_t dtype)
+{
+    switch (dtype) {
+    case GDN_DTYPE_BF16: return 2;
+    case GDN_DTYPE_F32: return 4;
+    case GDN_DTYPE_I32: return 4;
+    default: return 0;
+    }
+}
+
+bool aligned(const void *p, uintptr_t bytes) { return (reinterpret_cast<uintptr_t>(p) % bytes) == 0; }
+
+// Byte range a descriptor can reach: [lo, hi).  Empty when any dim is 0.
+struct Span {
+    uintptr_t lo = 0, hi = 0;
+    bool empty() const { return hi <= lo; }
+};
+
+Span span_of(const gdn_tensor *t)
+{
+    Span s;
+    if (!t || !t->data)
+        return s;
+    int64_t last = 0;
+    for (int d = 0; d < t->ndim; ++d) {
+        if (t->shape[d] == 0)
+            return s;
+        last += (t->shape[d] - 1) * t->stride[d];
+    }
+    s.lo = reinterpret_cast<uintptr_t>(t->data);
+    s.hi = s.lo + static_cast<uintptr_t>((last + 1) * elem_size(t->dtype));
+    return s;
+}
+
+bool overlap(const Span &x, const Span &y)
+{
+    if (x.empty() || y.empty())
+        return false;
+    return x.lo < y.hi && y.lo < x.hi;
+}
+
+// Basic descriptor sanity: rank, non-negative shape and strides, and a data
+// pointer unless the tensor has no elements.
+int check_desc(const gdn_tensor *t, int32_t dtype)
+{
+    if (!t)
+        return GDN_ERR_NULL_ARG;
+    if (t->dtype != dtype)
+        return GDN_ERR_DTYPE;
+    if (t->ndim < 1 || t->ndim > 4)
+        return GDN_ERR_SHAPE;
+    bool empty = false;
+    for (int d = 0; d < t->ndim; ++d) {
+        if (t->shape[d] < 0 || t->stride[d] < 0)
+            return GDN_ERR_SHAPE;
+        empty = empty || t->shape[d] == 0;
+    }
+    if (!t->data && !empty)
+        return GDN_ERR_NULL_ARG;
+    return GDN_OK;
+}
+
+// Token layout of an activation whose trailing `trail` dims are per token.
+// Varlen: leading dims [T_tot] or [1, T_tot].  Fixed length: [N, T], which
+// must flatten to one token dimension.
+struct TokenLayout {
+    int64_t T_tot = 0;   // tokens
+    int64_t T = 0;       // tokens per sequence (fixed-length mode)
+    int64_t tok = 0;     // stride between consecutive tokens, in elements
+};
+
+int token_layout(const gdn_tensor *t, int trail, bool varlen, int64_t N, TokenLayout *L)
+{
+    const int lead = t->ndim - trail;
+    if (varlen) {
+        if (lead == 1) {
+            L->T_tot = t->shape[0];
+            L->tok = t->stride[0];
+        } else if (lead == 2 && t->shape[0] == 1) {
+            L->T_tot = t->shape[1];
+            L->tok = t->stride[1];
+        } else {
+            return GDN_ERR_SHAPE;
+        }
+        L->T = -1;
+        return GDN_OK;
+    }
+    if (lead != 2 || t->shape[0] != N)
+        return GDN_ERR_SHAPE;
+    const int64_t T = t->shape[1];
+    L->T = T;
+    L->T_tot = N * T;
+    if (T == 0 || N == 0)
+        L->tok = 0;  // no tokens: the stride is never used
+    else if (T == 1)
+        L->tok = t->stride[0];
+    else if (N == 1)
+        L->tok = t->stride[1];
+    else if (t->stride[0] != T * t->stride[1])
+        return GDN_ERR_SHAPE;
+    else
+        L->tok = t->stride[1];
+    return GDN_OK;
+}
+
+// The stride of a dim matters only when the dim has more than one entry.
+bool stride_ok(int64_t extent, int64_t stride, int64_t multiple)
+{
+    return extent <= 1 || stride % multiple == 0;
+}
+
+#define GDN_TRY(expr)              \
+    do {                           \
+        const int rc_ = (expr);    \
+        if (rc_ != GDN_OK)         \
+            return rc_;            \
+    } while (0)
+
+// Host-side index check (GDN_CHECK_INDICES).
+int check_indices_on_host(const int32_t *d_idx, const int32_t *d_cu, int64_t N, int64_t num_slots,
+                          int64_t T_tot, cudaStream_t stream)
+{
+    std::vector<int32_t> idx(static_cast<size_t>(N));
+    std::vector<int32_t> cu(d_cu ? static_cast<size_t>(N + 1) : 0);
+    if (cudaMemcpyAsync(idx.data(), d_idx, sizeof(int32_t) * N, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (d_cu && cudaMemcpyAsync(cu.data(), d_cu, sizeof(int32_t) * (N + 1), cudaMemcpyDeviceToHost, stream) !=
+                    cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    std::vector<uint8_t> seen(static_cast<size_t>(num_slots), 0);
+    for (int64_t i = 0; i < N; ++i) {
+        const int32_t s = idx[i];
+        if (s < -1 || s >= num_slots)
+            return GDN_ERR_INDICES;
+        if (s >= 0) {
+            if (seen[s])
+                return GDN_ERR_INDICES;
+            seen[s] = 1;
+        }
+    }
+    if (d_cu) {
+        if (cu[0] < 0)
+            return GDN_ERR_INDICES;
+        for (int64_t i = 0; i < N; ++i)
+            if (cu[i + 1] < cu[i])
+                return GDN_ERR_INDICES;
+        if (cu[N] > T_tot)
+            return GDN_ERR_INDICES;
+    }
+    return GDN_OK;
+}
+
+template <int BV, int KG>
+cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream)
+{
+    using TS = gdn::TileShape<kHeadK, kHeadV, BV, KG>;
+    const dim3 grid(static_cast<unsigned>(units * TS::NV));
+    gdn::gdn_decode_kernel<kHeadK, kHeadV, BV, KG><<<grid, TS::THREADS, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+GDN_API int gdn_version(void) { return GDN_DECODE_ABI_VERSION; }
+
+GDN_API const char *gdn_status_string(int status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK: success";
+    case GDN_ERR_NULL_ARG: return "GDN_ERR_NULL_ARG: a required tensor or pointer is NULL";
+    case GDN_ERR_DTYPE: return "GDN_ERR_DTYPE: a tensor has the wrong dtype";
+    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: a tensor has the wrong rank, shape or strides";
+    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: a pointer or stride breaks an alignment rule";
+    case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: a written tensor overlaps another tensor";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: head size or V-tile not built";
+    case GDN_ERR_ARG: return "GDN_ERR_ARG: bad scalar argument or flag";
+    case GDN_ERR_INDICES: return "GDN_ERR_INDICES: bad or repeated state index, or bad cu_seqlens";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: the CUDA runtime refused the launch or copy";
+    default: return "unknown gdn status";
+    }
+}
+
+GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                              const gdn_tensor *a, const gdn_tensor *b, const gdn_tensor *A_log,
+                              const gdn_tensor *dt_bias, const gdn_tensor *state_pool,
+                              const gdn_tensor *state_indices, const gdn_tensor *cu_seqlens,
+                              const gdn_tensor *out, float scale, uint32_t flags, const gdn_extra *extra)
+{
+    // ---- scalars and flags
+    const uint32_t known = GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES;
+    if ((flags & ~known) != 0 || !std::isfinite(scale) || !(scale > 0.f))
+        return GDN_ERR_ARG;
+    if (extra && extra->reserved != 0)
+        return GDN_ERR_ARG;
+    const bool want_inter = (flags & GDN_WRITE_INTERMEDIATE) != 0;
+    const gdn_tensor *inter = extra ? extra->intermediate_states : nullptr;
+    if (want_inter && !inter)
+        return GDN_ERR_NULL_ARG;
+
+    // ---- descriptors and dtypes
+    GDN_TRY(check_desc(q, GDN_DTYPE_BF16));
+    GDN_TRY(check_desc(k, GDN_DTYPE_BF16));
+    GDN_TRY(check_desc(v, GDN_DTYPE_BF16));
+    GDN_TRY(check_desc(a, GDN_DTYPE_BF16));
+    GDN_TRY(check_desc(b, GDN_DTYPE_BF16));
+    GDN_TRY(check_desc(A_log, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(dt_bias, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(state_pool, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(state_indices, GDN_DTYPE_I32));
+    GDN_TRY(check_desc(out, GDN_DTYPE_BF16));
+    if (cu_seqlens)
+        GDN_TRY(check_desc(cu_seqlens, GDN_DTYPE_I32));
+    if (want_inter)
+        GDN_TRY(check_desc(inter, GDN_DTYPE_F32));
+    const bool varlen = cu_seqlens != nullptr;
+
+    // ---- shapes
+    if (state_indices->ndim != 1 || q->ndim < 3 || q->ndim > 4)
+        return GDN_ERR_SHAPE;
+    const int64_t N = state_indices->shape[0];
+    const int64_t H = q->shape[q->ndim - 2], K = q->shape[q->ndim - 1];
+    if (v->ndim != q->ndim)
+        return GDN_ERR_SHAPE;
+    const int64_t HV = v->shape[v->ndim - 2], V = v->shape[v->ndim - 1];
+    if (H <= 0 || HV <= 0 || HV % H != 0 || K <= 0 || V <= 0)
+        return GDN_ERR_SHAPE;
+
+    TokenLayout Lq, Lk, Lv, La, Lb, Lo;
+    GDN_TRY(token_layout(q, 2, varlen, N, &Lq));
+    GDN_TRY(token_layout(k, 2, varlen, N, &Lk));
+    GDN_TRY(token_layout(v, 2, varlen, N, &Lv));
+    GDN_TRY(token_layout(out, 2, varlen, N, &Lo));
+    if (a->ndim != q->ndim - 1 || b->ndim != q->ndim - 1 || out->ndim != q->ndim || k->ndim != q->ndim)
+        return GDN_ERR_SHAPE;
+    GDN_TRY(token_layout(a, 1, varlen, N, &La));
+    GDN_TRY(token_layout(b, 1, varlen, N, &Lb));
+    const int64_t T_tot = Lq.T_tot;
+    if (Lk.T_tot != T_tot || Lv.T_tot != T_tot || Lo.T_tot != T_tot || La.T_tot != T_tot || Lb.T_tot != T_tot)
+        return GDN_ERR_SHAPE;
+    if (k->shape[k->ndim - 2] != H || k->shape[k->ndim - 1] != K)
+        return GDN_ERR_SHAPE;
+    if (out->shape[out->ndim - 2] != HV || out->shape[out->ndim - 1] != V)
+        return GDN_ERR_SHAPE;
+    if (a->shape[a->ndim - 1] != HV || b->shape[b->ndim - 1] != HV)
+        return GDN_ERR_SHAPE;
+    if (A_log->ndim != 1 || A_log->shape[0] != HV || dt_bias->ndim != 1 || dt_bias->shape[0] != HV)
+        return GDN_ERR_SHAPE;
+    if (state_pool->ndim != 4 || state_pool->shape[1] != HV || state_pool->shape[2] != K ||
+        state_pool->shape[3] != V)
+        return GDN_ERR_SHAPE;
+    const int64_t num_slots = state_pool->shape[0];
+    if (varlen && (cu_seqlens->ndim != 1 || cu_seqlens->shape[0] != N + 1))
+        return GDN_ERR_SHAPE;
+    if (want_inter && (inter->ndim != 4 || inter->shape[0] != T_tot || inter->shape[1] != HV ||
+                       inter->shape[2] != K || inter->shape[3] != V))
+        return GDN_ERR_SHAPE;
+    if (N > INT32_MAX || T_tot > INT32_MAX || num_slots > INT32_MAX || HV > INT32_MAX ||
+        (!varlen && Lq.T > INT32_MAX))
+        return GDN_ERR_SHAPE;
+
+    // ---- contiguity and alignment
+    if (q->stride[q->ndim - 1] != 1 || k->stride[k->ndim - 1] != 1 || v->stride[v->ndim - 1] != 1 ||
+        out->stride[out->ndim - 1] != 1)
+        return GDN_ERR_SHAPE;
+    if (state_pool->stride[3] != 1 || state_pool->stride[2] != V)
+        return GDN_ERR_SHAPE;
+    if (want_inter && (inter->stride[3] != 1 || inter->stride[2] != V))
+        return GDN_ERR_SHAPE;
+    if (state_indices->stride[0] != 1 && N > 1)
+        return GDN_ERR_SHAPE;
+    if (varlen && cu_seqlens->stride[0] != 1)
+        return GDN_ERR_SHAPE;
+    for (const gdn_tensor *t : {q, k}) {
+        if (!aligned(t->data, 16) || !stride_ok(T_tot, t == q ? Lq.tok : Lk.tok, 8) ||
+            !stride_ok(H, t->stride[t->ndim - 2], 8))
+            return GDN_ERR_ALIGN;
+    }
+    for (const gdn_tensor *t : {v, out}) {
+        if (!aligned(t->data, 8) || !stride_ok(T_tot, t == v ? Lv.tok : Lo.tok, 4) ||
+            !stride_ok(HV, t->stride[t->ndim - 2], 4))
+            return GDN_ERR_ALIGN;
+    }
+    if (!aligned(a->data, 2) || !aligned(b->data, 2) || !aligned(A_log->data, 4) || !aligned(dt_bias->data, 4) ||
+        !aligned(state_indices->data, 4) || (varlen && !aligned(cu_seqlens->data, 4)))
+        return GDN_ERR_ALIGN;
+    if (!aligned(state_pool->data, 16) || !stride_ok(num_slots, state_pool->stride[0], 4) ||
+        !stride_ok(HV, state_pool->stride[1], 4))
+        return GDN_ERR_ALIGN;
+    if (want_inter && (!aligned(inter->data, 16) || !stride_ok(T_tot, inter->stride[0], 4) ||
+                       !stride_ok(HV, inter->stride[1], 4)))
+        return GDN_ERR_ALIGN;
+    if (extra && extra->device_status && !aligned(extra->device_status, 4))
+        return GDN_ERR_ALIGN;
+
+    // ---- aliasing: nothing written may overlap anything else
+    {
+        const Span s_out = span_of(out), s_pool = span_of(state_pool), s_inter = want_inter ? span_of(inter) : Span{};
+        const gdn_tensor *inputs[] = {q, k, v, a, b, A_log, dt_bias, state_indices, cu_seqlens};
+        for (const gdn_tensor *t : inputs) {
+            if (!t)
+                continue;
+            const Span s = span_of(t);
+            if (overlap(s, s_out) || overlap(s, s_pool) || overlap(s, s_inter))
+                return GDN_ERR_ALIAS;
+        }
+        if (overlap(s_out, s_pool) || overlap(s_out, s_inter) || overlap(s_pool, s_inter))
+            return GDN_ERR_ALIAS;
+        if (extra && extra->device_status) {
+            Span st;
+            st.lo = reinterpret_cast<uintptr_t>(extra->device_status);
+            st.hi = st.lo + sizeof(uint32_t);
+            if (overlap(st, s_out) || overlap(st, s_pool) || overlap(st, s_inter))
+                return GDN_ERR_ALIAS;
+        }
+    }
+
+    // ---- supported configurations
+    if (K != kHeadK || V != kHeadV)
+        return GDN_ERR_UNSUPPORTED;
+    const int tile_v = (extra && extra->tile_v) ? extra->tile_v : 32;
+    if (tile_v != 32 && tile_v != 64 && tile_v != 128)
+        return GDN_ERR_UNSUPPORTED;
+    const int64_t units = N * HV;
+    if (units * (kHeadV / tile_v) > INT32_MAX)
+        return GDN_ERR_SHAPE;
+
+    if (N == 0 || T_tot == 0)
+        return GDN_OK;
+
+    cudaStream_t stream = extra ? static_cast<cudaStream_t>(extra->stream) : nullptr;
+    if (flags & GDN_CHECK_INDICES)
+        GDN_TRY(check_indices_on_host(static_cast<const int32_t *>(state_indices->data),
+                                      varlen ? static_cast<const int32_t *>(cu_seqlens->data) : nullptr, N,
+                                      num_slots, T_tot, stream));
+
+    // ---- parameters
+    gdn::DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.q = static_cast<const __nv_bfloat16 *>(q->data);
+    p.k = static_cast<const __nv_bfloat16 *>(k->data);
+    p.v = static_cast<const __nv_bfloat16 *>(v->data);
+    p.a = static_cast<const __nv_bfloat16 *>(a->data);
+    p.b = static_cast<const __nv_bfloat16 *>(b->data);
+    p.A_log = static_cast<const float *>(A_log->data);
+    p.dt_bias = static_cast<const float *>(dt_bias->data);
+    p.state = static_cast<float *>(state_pool->data);
+    p.indices = static_cast<const int32_t *>(state_indices->data);
+    p.cu_seqlens = varlen ? static_cast<const int32_t *>(cu_seqlens->data) : nullptr;
+    p.out = static_cast<__nv_bfloat16 *>(out->data);
+    p.inter = want_inter ? static_cast<float *>(inter->data) : nullptr;
+    p.status = extra ? extra->device_status : nullptr;
+    p.q_tok = Lq.tok;
+    p.q_head = q->stride[q->ndim - 2];
+    p.k_tok = Lk.tok;
+    p.k_head = k->stride[k->ndim - 2];
+    p.v_tok = Lv.tok;
+    p.v_head = v->stride[v->ndim - 2];
+    p.o_tok = Lo.tok;
+    p.o_head = out->stride[out->ndim - 2];
+    p.a_tok = La.tok;
+    p.a_head = a->stride[a->ndim - 1];
+    p.b_tok = Lb.tok;
+    p.b_head = b->stride[b->ndim - 1];
+    p.A_stride = A_log->stride[0];
+    p.dt_stride = dt_bias->stride[0];
+    p.s_slot = state_pool->stride[0];
+    p.s_head = state_pool->stride[1];
+    p.i_tok = want_inter ? inter->stride[0] : 0;
+    p.i_head = want_inter ? inter->stride[1] : 0;
+    p.N = static_cast<int32_t>(N);
+    p.T_fixed = varlen ? 0 : static_cast<int32_t>(Lq.T);
+    p.T_tot = static_cast<int32_t>(T_tot);
+    p.HV = static_cast<int32_t>(HV);
+    p.G = static_cast<int32_t>(HV / H);
+    p.num_slots = static_cast<int32_t>(num_slots);
+    p.scale = scale;
+    p.flags = flags;
+
+    cudaError_t err;
+    switch (tile_v) {
+    case 32: err = launch<32, 16>(p, units, stream); break;
+    case 64: err = launch<64, 16>(p, units, stream); break;
+    default: err = launch<128, 8>(p, units, stream); break;
+    }
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // extern "C"

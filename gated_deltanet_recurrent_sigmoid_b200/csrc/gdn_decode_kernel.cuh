@@ -1,0 +1,286 @@
+// gdn_decode_kernel.cuh -- sm_100a kernel of the fused sigmoid-gating Gated
+// DeltaNet decode / speculative-decode state update (the operation is
+// stated in include/gdn_decode.h).
+//
+// Work decomposition.  One CTA owns one (sequence i, value head hv, V-tile)
+// unit: a [K, BV] slab of the fp32 state S = pool[slot_i, hv].  The slab is
+// split over the CTA's threads as a (KG x VG) grid: thread (kg, vq) holds
+// rows kg*R .. kg*R+R-1 (R = K/KG) and the four columns vq*4 .. vq*4+3, i.e.
+// R float4 registers.  Each warp-wide load touches whole 128-byte rows, so
+// the state moves with 128-bit, fully coalesced loads and stores, once per
+// sequence; the slab stays in registers across all tokens of the sequence
+// (the speculative-decode path).
+//
+// Per token the two contractions over K that the update needs -- u = S^T k
+// and w = S^T q on the state before this token -- are done in ONE pass over
+// the registers, together with |k|^2, |q|^2 and k.q (for the rsqrt
+// normalisation, which is a per-token scalar and therefore commutes with the
+// sums).  Partial sums are reduced with xor-shuffles inside the warp and
+// one shared-memory exchange across warps (one __syncthreads per token,
+// double-buffered by token parity).  Then, with decay = exp(g):
+//     delta = beta * (v - decay * u * rk)                (S^T k^ on the decayed S)
+//     o     = decay * w * qs + (k^ . q^) * delta         (= S'^T q^ after the update)
+//     S'    = decay * S + k^ delta^T
+// which is the update of the header rearranged so that S is read once.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gdn_decode.h"
+
+namespace gdn {
+
+struct DecodeParams {
+    const __nv_bfloat16 *q, *k, *v, *a, *b;
+    const float *A_log, *dt_bias;
+    float *state;
+    const int32_t *indices;
+    const int32_t *cu_seqlens;  // nullptr: fixed length T_fixed
+    __nv_bfloat16 *out;
+    float *inter;               // nullptr unless GDN_WRITE_INTERMEDIATE
+    uint32_t *status;           // nullptr: device errors are not reported
+    // strides in elements
+    int64_t q_tok, q_head, k_tok, k_head, v_tok, v_head;
+    int64_t a_tok, a_head, b_tok, b_head, o_tok, o_head;
+    int64_t A_stride, dt_stride;
+    int64_t s_slot, s_head, i_tok, i_head;
+    int32_t N, T_fixed, T_tot, HV, G, num_slots;
+    float scale;
+    uint32_t flags;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 u, float *f)
+{
+    f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
+    f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+    f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z);
+    f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ float load_bf16(const __nv_bfloat16 *p)
+{
+    const unsigned short bits = __ldg(reinterpret_cast<const unsigned short *>(p));
+    return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return l | (h << 16);
+}
+
+__device__ __forceinline__ void report(uint32_t *status, uint32_t bit)
+{
+    if (status)
+        atomicOr(status, bit);
+}
+
+template <int K, int V, int BV, int KG>
+struct TileShape {
+    static constexpr int VG = BV / 4;            // threads across the tile's columns
+    static constexpr int THREADS = VG * KG;
+    static constexpr int WARPS = THREADS / 32;
+    static constexpr int R = K / KG;             // state rows per thread
+    static constexpr int NV = V / BV;            // V-tiles per head
+    static constexpr int XW = 2 * BV + 4;        // exchange floats per warp: u, w, |k|^2, |q|^2, k.q
+    static_assert(BV % 4 == 0 && V % BV == 0, "V must split into BV-wide tiles");
+    static_assert(VG <= 32 && 32 % VG == 0, "a warp must hold whole k-groups");
+    static_assert(THREADS % 32 == 0 && THREADS <= 1024, "whole warps");
+    static_assert(K % KG == 0 && R % 8 == 0, "q/k rows are loaded 8 bf16 (16 bytes) at a time");
+};
+
+template <int K, int V, int BV, int KG>
+__global__ void __launch_bounds__(TileShape<K, V, BV, KG>::THREADS)
+gdn_decode_kernel(const __grid_constant__ DecodeParams p)
+{
+    using TS = TileShape<K, V, BV, KG>;
+    constexpr int VG = TS::VG, WARPS = TS::WARPS, R = TS::R, NV = TS::NV, XW = TS::XW;
+
+    __shared__ __align__(16) float xch[2][WARPS][XW];
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int vq = tid % VG;
+    const int kg = tid / VG;
+    const int row0 = kg * R;
+
+    int unit = blockIdx.x;
+    const int vt = unit % NV;
+    unit /= NV;
+    const int hv = unit % p.HV;
+    const int i = unit / p.HV;
+    const int col0 = vt * BV + vq * 4;
+
+    // ---- token range and slot of sequence i -------------------------
+    int64_t bos;
+    int len;
+    if (p.cu_seqlens) {
+        const int b0 = __ldg(p.cu_seqlens + i);
+        const int e0 = __ldg(p.cu_seqlens + i + 1);
+        if (b0 < 0 || e0 < b0 || e0 > p.T_tot) {
+            if (tid == 0)
+                report(p.status, GDN_DEV_BAD_SEQLENS);
+            return;
+        }
+        bos = b0;
+        len = e0 - b0;
+    } else {
+        bos = static_cast<int64_t>(i) * p.T_fixed;
+        len = p.T_fixed;
+    }
+    const int slot = __ldg(p.indices + i);
+    if (slot < -1 || slot >= p.num_slots) {
+        if (tid == 0)
+            report(p.status, GDN_DEV_BAD_SLOT);
+        return;
+    }
+    if (slot < 0) {
+        // Padded sequence: zero output rows of this tile, no state access.
+        if (kg == 0)
+            for (int t = 0; t < len; ++t)
+                *reinterpret_cast<uint2 *>(p.out + (bos + t) * p.o_tok + hv * p.o_head + col0) =
+                    make_uint2(0u, 0u);
+        return;
+    }
+    if (len == 0)
+        return;
+
+    // ---- state slab -> registers (128-bit, streamed once) ------------
+    float *const s_ptr = p.state + static_cast<int64_t>(slot) * p.s_slot + hv * p.s_head +
+                         static_cast<int64_t>(row0) * V + col0;
+    float4 s[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j)
+        s[j] = __ldcs(reinterpret_cast<const float4 *>(s_ptr + j * V));
+
+    const int h = hv / p.G;
+    const float neg_A = -expf(__ldg(p.A_log + hv * p.A_stride));
+    const float dt_b = __ldg(p.dt_bias + hv * p.dt_stride);
+    const bool l2norm = (p.flags & GDN_L2NORM_QK) != 0;
+    const bool write_inter = (p.flags & GDN_WRITE_INTERMEDIATE) != 0;
+
+    for (int t = 0; t < len; ++t) {
+        const int64_t tok = bos + t;
+
+        // ---- inputs: this thread's R rows of q and k, 4 columns of v
+        float kr[R], qr[R];
+        const uint4 *kp = reinterpret_cast<const uint4 *>(p.k + tok * p.k_tok + h * p.k_head + row0);
+        const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + tok * p.q_tok + h * p.q_head + row0);
+#pragma unroll
+        for (int c = 0; c < R / 8; ++c) {
+            unpack8(__ldg(kp + c), kr + 8 * c);
+            unpack8(__ldg(qp + c), qr + 8 * c);
+        }
+        const uint2 v_raw = __ldg(reinterpret_cast<const uint2 *>(p.v + tok * p.v_tok + hv * p.v_head + col0));
+        const float a_t = load_bf16(p.a + tok * p.a_tok + hv * p.a_head);
+        const float b_t = load_bf16(p.b + tok * p.b_tok + hv * p.b_head);
+
+        // ---- partial S^T k, S^T q, |k|^2, |q|^2, k.q over my rows ----
+        float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
+        float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f;
+        float skk = 0.f, sqq = 0.f, skq = 0.f;
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            u0 = fmaf(s[j].x, kr[j], u0); u1 = fmaf(s[j].y, kr[j], u1);
+            u2 = fmaf(s[j].z, kr[j], u2); u3 = fmaf(s[j].w, kr[j], u3);
+            w0 = fmaf(s[j].x, qr[j], w0); w1 = fmaf(s[j].y, qr[j], w1);
+            w2 = fmaf(s[j].z, qr[j], w2); w3 = fmaf(s[j].w, qr[j], w3);
+            skk = fmaf(kr[j], kr[j], skk);
+            sqq = fmaf(qr[j], qr[j], sqq);
+            skq = fmaf(kr[j], qr[j], skq);
+        }
+        // lanes that differ only in their k-group hold the same columns
+#pragma unroll
+        for (int off = VG; off < 32; off <<= 1) {
+            u0 += __shfl_xor_sync(0xffffffffu, u0, off); u1 += __shfl_xor_sync(0xffffffffu, u1, off);
+            u2 += __shfl_xor_sync(0xffffffffu, u2, off); u3 += __shfl_xor_sync(0xffffffffu, u3, off);
+            w0 += __shfl_xor_sync(0xffffffffu, w0, off); w1 += __shfl_xor_sync(0xffffffffu, w1, off);
+            w2 += __shfl_xor_sync(0xffffffffu, w2, off); w3 += __shfl_xor_sync(0xffffffffu, w3, off);
+            skk += __shfl_xor_sync(0xffffffffu, skk, off);
+            sqq += __shfl_xor_sync(0xffffffffu, sqq, off);
+            skq += __shfl_xor_sync(0xffffffffu, skq, off);
+        }
+        const int buf = t & 1;
+        if (lane < VG) {
+            *reinterpret_cast<float4 *>(&xch[buf][warp][vq * 4]) = make_float4(u0, u1, u2, u3);
+            *reinterpret_cast<float4 *>(&xch[buf][warp][BV + vq * 4]) = make_float4(w0, w1, w2, w3);
+            if (lane == 0) {
+                xch[buf][warp][2 * BV + 0] = skk;
+                xch[buf][warp][2 * BV + 1] = sqq;
+                xch[buf][warp][2 * BV + 2] = skq;
+            }
+        }
+        __syncthreads();
+        float4 U = make_float4(0.f, 0.f, 0.f, 0.f), W = U;
+        float SKK = 0.f, SQQ = 0.f, SKQ = 0.f;
+#pragma unroll
+        for (int wi = 0; wi < WARPS; ++wi) {
+            const float4 uu = *reinterpret_cast<const float4 *>(&xch[buf][wi][vq * 4]);
+            const float4 ww = *reinterpret_cast<const float4 *>(&xch[buf][wi][BV + vq * 4]);
+            U.x += uu.x; U.y += uu.y; U.z += uu.z; U.w += uu.w;
+            W.x += ww.x; W.y += ww.y; W.z += ww.z; W.w += ww.w;
+            SKK += xch[buf][wi][2 * BV + 0];
+            SQQ += xch[buf][wi][2 * BV + 1];
+            SKQ += xch[buf][wi][2 * BV + 2];
+        }
+
+        // ---- gates and norms (scalars, computed by every thread) ----
+        const float rk = l2norm ? rsqrtf(SKK + 1e-6f) : 1.f;
+        const float qs = (l2norm ? rsqrtf(SQQ + 1e-6f) : 1.f) * p.scale;
+        const float x = a_t + dt_b;
+        const float sp = x > 20.f ? x : log1pf(expf(x));
+        const float decay = expf(neg_A * sp);
+        const float beta = 1.f / (1.f + expf(-b_t));
+        const float kq = SKQ * rk * qs;
+
+        // ---- delta and output ----------------------------------
+        const float dku = decay * rk;
+        const float dwq = decay * qs;
+        const float d0 = beta * (bf16_lo(v_raw.x) - dku * U.x);
+        const float d1 = beta * (bf16_hi(v_raw.x) - dku * U.y);
+        const float d2 = beta * (bf16_lo(v_raw.y) - dku * U.z);
+        const float d3 = beta * (bf16_hi(v_raw.y) - dku * U.w);
+
+        // ---- S <- decay S + k^ delta^T -----------------------------
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            const float kh = kr[j] * rk;
+            s[j].x = fmaf(kh, d0, decay * s[j].x);
+            s[j].y = fmaf(kh, d1, decay * s[j].y);
+            s[j].z = fmaf(kh, d2, decay * s[j].z);
+            s[j].w = fmaf(kh, d3, decay * s[j].w);
+        }
+
+        if (kg == 0) {
+            const float o0 = fmaf(kq, d0, dwq * W.x);
+            const float o1 = fmaf(kq, d1, dwq * W.y);
+            const float o2 = fmaf(kq, d2, dwq * W.z);
+            const float o3 = fmaf(kq, d3, dwq * W.w);
+            *reinterpret_cast<uint2 *>(p.out + tok * p.o_tok + hv * p.o_head + col0) =
+                make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        }
+
+        // ---- optional per-token state ------------------------------
+        if (write_inter) {
+            float *ip = p.inter + tok * p.i_tok + hv * p.i_head + static_cast<int64_t>(row0) * V + col0;
+#pragma unroll
+            for (int j = 0; j < R; ++j)
+                __stcs(reinterpret_cast<float4 *>(ip + j * V), s[j]);
+        }
+    }
+
+    // ---- write the slab back in place ------------------------------
+    if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
+#pragma unroll
+        for (int j = 0; j < R; ++j)
+            __stcs(reinterpret_cast<float4 *>(s_ptr + j * V), s[j]);
+    }
+}
+
+}  // namespace gdn

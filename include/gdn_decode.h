@@ -1,0 +1,158 @@
+/*
+ * gdn_decode.h -- C ABI of the B200 (sm_100a) fused sigmoid-gating Gated
+ * DeltaNet decode / speculative-decode state update.
+ *
+ * The operation (the pages' fused_sigmoid_gating_delta_rule_update):
+ *   "[Qwen3Next] Optimize fused_sigmoid_gating_delta_rule_update_kernel"
+ *   (sglang PR 18271, Motivation, Highlights) and the vLLM PR 35777 summary
+ *   (sections 执行摘要 and 实现拆解) describe one kernel that replaces
+ *   fused_gdn_gating + fused_recurrent_gated_delta_rule, takes A_log, a, b
+ *   and dt_bias, normalises q/k with rsqrt and serves both the single-token
+ *   and the speculative (several tokens per sequence) decode paths.  For
+ *   every sequence i, value head hv and token t of that sequence:
+ *
+ *     g     = -exp(A_log[hv]) * softplus(a[t,hv] + dt_bias[hv])
+ *     beta  = sigmoid(b[t,hv])
+ *     k^    = k[t,h] * rsqrt(|k[t,h]|^2 + 1e-6)               (GDN_L2NORM_QK)
+ *     q^    = scale * q[t,h] * rsqrt(|q[t,h]|^2 + 1e-6)
+ *     S     <- exp(g) * S                                    (S: fp32 [K, V])
+ *     S     <- S + k^ (beta * (v[t,hv] - S^T k^))^T
+ *     out[t,hv] = S^T q^                                     (rounded to bf16)
+ *
+ *   with h = hv / (HV / H): value heads are grouped contiguously under key
+ *   heads (the `ba` reshape to (num_k_heads, 2*num_v_heads/num_k_heads) in
+ *   the vLLM PR 37975 report, 实现拆解).  S is read once per sequence from
+ *   state_pool[state_indices[i], hv], carried on chip across the sequence's
+ *   tokens and written back in place.  A state index of -1 marks a padded
+ *   sequence: its output rows are written as zeros and no state is touched.
+ *   softplus(x) returns x for x > 20.
+ *
+ * Tensor descriptors.  Every tensor is passed as a gdn_tensor: a DEVICE
+ * pointer, a dtype code, a rank (1..4), a shape and strides in ELEMENTS.
+ * The caller owns all memory; the library allocates no device memory and
+ * keeps no pointer after the call returns.  Strides must be >= 0.
+ *
+ *   argument        dtype  shape                                  layout rules
+ *   q, k            bf16   [T_tot, H, K] | [1, T_tot, H, K]       K contiguous; token and
+ *                          (varlen) or [N, T, H, K] (fixed T)     head strides % 8 == 0;
+ *                                                                 data 16-byte aligned
+ *   v, out          bf16   same leading dims, [.., HV, V]         V contiguous; strides % 4
+ *                                                                 == 0; data 8-byte aligned
+ *   a, b            bf16   [T_tot, HV] | [1, T_tot, HV] | [N,T,HV] any strides (packed `ba`
+ *                                                                 projections are fine)
+ *   A_log, dt_bias  fp32   [HV]                                   any stride
+ *   state_pool      fp32   [num_slots, HV, K, V]                  K, V contiguous (strides
+ *                                                                 V, 1); slot/head strides
+ *                                                                 % 4 == 0; 16-byte aligned
+ *   state_indices   int32  [N]                                    contiguous
+ *   cu_seqlens      int32  [N + 1] or NULL                        contiguous; NULL = every
+ *                                                                 sequence has T tokens
+ *   intermediate_   fp32   [T_tot, HV, K, V]                      as state_pool
+ *     states (extra)
+ *
+ * With fixed T (cu_seqlens NULL) the leading [N, T] dims of q, k, v, a, b
+ * and out must flatten to a single token dimension (stride[0] ==
+ * T * stride[1] when N > 1 and T > 1).  Supported head sizes: K = V = 128.
+ *
+ * Ownership and aliasing.  state_pool is read and written in place (only
+ * the slots named by state_indices); out and intermediate_states are
+ * written; every other tensor is read only.  No written tensor may overlap
+ * any other tensor.  The non-negative entries of state_indices must be
+ * distinct (GDN_CHECK_INDICES verifies it on the host).
+ *
+ * Errors.  The call returns GDN_OK or a negative gdn_status.  Every argument
+ * check happens on the host before anything is enqueued; on any error
+ * nothing is launched and no memory is touched.  The call is asynchronous
+ * on extra->stream (NULL: the legacy default stream).  N = 0 or T_tot = 0 is
+ * GDN_OK with no launch.  Problems only the device can see (a slot index
+ * < -1 or >= num_slots, cu_seqlens not monotone or past T_tot) are reported
+ * by OR-ing GDN_DEV_* bits into *extra->device_status (when given); the
+ * offending sequence is skipped whole and nothing traps.
+ */
+#ifndef GDN_DECODE_H
+#define GDN_DECODE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_DECODE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+/* dtype codes */
+#define GDN_DTYPE_BF16 1
+#define GDN_DTYPE_F32  2
+#define GDN_DTYPE_I32  3
+
+/* flags */
+#define GDN_L2NORM_QK          (1u << 0) /* L2-normalise q and k (default on) */
+#define GDN_WRITE_INTERMEDIATE (1u << 1) /* store S after every token */
+#define GDN_NO_FINAL_WRITEBACK (1u << 2) /* leave state_pool untouched */
+#define GDN_CHECK_INDICES      (1u << 3) /* host check of indices / cu_seqlens
+                                            (copies them to the host and
+                                            synchronises extra->stream) */
+
+/* status codes returned by the host call */
+#define GDN_OK               0
+#define GDN_ERR_NULL_ARG    (-1) /* a required pointer or descriptor is NULL */
+#define GDN_ERR_DTYPE       (-2) /* wrong dtype code */
+#define GDN_ERR_SHAPE       (-3) /* wrong rank, shape or inconsistent sizes */
+#define GDN_ERR_ALIGN       (-4) /* pointer or stride breaks an alignment rule */
+#define GDN_ERR_ALIAS       (-5) /* a written tensor overlaps another tensor */
+#define GDN_ERR_UNSUPPORTED (-6) /* head size or tile not built */
+#define GDN_ERR_ARG         (-7) /* bad scalar: scale <= 0 or not finite, unknown flag */
+#define GDN_ERR_INDICES     (-8) /* GDN_CHECK_INDICES found a bad or repeated slot,
+                                    or bad cu_seqlens */
+#define GDN_ERR_CUDA        (-9) /* the CUDA runtime refused the launch or copy */
+
+/* bits OR-ed into *device_status by the kernel */
+#define GDN_DEV_BAD_SLOT    1u
+#define GDN_DEV_BAD_SEQLENS 2u
+
+typedef struct gdn_tensor {
+    void *data;          /* device pointer */
+    int32_t dtype;       /* GDN_DTYPE_* */
+    int32_t ndim;        /* 1..4 */
+    int64_t shape[4];
+    int64_t stride[4];   /* in elements */
+} gdn_tensor;
+
+typedef struct gdn_extra {
+    void *stream;                          /* cudaStream_t; NULL = legacy default */
+    const gdn_tensor *intermediate_states; /* required with GDN_WRITE_INTERMEDIATE */
+    uint32_t *device_status;               /* device word for GDN_DEV_* bits, or NULL */
+    int32_t tile_v;                        /* 0 = library choice, else V-tile width */
+    int32_t reserved;                      /* must be 0 */
+} gdn_extra;
+
+/*
+ * One fused decode / speculative-decode update (see the top of this file).
+ * The first eleven arguments follow the pages' parameter order; `scale` is
+ * normally 1/sqrt(K); `extra` may be NULL (default stream, no intermediate
+ * states, no status word, library tile choice).
+ */
+GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                      const gdn_tensor *a, const gdn_tensor *b,
+                      const gdn_tensor *A_log, const gdn_tensor *dt_bias,
+                      const gdn_tensor *state_pool, const gdn_tensor *state_indices,
+                      const gdn_tensor *cu_seqlens, const gdn_tensor *out,
+                      float scale, uint32_t flags, const gdn_extra *extra);
+
+/* Static text for a gdn_status value (never NULL). */
+GDN_API const char *gdn_status_string(int status);
+
+/* GDN_DECODE_ABI_VERSION of the loaded library. */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_DECODE_H */

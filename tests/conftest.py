@@ -19,3 +19,12 @@ def oracle_lib():
     import oracle
     oracle._load()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def gdn_lib():
+    """Build the CUDA library if its sources are newer (nvcc cross-compiles
+    without a GPU) and load it through the binding."""
+    from gated_deltanet_recurrent_sigmoid_b200 import binding, build
+    build.build()
+    return binding.load()

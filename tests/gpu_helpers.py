@@ -1,0 +1,107 @@
+"""Helpers for the GPU parity tests: move a workload to the device, run the
+CUDA path through the C ABI, run the oracle on the same inputs (whole or on a
+sample of sequences), and compare with the stated tolerances.
+
+Tolerances (fixed for this path): state max |S_gpu - S_ref| <= 1e-4;
+output |o - o_ref| <= 1e-2 + 1e-2 |o_ref|; slots and indices bit-exact.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from gated_deltanet_recurrent_sigmoid_b200 import binding
+from gated_deltanet_recurrent_sigmoid_b200.workloads import Workload, bf16_bits_to_f32
+
+STATE_ATOL = 1e-4
+OUT_ATOL = 1e-2
+OUT_RTOL = 1e-2
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def to_device(w: Workload, device="cuda") -> dict:
+    d = dict(q=bf16_tensor(w.q, device), k=bf16_tensor(w.k, device), v=bf16_tensor(w.v, device),
+             a=bf16_tensor(w.a, device), b=bf16_tensor(w.b, device),
+             A_log=torch.from_numpy(w.A_log).to(device), dt_bias=torch.from_numpy(w.dt_bias).to(device),
+             state_pool=torch.from_numpy(w.state_pool).to(device),
+             state_indices=torch.from_numpy(w.state_indices).to(device),
+             cu_seqlens=None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).to(device))
+    d["out"] = torch.full(w.v.shape, float("nan"), dtype=torch.bfloat16, device=device)
+    return d
+
+
+def run_gpu(w: Workload, flags=binding.L2NORM_QK, inter=False, tile_v=0, d=None, scale=None):
+    """Run the CUDA path once; returns (device dict, status word, inter tensor)."""
+    d = d or to_device(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    inter_t = None
+    if inter:
+        inter_t = torch.full((w.T_tot, w.spec.HV, w.spec.K, w.spec.V), float("nan"), device="cuda")
+    binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"],
+                          d["state_indices"], d["cu_seqlens"], d["out"], scale=scale, flags=flags,
+                          intermediate_states=inter_t, device_status=status, tile_v=tile_v)
+    torch.cuda.synchronize()
+    return d, int(status.item()), inter_t
+
+
+def run_oracle(w: Workload, flags=oracle.L2NORM_QK, scale=None):
+    return oracle.update(w.q, w.k, w.v, w.a, w.b, w.A_log, w.dt_bias, w.state_pool, w.state_indices,
+                         w.cu_seqlens, scale=scale, flags=flags)
+
+
+def token_rows(w: Workload, seqs) -> np.ndarray:
+    lens = w.seq_lens
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    return np.concatenate([np.arange(starts[i], starts[i] + lens[i]) for i in seqs]).astype(np.int64) \
+        if len(seqs) else np.zeros(0, np.int64)
+
+
+def sample_subproblem(w: Workload, seqs):
+    """The oracle's inputs for a subset of sequences (sequences are
+    independent, so the subset's results are exactly those of the full call).
+    Returns (arrays, token rows in the full problem, slots in the full pool)."""
+    seqs = np.asarray(seqs)
+    rows = token_rows(w, seqs)
+    flat = lambda x, tail: x.reshape((-1,) + x.shape[-tail:])[rows]
+    slots = w.state_indices[seqs]
+    live = slots >= 0
+    sub_pool = w.state_pool[slots[live]]
+    new_idx = np.full(len(seqs), -1, dtype=np.int32)
+    new_idx[live] = np.arange(live.sum(), dtype=np.int32)
+    lens = w.seq_lens[seqs]
+    cu = np.zeros(len(seqs) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    arrays = dict(q=flat(w.q, 2), k=flat(w.k, 2), v=flat(w.v, 2), a=flat(w.a, 1), b=flat(w.b, 1),
+                  A_log=w.A_log, dt_bias=w.dt_bias, state_pool=np.ascontiguousarray(sub_pool),
+                  state_indices=new_idx, cu_seqlens=cu)
+    return arrays, rows, slots
+
+
+def oracle_on(arrays, flags=oracle.L2NORM_QK, scale=None):
+    return oracle.update(arrays["q"], arrays["k"], arrays["v"], arrays["a"], arrays["b"], arrays["A_log"],
+                         arrays["dt_bias"], arrays["state_pool"], arrays["state_indices"], arrays["cu_seqlens"],
+                         scale=scale, flags=flags)
+
+
+def out_as_f32(out: torch.Tensor) -> np.ndarray:
+    return out.float().cpu().numpy()
+
+
+def assert_out_close(o_gpu: np.ndarray, o_ref: np.ndarray, what="out"):
+    o_gpu = o_gpu.reshape(o_ref.shape).astype(np.float64)
+    nan_ref = np.isnan(o_ref)
+    assert np.array_equal(np.isnan(o_gpu), nan_ref), f"{what}: written rows differ"
+    err = np.abs(o_gpu - o_ref)[~nan_ref]
+    bound = (OUT_ATOL + OUT_RTOL * np.abs(o_ref))[~nan_ref]
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} elements out of tolerance, worst {err.max():.3e}"
+
+
+def assert_state_close(s_gpu: np.ndarray, s_ref: np.ndarray, what="state"):
+    err = np.abs(s_gpu.astype(np.float64) - s_ref)
+    assert np.isfinite(s_gpu).all(), f"{what}: non-finite values"
+    assert err.max() <= STATE_ATOL, f"{what}: max abs err {err.max():.3e} > {STATE_ATOL}"

@@ -1,0 +1,153 @@
+"""The C-ABI library on the CPU: it loads, exports every declared symbol,
+and its host-side validation rejects bad arguments before any CUDA call.
+
+These tests never launch a kernel: every call below either fails a host
+check or has nothing to do (N = 0), so no GPU is needed.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from gated_deltanet_recurrent_sigmoid_b200 import binding, build
+
+HEADER = os.path.join(build.INCLUDE, "gdn_decode.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)
+
+
+def test_header_declares_the_abi():
+    assert set(declared_functions()) == {"gdn_decode_update", "gdn_status_string", "gdn_version"}
+
+
+def test_library_exports_every_declared_symbol(gdn_lib):
+    nm = subprocess.run(["nm", "-D", "--defined-only", build.LIB_PATH], capture_output=True, text=True,
+                        check=True).stdout
+    exported = {line.split()[-1] for line in nm.splitlines() if " T " in line}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(gdn_lib, name)
+    # nothing else leaks out of the library
+    assert {e for e in exported if e.startswith("gdn")} == set(declared_functions())
+
+
+def test_version_matches_header(gdn_lib):
+    m = re.search(r"#define GDN_DECODE_ABI_VERSION (\d+)", open(HEADER).read())
+    assert gdn_lib.gdn_version() == int(m.group(1))
+
+
+def test_status_strings(gdn_lib):
+    for code in range(0, -10, -1):
+        s = binding.status_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in binding.status_string(-100)
+
+
+def test_header_constants_match_binding():
+    text = open(HEADER).read()
+    def define(name):
+        m = re.search(rf"#define {name}\s+\(?(-?\d+)(u << (\d+))?\)?", text)
+        return int(m.group(1)) << int(m.group(3)) if m.group(3) else int(m.group(1))
+    assert define("GDN_L2NORM_QK") == binding.L2NORM_QK
+    assert define("GDN_WRITE_INTERMEDIATE") == binding.WRITE_INTERMEDIATE
+    assert define("GDN_NO_FINAL_WRITEBACK") == binding.NO_FINAL_WRITEBACK
+    assert define("GDN_CHECK_INDICES") == binding.CHECK_INDICES
+    for name, val in [("GDN_ERR_NULL_ARG", -1), ("GDN_ERR_DTYPE", -2), ("GDN_ERR_SHAPE", -3),
+                      ("GDN_ERR_ALIGN", -4), ("GDN_ERR_ALIAS", -5), ("GDN_ERR_UNSUPPORTED", -6),
+                      ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9)]:
+        assert int(re.search(rf"#define {name}\s+\((-?\d+)\)", text).group(1)) == val
+    assert ctypes.sizeof(binding.GdnTensor) == 8 + 4 + 4 + 8 * 4 + 8 * 4
+    assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 + 4
+
+
+def make(N=4, T=1, H=2, HV=4, K=128, V=128, slots=8, varlen=True):
+    """CPU tensors shaped like a valid call (host pointers are fine for the
+    host checks; the library never dereferences them before launching)."""
+    bf = torch.bfloat16
+    lead = (N * T,) if varlen else (N, T)
+    t = dict(q=torch.zeros(*lead, H, K, dtype=bf), k=torch.zeros(*lead, H, K, dtype=bf),
+             v=torch.zeros(*lead, HV, V, dtype=bf), a=torch.zeros(*lead, HV, dtype=bf),
+             b=torch.zeros(*lead, HV, dtype=bf), A_log=torch.zeros(HV), dt_bias=torch.zeros(HV),
+             state_pool=torch.zeros(slots, HV, K, V), state_indices=torch.arange(N, dtype=torch.int32),
+             cu_seqlens=torch.arange(0, N * T + 1, T, dtype=torch.int32) if varlen else None,
+             out=torch.zeros(*lead, HV, V, dtype=bf))
+    return t
+
+
+def call(t, **kw):
+    return binding.decode_update(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"],
+                                 t["state_pool"], t["state_indices"], t["cu_seqlens"], t["out"],
+                                 stream=None, **kw)
+
+
+def expect(code, t, **kw):
+    with pytest.raises(binding.GdnError) as e:
+        call(t, **kw)
+    assert e.value.status == code, binding.status_string(e.value.status)
+
+
+def test_empty_batch_is_ok_without_launch(gdn_lib):
+    t = make(N=0)
+    assert call(t) is t["out"]
+    t = make(N=3, T=0, varlen=False)
+    call(t)
+
+
+def test_rejects_bad_dtypes_and_shapes(gdn_lib):
+    t = make(); t["q"] = t["q"].float(); expect(binding.ERR_DTYPE, t)
+    t = make(); t["state_pool"] = t["state_pool"].double(); expect(binding.ERR_DTYPE, t)
+    t = make(); t["state_indices"] = t["state_indices"].long(); expect(binding.ERR_DTYPE, t)
+    t = make(); t["v"] = t["v"][:, :3]; expect(binding.ERR_SHAPE, t)            # HV mismatch with out
+    t = make(HV=3); expect(binding.ERR_SHAPE, t)                                  # HV % H != 0
+    t = make(); t["cu_seqlens"] = t["cu_seqlens"][:-1]; expect(binding.ERR_SHAPE, t)
+    t = make(); t["A_log"] = torch.zeros(3); expect(binding.ERR_SHAPE, t)
+    t = make(); t["state_pool"] = t["state_pool"].transpose(2, 3); expect(binding.ERR_SHAPE, t)
+    t = make(varlen=False, T=2); t["q"] = t["q"][:, :, :, :64]; expect(binding.ERR_SHAPE, t)
+
+
+def test_rejects_unsupported_head_size(gdn_lib):
+    expect(binding.ERR_UNSUPPORTED, make(K=64, V=64))
+    expect(binding.ERR_UNSUPPORTED, make(), tile_v=16)
+
+
+def test_rejects_misalignment(gdn_lib):
+    t = make()
+    raw = torch.zeros(t["q"].numel() + 8, dtype=torch.bfloat16)
+    t["q"] = raw[1:1 + t["q"].numel()].view(t["q"].shape)                         # 2-byte offset
+    expect(binding.ERR_ALIGN, t)
+    t = make()
+    raw = torch.zeros(t["state_pool"].numel() + 4)
+    t["state_pool"] = raw[1:1 + t["state_pool"].numel()].view(t["state_pool"].shape)
+    expect(binding.ERR_ALIGN, t)
+
+
+def test_rejects_aliasing(gdn_lib):
+    t = make(); t["out"] = t["v"]; expect(binding.ERR_ALIAS, t)
+    t = make(); t["A_log"] = t["state_pool"].view(-1)[:4]; expect(binding.ERR_ALIAS, t)
+    t = make(); buf = torch.zeros(2 * t["out"].numel(), dtype=torch.bfloat16)
+    t["out"] = buf[: t["out"].numel()].view(t["out"].shape)
+    t["v"] = buf[t["out"].numel() // 2:][: t["v"].numel()].view(t["v"].shape)   # half overlap
+    expect(binding.ERR_ALIAS, t)
+
+
+def test_rejects_bad_scalars_and_flags(gdn_lib):
+    expect(binding.ERR_ARG, make(), scale=0.0)
+    expect(binding.ERR_ARG, make(), scale=float("nan"))
+    expect(binding.ERR_ARG, make(), flags=1 << 7)
+
+
+def test_intermediate_required_with_flag(gdn_lib):
+    expect(binding.ERR_NULL_ARG, make(), flags=binding.L2NORM_QK | binding.WRITE_INTERMEDIATE)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(binding, "_LIB", None)
+    monkeypatch.setattr(build, "LIB_PATH", "/nonexistent/libgdn_decode.so")
+    with pytest.raises(binding.GdnError):
+        binding.load()
