@@ -225,7 +225,7 @@ def test_guard_bands_untouched():
     w = wl.generate(spec)
     ref, _, iref = run_gpu(w, flags=L2 | INTER, inter=True)
     d = to_device(w)
-    sentinel = -12345.0
+    sentinel = -1024.0          # exact in bf16 and fp32
     S, HV = spec.num_slots, spec.HV
     pool_buf = torch.full((S + 2, HV, 128, 128), sentinel, device="cuda")
     pool_buf[1:-1] = d["state_pool"]
