@@ -47,7 +47,8 @@ ROTATING_COPIES = 4
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"kernel_sha256": "b4c54bba8390bf24727314370b03fe02fd473850fb91495c81cec9ef9267daa1",
+               "bytes_per_launch": 257369600 + 198541824}
 
 
 def kernel_source_hash() -> str:
@@ -204,6 +205,17 @@ def run_reference(args, w):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def kernel_name(schedule, tile_v, tile_rows, one_token):
+    """Name of the kernel the library launches for these settings (mirrors
+    the library's documented choice)."""
+    from gated_deltanet_recurrent_sigmoid_b200 import binding
+    if schedule == binding.SCHEDULE_PIPELINED:
+        return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
+    bv = tile_v or (64 if one_token else 16)
+    rows = tile_rows or (32 if bv == 64 and one_token else 16)
+    return f"gdn::gdn_decode_kernel<128,128,{bv},{128 // rows}>"
+
+
 def workload_config(w, world):
     s = w.spec
     return {"workload": s.name, "B": s.N, "T": s.T if s.T is not None else "U{1..64}", "H": s.H, "HV": s.HV,
@@ -235,6 +247,8 @@ def main():
     ap.add_argument("--workload", default=wl.DECODE_B512.name, choices=sorted(wl.BY_NAME))
     ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
     ap.add_argument("--tile-v", type=int, default=0)
+    ap.add_argument("--tile-rows", type=int, default=0)
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -266,12 +280,15 @@ def main():
         dist.barrier()
     binding.load()
 
+    schedule = {"auto": binding.SCHEDULE_AUTO, "per_tile": binding.SCHEDULE_PER_TILE,
+                "pipelined": binding.SCHEDULE_PIPELINED}[args.schedule]
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
     calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"], c["state_pool"],
                                   c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
-                                  intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v)
+                                  intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
+                                  schedule=schedule, tile_rows=args.tile_rows)
              for c in copies]
     nbytes = wl.algorithmic_bytes(w)
     torch.cuda.synchronize(device)
@@ -281,9 +298,9 @@ def main():
         calls[s % len(calls)]()
     stream.synchronize()
 
-    # timed region: K steps, one fused kernel each, events on the launch stream
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # timed region: K steps, one fused kernel each, back to back on the launch
+    # stream, bracketed by CUDA events on that stream (the region holds only
+    # this kernel, so its average launch duration is the region time / K)
     region0 = torch.cuda.Event(enable_timing=True)
     region1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -293,17 +310,14 @@ def main():
     time.sleep(0.2)
     region0.record(stream)
     for s in range(args.steps):
-        starts[s].record(stream)
         calls[s % len(calls)]()
-        ends[s].record(stream)
     region1.record(stream)
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     region_ms = region0.elapsed_time(region1)
-    kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    avg_kernel_ms = sum(kernel_ms) / len(kernel_ms)
+    avg_kernel_ms = region_ms / args.steps
 
     t = torch.tensor([region_ms], dtype=torch.float64, device=device)
     if world > 1:
@@ -324,7 +338,8 @@ def main():
         h2d = sum(host[n].numel() * host[n].element_size() for n in host if n != "out")
         d2h = host["out"].numel() * host["out"].element_size()
         for _ in range(3):
-            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v)
+            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v,
+                                       schedule=schedule, tile_rows=args.tile_rows)
             stream.synchronize()
         if world > 1:
             dist.barrier()
@@ -332,7 +347,8 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
-            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v)
+            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v,
+                                       schedule=schedule, tile_rows=args.tile_rows)
             stream.synchronize()          # the step ends when the host holds the output
         e1.record(stream)
         torch.cuda.synchronize(device)
@@ -360,7 +376,8 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
-                         "kernel": "gdn::gdn_decode_kernel"},
+                         "kernel": kernel_name(schedule, args.tile_v, args.tile_rows,
+                                               w.T_tot == w.spec.N and not w.spec.intermediate)},
             "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clocks,

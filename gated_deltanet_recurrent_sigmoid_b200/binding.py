@@ -24,6 +24,11 @@ CHECK_INDICES = 1 << 3
 
 DEV_BAD_SLOT = 1
 DEV_BAD_SEQLENS = 2
+DEV_TIMEOUT = 4
+
+SCHEDULE_AUTO = 0
+SCHEDULE_PER_TILE = 1
+SCHEDULE_PIPELINED = 2
 
 OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5
@@ -48,7 +53,7 @@ class GdnTensor(ctypes.Structure):
 class GdnExtra(ctypes.Structure):
     _fields_ = [("stream", ctypes.c_void_p), ("intermediate_states", ctypes.POINTER(GdnTensor)),
                 ("device_status", ctypes.c_void_p), ("tile_v", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("tile_rows", ctypes.c_int32), ("schedule", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _LIB = None
@@ -108,7 +113,8 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
                   scale: Optional[float] = None, flags: int = L2NORM_QK,
                   intermediate_states: Optional[torch.Tensor] = None,
                   device_status: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0) -> torch.Tensor:
+                  stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
+                  schedule: int = SCHEDULE_AUTO, tile_rows: int = 0) -> torch.Tensor:
     """Fused sigmoid-gating GDN decode update, in place on ``state_pool``.
 
     Shapes, dtypes and semantics are those of ``gdn_decode_update`` in
@@ -131,7 +137,8 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     extra.intermediate_states = ctypes.pointer(inter) if inter is not None else None
     extra.device_status = device_status.data_ptr() if device_status is not None else None
     extra.tile_v = int(tile_v)
-    extra.reserved = 0
+    extra.tile_rows = int(tile_rows)
+    extra.schedule = int(schedule)
     status = lib.gdn_decode_update(*[_ref(d) for d in descs], ctypes.c_float(scale), ctypes.c_uint32(flags),
                                    ctypes.byref(extra))
     if status != OK:
@@ -140,7 +147,8 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
 
 
 def decode_update_host(host: dict, device: dict, *, scale: Optional[float] = None, flags: int = L2NORM_QK,
-                       stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0) -> None:
+                       stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
+                       schedule: int = SCHEDULE_AUTO, tile_rows: int = 0) -> None:
     """End-to-end call from pinned host buffers.
 
     ``host`` holds pinned CPU tensors q, k, v, a, b, state_indices,
@@ -159,7 +167,8 @@ def decode_update_host(host: dict, device: dict, *, scale: Optional[float] = Non
         decode_update(device["q"], device["k"], device["v"], device["a"], device["b"], device["A_log"],
                       device["dt_bias"], device["state_pool"], device["state_indices"], device.get("cu_seqlens"),
                       device["out"], scale=scale, flags=flags,
-                      intermediate_states=device.get("intermediate_states"), stream=stream, tile_v=tile_v)
+                      intermediate_states=device.get("intermediate_states"), stream=stream, tile_v=tile_v,
+                      schedule=schedule, tile_rows=tile_rows)
         host["out"].copy_(device["out"], non_blocking=True)
 
 
@@ -175,7 +184,8 @@ class PreparedCall:
 
     def __init__(self, q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
                  scale: Optional[float] = None, flags: int = L2NORM_QK, intermediate_states=None,
-                 device_status=None, stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0):
+                 device_status=None, stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
+                 schedule: int = SCHEDULE_AUTO, tile_rows: int = 0):
         self._lib = load()
         self._keep = (q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
                       intermediate_states, device_status)
@@ -191,6 +201,8 @@ class PreparedCall:
         self._extra.intermediate_states = ctypes.pointer(self._inter) if self._inter is not None else None
         self._extra.device_status = device_status.data_ptr() if device_status is not None else None
         self._extra.tile_v = int(tile_v)
+        self._extra.tile_rows = int(tile_rows)
+        self._extra.schedule = int(schedule)
         self._args = [_ref(d) for d in self._descs] + [ctypes.c_float(scale), ctypes.c_uint32(flags),
                                                        ctypes.byref(self._extra)]
         self._fn = self._lib.gdn_decode_update

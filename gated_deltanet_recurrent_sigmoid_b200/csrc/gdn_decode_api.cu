@@ -14,6 +14,7 @@
 
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
+#include "gdn_decode_pipelined.cuh"
 
 namespace {
 
@@ -183,6 +184,42 @@ cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t strea
     return cudaGetLastError();
 }
 
+constexpr int kPipeStages = 3;
+
+// Per-device one-time setup of the pipelined kernel: its dynamic shared
+// memory opt-in and the SM count that sizes its persistent grid.
+struct PipeDevice {
+    int sms = 0;
+    bool ready = false;
+};
+
+cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream)
+{
+    static PipeDevice devices[64];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    const size_t smem = sizeof(gdn::pipe::Smem<kPipeStages>);
+    PipeDevice &d = devices[dev];
+    if (!d.ready) {
+        err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess)
+            return err;
+        err = cudaFuncSetAttribute(gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (err != cudaSuccess)
+            return err;
+        d.ready = true;
+    }
+    const int64_t grid = units < d.sms ? units : d.sms;
+    gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>
+        <<<static_cast<unsigned>(grid), gdn::pipe::THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,6 +252,9 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     // ---- scalars and flags
     const uint32_t known = GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES;
     if ((flags & ~known) != 0 || !std::isfinite(scale) || !(scale > 0.f))
+        return GDN_ERR_ARG;
+    const int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
+    if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED)
         return GDN_ERR_ARG;
     if (extra && extra->reserved != 0)
         return GDN_ERR_ARG;
@@ -340,11 +380,19 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         }
     }
 
-    // ---- supported configurations
+    // ---- supported configurations and the library's choices
     if (K != kHeadK || V != kHeadV)
         return GDN_ERR_UNSUPPORTED;
-    const int tile_v = (extra && extra->tile_v) ? extra->tile_v : 32;
-    if (tile_v != 32 && tile_v != 64 && tile_v != 128)
+    // Single-token decode is a pure stream of state bytes: the widest tile
+    // with the most rows per thread keeps the most bytes in flight per
+    // register.  With several tokens per sequence the per-token reduction
+    // latency dominates: one-warp 16-column tiles need no block barrier.
+    const bool one_token = T_tot == N && !want_inter;
+    int tile_v = (extra && extra->tile_v) ? extra->tile_v : (one_token ? 64 : 16);
+    int tile_rows = (extra && extra->tile_rows) ? extra->tile_rows : (tile_v == 64 && one_token ? 32 : 16);
+    const bool tile_ok = (tile_v == 16 && tile_rows == 16) || (tile_v == 32 && (tile_rows == 16 || tile_rows == 32)) ||
+                         (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
+    if (!tile_ok)
         return GDN_ERR_UNSUPPORTED;
     const int64_t units = N * HV;
     if (units * (kHeadV / tile_v) > INT32_MAX)
@@ -402,11 +450,20 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     p.scale = scale;
     p.flags = flags;
 
+    // Library choice: the per-tile schedule (measured faster on every
+    // workload shape); the pipelined one only on request.
     cudaError_t err;
-    switch (tile_v) {
-    case 32: err = launch<32, 16>(p, units, stream); break;
-    case 64: err = launch<64, 16>(p, units, stream); break;
-    default: err = launch<128, 8>(p, units, stream); break;
+    if (schedule == GDN_SCHEDULE_PIPELINED) {
+        err = launch_pipelined(p, units, stream);
+    } else {
+        // KG (row groups per tile) = K / tile_rows
+        switch (tile_v * 100 + tile_rows) {
+        case 1616: err = launch<16, 8>(p, units, stream); break;
+        case 3216: err = launch<32, 8>(p, units, stream); break;
+        case 3232: err = launch<32, 4>(p, units, stream); break;
+        case 6416: err = launch<64, 8>(p, units, stream); break;
+        default: err = launch<64, 4>(p, units, stream); break;
+        }
     }
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

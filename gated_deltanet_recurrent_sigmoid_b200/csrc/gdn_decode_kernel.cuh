@@ -101,7 +101,7 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
     using TS = TileShape<K, V, BV, KG>;
     constexpr int VG = TS::VG, WARPS = TS::WARPS, R = TS::R, NV = TS::NV, XW = TS::XW;
 
-    __shared__ __align__(16) float xch[2][WARPS][XW];
+    __shared__ __align__(16) float xch[2][WARPS > 1 ? WARPS : 1][WARPS > 1 ? XW : 4];
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -206,6 +206,14 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             sqq += __shfl_xor_sync(0xffffffffu, sqq, off);
             skq += __shfl_xor_sync(0xffffffffu, skq, off);
         }
+        float4 U, W;
+        float SKK, SQQ, SKQ;
+        if constexpr (WARPS == 1) {
+            // the whole tile lives in one warp: the shuffles already summed all rows
+            U = make_float4(u0, u1, u2, u3);
+            W = make_float4(w0, w1, w2, w3);
+            SKK = skk; SQQ = sqq; SKQ = skq;
+        } else {
         const int buf = t & 1;
         if (lane < VG) {
             *reinterpret_cast<float4 *>(&xch[buf][warp][vq * 4]) = make_float4(u0, u1, u2, u3);
@@ -217,8 +225,9 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             }
         }
         __syncthreads();
-        float4 U = make_float4(0.f, 0.f, 0.f, 0.f), W = U;
-        float SKK = 0.f, SQQ = 0.f, SKQ = 0.f;
+        U = make_float4(0.f, 0.f, 0.f, 0.f);
+        W = U;
+        SKK = 0.f; SQQ = 0.f; SKQ = 0.f;
 #pragma unroll
         for (int wi = 0; wi < WARPS; ++wi) {
             const float4 uu = *reinterpret_cast<const float4 *>(&xch[buf][wi][vq * 4]);
@@ -228,6 +237,7 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             SKK += xch[buf][wi][2 * BV + 0];
             SQQ += xch[buf][wi][2 * BV + 1];
             SKQ += xch[buf][wi][2 * BV + 2];
+        }
         }
 
         // ---- gates and norms (scalars, computed by every thread) ----

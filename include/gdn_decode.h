@@ -112,9 +112,22 @@ extern "C" {
                                     or bad cu_seqlens */
 #define GDN_ERR_CUDA        (-9) /* the CUDA runtime refused the launch or copy */
 
+/* work schedules (gdn_extra.schedule); all compute the same update */
+#define GDN_SCHEDULE_AUTO      0 /* library choice */
+#define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
+                                    state tile moves through registers.  Tiles
+                                    (tile_v x tile_rows): 16x16, 32x16, 32x32,
+                                    64x16, 64x32.  Library choice: 64x32 when
+                                    every sequence has one token, else 16x16 */
+#define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
+                                    tiles stream through a shared-memory ring of
+                                    bulk async copies (cp.async.bulk) */
+
 /* bits OR-ed into *device_status by the kernel */
 #define GDN_DEV_BAD_SLOT    1u
 #define GDN_DEV_BAD_SEQLENS 2u
+#define GDN_DEV_TIMEOUT     4u  /* a bounded wait inside the kernel gave up (the
+                                   call's results are then incomplete) */
 
 typedef struct gdn_tensor {
     void *data;          /* device pointer */
@@ -128,7 +141,11 @@ typedef struct gdn_extra {
     void *stream;                          /* cudaStream_t; NULL = legacy default */
     const gdn_tensor *intermediate_states; /* required with GDN_WRITE_INTERMEDIATE */
     uint32_t *device_status;               /* device word for GDN_DEV_* bits, or NULL */
-    int32_t tile_v;                        /* 0 = library choice, else V-tile width */
+    int32_t tile_v;                        /* per-tile schedule: V-tile width (16, 32
+                                              or 64; 0 = library choice) */
+    int32_t tile_rows;                     /* per-tile schedule: state rows per thread
+                                              (16 or 32; 0 = library choice) */
+    int32_t schedule;                      /* GDN_SCHEDULE_* (0 = library choice) */
     int32_t reserved;                      /* must be 0 */
 } gdn_extra;
 

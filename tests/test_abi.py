@@ -63,7 +63,7 @@ def test_header_constants_match_binding():
                       ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9)]:
         assert int(re.search(rf"#define {name}\s+\((-?\d+)\)", text).group(1)) == val
     assert ctypes.sizeof(binding.GdnTensor) == 8 + 4 + 4 + 8 * 4 + 8 * 4
-    assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 + 4
+    assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 * 4
 
 
 def make(N=4, T=1, H=2, HV=4, K=128, V=128, slots=8, varlen=True):
@@ -113,7 +113,9 @@ def test_rejects_bad_dtypes_and_shapes(gdn_lib):
 
 def test_rejects_unsupported_head_size(gdn_lib):
     expect(binding.ERR_UNSUPPORTED, make(K=64, V=64))
-    expect(binding.ERR_UNSUPPORTED, make(), tile_v=16)
+    expect(binding.ERR_UNSUPPORTED, make(), tile_v=128)
+    expect(binding.ERR_UNSUPPORTED, make(), tile_v=16, tile_rows=32)
+    expect(binding.ERR_ARG, make(), schedule=7)
 
 
 def test_rejects_misalignment(gdn_lib):

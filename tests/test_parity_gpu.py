@@ -27,10 +27,26 @@ def _lib(gdn_lib):
     return gdn_lib
 
 
-def check_full(w, flags=L2, tile_v=0, scale=None):
+PER_TILE = binding.SCHEDULE_PER_TILE
+PIPELINED = binding.SCHEDULE_PIPELINED
+# (schedule, V-tile width, rows per thread) of every kernel the library can launch
+KERNELS = [(PER_TILE, 16, 16), (PER_TILE, 32, 16), (PER_TILE, 32, 32), (PER_TILE, 64, 16), (PER_TILE, 64, 32),
+           (PIPELINED, 0, 0)]
+KERNEL_IDS = ["tile16x16", "tile32x16", "tile32x32", "tile64x16", "tile64x32", "pipelined"]
+# the library's two default tiles and the pipelined schedule
+MAIN = [KERNELS[0], KERNELS[4], KERNELS[5]]
+MAIN_IDS = ["tile16x16", "tile64x32", "pipelined"]
+
+
+def kw_of(kernel):
+    return dict(schedule=kernel[0], tile_v=kernel[1], tile_rows=kernel[2])
+
+
+def check_full(w, flags=L2, tile_v=0, scale=None, schedule=binding.SCHEDULE_AUTO, tile_rows=0):
     """Whole-problem comparison: outputs, every pool slot, intermediates."""
     inter = bool(flags & INTER)
-    d, status, inter_t = run_gpu(w, flags=flags, inter=inter, tile_v=tile_v, scale=scale)
+    d, status, inter_t = run_gpu(w, flags=flags, inter=inter, tile_v=tile_v, scale=scale, schedule=schedule,
+                                 tile_rows=tile_rows)
     ostatus, o_ref, s_ref, i_ref = run_oracle(w, flags=flags, scale=scale)
     assert status == ostatus
     assert_out_close(out_as_f32(d["out"]), o_ref)
@@ -60,29 +76,30 @@ SMALL = [
 
 
 @pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
-@pytest.mark.parametrize("tile_v", [32, 64, 128])
-def test_small_configs_match_oracle(spec, tile_v):
+@pytest.mark.parametrize("kernel", KERNELS, ids=KERNEL_IDS)
+def test_small_configs_match_oracle(spec, kernel):
     w = wl.generate(spec)
     flags = L2 | (INTER if spec.intermediate else 0)
-    check_full(w, flags=flags, tile_v=tile_v)
+    check_full(w, flags=flags, **kw_of(kernel))
 
 
 @pytest.mark.parametrize("spec", [wl.TINY, wl.SPEC_B128_T4, wl.sweep_spec(1), wl.sweep_spec(8),
                                   wl.sweep_spec(64)], ids=lambda s: s.name)
-def test_full_size_configs_match_oracle(spec):
+@pytest.mark.parametrize("kernel", [(binding.SCHEDULE_AUTO, 0, 0), KERNELS[5]], ids=["default", "pipelined"])
+def test_full_size_configs_match_oracle(spec, kernel):
     """Full-size configurations the oracle finishes in seconds, compared whole."""
     w = wl.generate(spec)
-    check_full(w, flags=L2 | (INTER if spec.intermediate else 0))
+    check_full(w, flags=L2 | (INTER if spec.intermediate else 0), **kw_of(kernel))
 
 
-def sampled_check(spec, n_sample, seed=0):
+def sampled_check(spec, n_sample, seed=0, schedule=binding.SCHEDULE_AUTO, tile_v=0, tile_rows=0):
     """Full-size problem in the benchmark's launch configuration; the oracle
     recomputes a sample of sequences (always including padded ones and the
     longest), everything else is checked through properties."""
     w = wl.generate(spec)
     d = to_device(w)
     pool_before = d["state_pool"].clone()
-    d, status, _ = run_gpu(w, d=d)
+    d, status, _ = run_gpu(w, d=d, schedule=schedule, tile_v=tile_v, tile_rows=tile_rows)
     assert status == 0
     rng = np.random.default_rng(seed)
     N = spec.N
@@ -115,6 +132,14 @@ def np_token_rows(w, seqs):
 
 def test_decode_b512_full_size_sampled():
     sampled_check(wl.DECODE_B512, 96)
+
+
+def test_decode_b512_full_size_sampled_pipelined():
+    sampled_check(wl.DECODE_B512, 48, schedule=PIPELINED)
+
+
+def test_decode_b512_full_size_sampled_tile16():
+    sampled_check(wl.DECODE_B512, 48, schedule=PER_TILE, tile_v=16, tile_rows=16)
 
 
 def test_fullhead_b256_full_size_sampled():
@@ -150,7 +175,8 @@ def test_chained_single_token_calls_match_multi_token_call():
 def test_intermediate_states_equal_prefix_states():
     """inter[bos + t] equals the pool after a call over the first t+1 tokens."""
     w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 8))
-    _, _, inter = run_gpu(w, flags=L2 | INTER, inter=True)
+    tile = dict(schedule=PER_TILE, tile_v=16, tile_rows=16)       # same kernel for every call
+    _, _, inter = run_gpu(w, flags=L2 | INTER, inter=True, **tile)
     T = 4
     for t in range(T):
         d = to_device(w)
@@ -159,18 +185,18 @@ def test_intermediate_states_equal_prefix_states():
         o = torch.empty(len(rows), w.spec.HV, w.spec.V, dtype=torch.bfloat16, device="cuda")
         binding.decode_update(d["q"][rows].contiguous(), d["k"][rows].contiguous(), d["v"][rows].contiguous(),
                               d["a"][rows].contiguous(), d["b"][rows].contiguous(), d["A_log"], d["dt_bias"],
-                              d["state_pool"], d["state_indices"], cu, o)
+                              d["state_pool"], d["state_indices"], cu, o, **tile)
         torch.cuda.synchronize()
         idx = torch.from_numpy(w.state_indices.astype(np.int64)).cuda()
         got = inter.view(w.spec.N, T, w.spec.HV, 128, 128)[:, t]
         assert torch.equal(got, d["state_pool"][idx])
 
 
-def test_tiles_agree():
+def test_kernels_agree():
     w = wl.generate(wl.shrink(wl.sweep_spec(64), 16))
-    ref, _, _ = run_gpu(w, tile_v=32)
-    for tv in (64, 128):
-        d, _, _ = run_gpu(w, tile_v=tv)
+    ref, _, _ = run_gpu(w, **kw_of(KERNELS[0]))
+    for kernel in KERNELS[1:]:
+        d, _, _ = run_gpu(w, **kw_of(kernel))
         assert (d["state_pool"] - ref["state_pool"]).abs().max().item() <= 1e-5
         assert (d["out"].float() - ref["out"].float()).abs().max().item() <= 2e-2
 
@@ -240,7 +266,8 @@ def test_guard_bands_untouched():
     assert torch.equal(inter_buf[1:-1], iref)
 
 
-def test_device_status_and_skipped_sequences():
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_device_status_and_skipped_sequences(kernel):
     rng = np.random.default_rng(5)
     p = random_problem(rng, lens=[2, 1, 3, 2], H=2, HV=4, K=128, V=128, num_slots=8)
     p["state_indices"][1] = 8          # out of range
@@ -248,7 +275,7 @@ def test_device_status_and_skipped_sequences():
     spec = wl.WorkloadSpec("bad", N=4, H=2, HV=4, num_slots=8, seed=0, T=None)
     w = wl.Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
                     p["state_indices"], p["cu_seqlens"])
-    d, status, _ = run_gpu(w)
+    d, status, _ = run_gpu(w, **kw_of(kernel))
     ostatus, o_ref, s_ref, _ = run_oracle(w)
     assert status == ostatus == oracle.BAD_SLOT
     assert_out_close(out_as_f32(d["out"]), o_ref)       # skipped rows stay NaN on both sides
@@ -260,33 +287,37 @@ def test_device_status_and_skipped_sequences():
     p["state_indices"] = rng.permutation(8)[:4].astype(np.int32)
     w2 = wl.Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
                      p["state_indices"], np.array([0, 2, 3, 6, 9], dtype=np.int32))   # last runs past T_tot
-    d2, status2, _ = run_gpu(w2)
+    d2, status2, _ = run_gpu(w2, **kw_of(kernel))
     ostatus2, o_ref2, _, _ = run_oracle(w2)
     assert status2 == ostatus2 == oracle.BAD_SEQLENS
     assert_out_close(out_as_f32(d2["out"]), o_ref2)
 
 
-def test_empty_sequences_all_padded_and_no_tokens():
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_empty_sequences_all_padded_and_no_tokens(kernel):
     rng = np.random.default_rng(6)
     p = random_problem(rng, lens=[0, 3, 0, 1], H=1, HV=2, K=128, V=128, num_slots=6, pad=(3,))
     spec = wl.WorkloadSpec("empties", N=4, H=1, HV=2, num_slots=6, seed=0, T=None)
     w = wl.Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
                     p["state_indices"], p["cu_seqlens"])
-    check_full(w)
+    check_full(w, **kw_of(kernel))
     p2 = dict(p, state_indices=np.full(4, -1, dtype=np.int32))
     w2 = wl.Workload(spec, p2["q"], p2["k"], p2["v"], p2["a"], p2["b"], p2["A_log"], p2["dt_bias"],
                      p2["state_pool"], p2["state_indices"], p2["cu_seqlens"])
-    check_full(w2)
+    check_full(w2, **kw_of(kernel))
 
 
-def test_no_final_writeback_and_l2norm_off():
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_no_final_writeback_and_l2norm_off(kernel):
     w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 12))
-    check_full(w, flags=L2 | INTER | binding.NO_FINAL_WRITEBACK)
-    check_full(w, flags=INTER)
-    check_full(w, flags=L2, scale=0.3)
+    kw = kw_of(kernel)
+    check_full(w, flags=L2 | INTER | binding.NO_FINAL_WRITEBACK, **kw)
+    check_full(w, flags=INTER, **kw)
+    check_full(w, flags=L2, scale=0.3, **kw)
 
 
-def test_special_gate_values_match_oracle():
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_special_gate_values_match_oracle(kernel):
     """Infinite a and b (decay 1, beta 0 or 1), A_log = -inf, softplus above
     its threshold and one-hot q/k: the same special cases that pin the oracle."""
     rng = np.random.default_rng(7)
@@ -303,8 +334,8 @@ def test_special_gate_values_match_oracle():
     spec = wl.WorkloadSpec("special", N=N, H=H, HV=HV, num_slots=2 * N, seed=0, T=None)
     w = wl.Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
                     p["state_indices"], p["cu_seqlens"])
-    check_full(w)
-    check_full(w, flags=0)
+    check_full(w, **kw_of(kernel))
+    check_full(w, flags=0, **kw_of(kernel))
 
 
 def test_check_indices_flag_rejects_duplicates():
