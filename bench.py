@@ -47,8 +47,8 @@ ROTATING_COPIES = 4
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": "b4c54bba8390bf24727314370b03fe02fd473850fb91495c81cec9ef9267daa1",
-               "bytes_per_launch": 257369600 + 198541824}
+NCU_TRAFFIC = {"kernel_sha256": "f7124fe1765f103b692eb6286daad783c1830477a4635c28061214b504f787fa",
+               "bytes_per_launch": 257369856 + 198864384}
 
 
 def kernel_source_hash() -> str:
@@ -205,14 +205,17 @@ def run_reference(args, w):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def kernel_name(schedule, tile_v, tile_rows, one_token):
+def kernel_name(schedule, tile_v, tile_rows, one_token, pairs):
     """Name of the kernel the library launches for these settings (mirrors
     the library's documented choice)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
-    bv = tile_v or (64 if one_token else 16)
-    rows = tile_rows or (32 if bv == 64 and one_token else 16)
+    if tile_v:
+        bv, rows = tile_v, tile_rows or 16
+    else:
+        bv, rows = (64, 32) if one_token else ((32, 32) if pairs >= 4096 else (16, 16))
+        rows = tile_rows or rows
     return f"gdn::gdn_decode_kernel<128,128,{bv},{128 // rows}>"
 
 
@@ -377,7 +380,8 @@ def main():
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
                          "kernel": kernel_name(schedule, args.tile_v, args.tile_rows,
-                                               w.T_tot == w.spec.N and not w.spec.intermediate)},
+                                               w.T_tot == w.spec.N and not w.spec.intermediate,
+                                               w.spec.N * w.spec.HV)},
             "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clocks,

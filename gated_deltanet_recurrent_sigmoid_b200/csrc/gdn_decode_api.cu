@@ -385,11 +385,30 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         return GDN_ERR_UNSUPPORTED;
     // Single-token decode is a pure stream of state bytes: the widest tile
     // with the most rows per thread keeps the most bytes in flight per
-    // register.  With several tokens per sequence the per-token reduction
-    // latency dominates: one-warp 16-column tiles need no block barrier.
+    // register (64 x 32).  With several tokens per sequence the work per
+    // state byte grows with the length and the per-token dependency chain
+    // (reduction over K, then the update) sets the time: one-warp tiles need
+    // no block barrier -- 32 x 32 when there are many (sequence, head)
+    // pairs, 16 x 16 (twice the CTAs, shorter chains) when there are few.
     const bool one_token = T_tot == N && !want_inter;
-    int tile_v = (extra && extra->tile_v) ? extra->tile_v : (one_token ? 64 : 16);
-    int tile_rows = (extra && extra->tile_rows) ? extra->tile_rows : (tile_v == 64 && one_token ? 32 : 16);
+    const int64_t pairs = N * HV;
+    int tile_v, tile_rows;
+    if (one_token) {
+        tile_v = 64;
+        tile_rows = 32;
+    } else if (pairs >= 4096) {
+        tile_v = 32;
+        tile_rows = 32;
+    } else {
+        tile_v = 16;
+        tile_rows = 16;
+    }
+    if (extra && extra->tile_v) {
+        tile_v = extra->tile_v;
+        tile_rows = extra->tile_rows ? extra->tile_rows : 16;
+    } else if (extra && extra->tile_rows) {
+        tile_rows = extra->tile_rows;
+    }
     const bool tile_ok = (tile_v == 16 && tile_rows == 16) || (tile_v == 32 && (tile_rows == 16 || tile_rows == 32)) ||
                          (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
     if (!tile_ok)

@@ -165,21 +165,40 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
     const bool l2norm = (p.flags & GDN_L2NORM_QK) != 0;
     const bool write_inter = (p.flags & GDN_WRITE_INTERMEDIATE) != 0;
 
+    // Token inputs are software-pipelined: the raw bf16 words of token t+1
+    // are in flight while token t is computed.
+    uint4 k_nx[R / 8], q_nx[R / 8];
+    uint2 v_nx;
+    unsigned short a_nx, b_nx;
+    auto fetch = [&](int64_t tok) {
+        const uint4 *kp = reinterpret_cast<const uint4 *>(p.k + tok * p.k_tok + h * p.k_head + row0);
+        const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + tok * p.q_tok + h * p.q_head + row0);
+#pragma unroll
+        for (int c = 0; c < R / 8; ++c) {
+            k_nx[c] = __ldg(kp + c);
+            q_nx[c] = __ldg(qp + c);
+        }
+        v_nx = __ldg(reinterpret_cast<const uint2 *>(p.v + tok * p.v_tok + hv * p.v_head + col0));
+        a_nx = __ldg(reinterpret_cast<const unsigned short *>(p.a + tok * p.a_tok + hv * p.a_head));
+        b_nx = __ldg(reinterpret_cast<const unsigned short *>(p.b + tok * p.b_tok + hv * p.b_head));
+    };
+    fetch(bos);
+
     for (int t = 0; t < len; ++t) {
         const int64_t tok = bos + t;
 
         // ---- inputs: this thread's R rows of q and k, 4 columns of v
         float kr[R], qr[R];
-        const uint4 *kp = reinterpret_cast<const uint4 *>(p.k + tok * p.k_tok + h * p.k_head + row0);
-        const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + tok * p.q_tok + h * p.q_head + row0);
 #pragma unroll
         for (int c = 0; c < R / 8; ++c) {
-            unpack8(__ldg(kp + c), kr + 8 * c);
-            unpack8(__ldg(qp + c), qr + 8 * c);
+            unpack8(k_nx[c], kr + 8 * c);
+            unpack8(q_nx[c], qr + 8 * c);
         }
-        const uint2 v_raw = __ldg(reinterpret_cast<const uint2 *>(p.v + tok * p.v_tok + hv * p.v_head + col0));
-        const float a_t = load_bf16(p.a + tok * p.a_tok + hv * p.a_head);
-        const float b_t = load_bf16(p.b + tok * p.b_tok + hv * p.b_head);
+        const uint2 v_raw = v_nx;
+        const float a_t = __uint_as_float(static_cast<uint32_t>(a_nx) << 16);
+        const float b_t = __uint_as_float(static_cast<uint32_t>(b_nx) << 16);
+        if (t + 1 < len)
+            fetch(tok + 1);
 
         // ---- partial S^T k, S^T q, |k|^2, |q|^2, k.q over my rows ----
         float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;

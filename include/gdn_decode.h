@@ -118,7 +118,9 @@ extern "C" {
                                     state tile moves through registers.  Tiles
                                     (tile_v x tile_rows): 16x16, 32x16, 32x32,
                                     64x16, 64x32.  Library choice: 64x32 when
-                                    every sequence has one token, else 16x16 */
+                                    every sequence has one token, else 32x32
+                                    with >= 4096 (sequence, value head) pairs,
+                                    else 16x16 */
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
                                     tiles stream through a shared-memory ring of
                                     bulk async copies (cp.async.bulk) */
