@@ -47,8 +47,7 @@ ROTATING_COPIES = 4
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": "f7124fe1765f103b692eb6286daad783c1830477a4635c28061214b504f787fa",
-               "bytes_per_launch": 257369856 + 198864384}
+NCU_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None}
 
 
 def kernel_source_hash() -> str:
@@ -219,12 +218,13 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs):
     return f"gdn::gdn_decode_kernel<128,128,{bv},{128 // rows}>"
 
 
-def workload_config(w, world):
+def workload_config(w, world, pdl=False):
     s = w.spec
     return {"workload": s.name, "B": s.N, "T": s.T if s.T is not None else "U{1..64}", "H": s.H, "HV": s.HV,
             "K": s.K, "V": s.V, "num_slots": s.num_slots, "padded": int((w.state_indices < 0).sum()),
             "state_dtype": "f32", "activation_dtype": "bf16",
             "l2": f"inputs larger than L2: steps rotate over {ROTATING_COPIES} input copies",
+            "launch": "programmatic dependent launch" if pdl else "plain stream order",
             "parallelism": "replicas" if world == 1 else f"dp{world}"}
 
 
@@ -255,6 +255,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--no-pdl", dest="pdl", action="store_false",
+                    help="launch in plain stream order instead of with programmatic dependent launch")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -288,6 +290,8 @@ def main():
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
+    if args.pdl:
+        flags |= binding.LAUNCH_PDL
     calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"], c["state_pool"],
                                   c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
                                   intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
@@ -329,20 +333,22 @@ def main():
     ms_per_step = max_region_ms / args.steps
     value = nbytes * world * args.steps / (max_region_ms * 1e-3) / 1e9
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: each step
+    # copies its inputs host -> device (one packed copy), launches, copies the
+    # output back and synchronises on it
     e2e = None
     if not args.skip_e2e:
-        host = {n: copies[0][n].cpu().pin_memory() for n in ("q", "k", "v", "a", "b", "state_indices")}
-        if copies[0]["cu_seqlens"] is not None:
-            host["cu_seqlens"] = copies[0]["cu_seqlens"].cpu().pin_memory()
-        host["out"] = torch.empty(copies[0]["out"].shape, dtype=torch.bfloat16).pin_memory()
-        dev = dict(copies[0])
-        dev["intermediate_states"] = dev.pop("inter", None)
-        h2d = sum(host[n].numel() * host[n].element_size() for n in host if n != "out")
-        d2h = host["out"].numel() * host["out"].element_size()
+        c0 = copies[0]
+        s = w.spec
+        staged = binding.HostStagedDecode(c0["q"].shape[:-2], s.H, s.HV, s.K, s.V, s.N, c0["A_log"], c0["dt_bias"],
+                                          c0["state_pool"], varlen=c0["cu_seqlens"] is not None, flags=flags,
+                                          intermediate_states=c0.get("inter"), stream=stream, tile_v=args.tile_v,
+                                          tile_rows=args.tile_rows, schedule=schedule)
+        for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
+            if c0.get(name) is not None:
+                getattr(staged, name).copy_(c0[name].cpu())
         for _ in range(3):
-            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v,
-                                       schedule=schedule, tile_rows=args.tile_rows)
+            staged.step()
             stream.synchronize()
         if world > 1:
             dist.barrier()
@@ -350,8 +356,7 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
-            binding.decode_update_host(host, dev, flags=flags, stream=stream, tile_v=args.tile_v,
-                                       schedule=schedule, tile_rows=args.tile_rows)
+            staged.step()
             stream.synchronize()          # the step ends when the host holds the output
         e1.record(stream)
         torch.cuda.synchronize(device)
@@ -360,7 +365,9 @@ def main():
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e_ms = float(te.item()) / args.e2e_steps
         e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
-               "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(staged.h2d_bytes),
+               "d2h_bytes_per_step": int(staged.d2h_bytes), "api": "binding.HostStagedDecode"}
+        del staged
 
     if rank == 0:
         peak, peak_src = hbm_peak()
@@ -372,7 +379,7 @@ def main():
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world, args.pdl),
             "us_per_call": round(avg_kernel_ms * 1e3, 3),
             "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                          "peak_source": peak_src},

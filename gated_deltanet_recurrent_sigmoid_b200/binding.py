@@ -21,6 +21,7 @@ L2NORM_QK = 1 << 0
 WRITE_INTERMEDIATE = 1 << 1
 NO_FINAL_WRITEBACK = 1 << 2
 CHECK_INDICES = 1 << 3
+LAUNCH_PDL = 1 << 4
 
 DEV_BAD_SLOT = 1
 DEV_BAD_SEQLENS = 2
@@ -211,3 +212,63 @@ class PreparedCall:
         status = self._fn(*self._args)
         if status != OK:
             raise GdnError(status, status_string(status))
+
+
+class HostStagedDecode:
+    """A decode step fed from pinned host memory, with the fewest transfers.
+
+    All per-step inputs (q, k, v, a, b, state_indices and cu_seqlens) live in
+    ONE pinned host buffer, mirrored by one device buffer; each ``step()`` is
+    one host-to-device copy of that buffer, one kernel launch and one
+    device-to-host copy of ``out``, all on ``stream`` (asynchronous: sync the
+    stream before reading ``out_host``).  Write a step's inputs into the host
+    views (``q``, ``k``, ... attributes) before calling ``step()``.  The
+    state pool, A_log and dt_bias stay resident on the device.
+
+    Shapes follow ``decode_update``: q, k [T_tot, H, K]; v, out [T_tot, HV, V];
+    a, b [T_tot, HV]; state_indices [N]; cu_seqlens [N+1] or None with
+    fixed-length [N, T, ...] leading dims given by ``tokens_shape``.
+    """
+
+    _ALIGN = 256
+
+    def __init__(self, tokens_shape, H, HV, K, V, N, A_log, dt_bias, state_pool, varlen=True,
+                 scale: Optional[float] = None, flags: int = L2NORM_QK, intermediate_states=None,
+                 stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0, tile_rows: int = 0,
+                 schedule: int = SCHEDULE_AUTO):
+        dev = state_pool.device
+        tokens_shape = tuple(tokens_shape)
+        layout = [("q", tokens_shape + (H, K), torch.bfloat16), ("k", tokens_shape + (H, K), torch.bfloat16),
+                  ("v", tokens_shape + (HV, V), torch.bfloat16), ("a", tokens_shape + (HV,), torch.bfloat16),
+                  ("b", tokens_shape + (HV,), torch.bfloat16), ("state_indices", (N,), torch.int32)]
+        if varlen:
+            layout.append(("cu_seqlens", (N + 1,), torch.int32))
+        offsets, off = {}, 0
+        for name, shape, dt in layout:
+            nbytes = math.prod(shape) * torch.tensor([], dtype=dt).element_size()
+            offsets[name] = (off, nbytes, shape, dt)
+            off += -(-nbytes // self._ALIGN) * self._ALIGN
+        self.host_buffer = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.device_buffer = torch.empty(off, dtype=torch.uint8, device=dev)
+        views = {}
+        for name, (o, n, shape, dt) in offsets.items():
+            setattr(self, name, self.host_buffer[o:o + n].view(dt).view(shape))
+            views[name] = self.device_buffer[o:o + n].view(dt).view(shape)
+        if not varlen:
+            self.cu_seqlens = None
+        self.out_device = torch.empty(tokens_shape + (HV, V), dtype=torch.bfloat16, device=dev)
+        self.out_host = torch.empty(self.out_device.shape, dtype=torch.bfloat16).pin_memory()
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        self._call = PreparedCall(views["q"], views["k"], views["v"], views["a"], views["b"], A_log, dt_bias,
+                                  state_pool, views["state_indices"], views.get("cu_seqlens"), self.out_device,
+                                  scale=scale, flags=flags, intermediate_states=intermediate_states,
+                                  stream=self.stream, tile_v=tile_v, tile_rows=tile_rows, schedule=schedule)
+        self.h2d_bytes = off
+        self.d2h_bytes = self.out_host.numel() * self.out_host.element_size()
+
+    def step(self) -> torch.Tensor:
+        with torch.cuda.stream(self.stream):
+            self.device_buffer.copy_(self.host_buffer, non_blocking=True)
+            self._call()
+            self.out_host.copy_(self.out_device, non_blocking=True)
+        return self.out_host

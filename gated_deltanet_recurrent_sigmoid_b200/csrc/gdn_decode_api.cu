@@ -175,13 +175,30 @@ int check_indices_on_host(const int32_t *d_idx, const int32_t *d_cu, int64_t N, 
     return GDN_OK;
 }
 
+// Launch with or without the programmatic-stream-serialization attribute.
+template <typename Kernel>
+cudaError_t launch_ex(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                      const gdn::DecodeParams &p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <int BV, int KG>
-cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream)
+cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl)
 {
     using TS = gdn::TileShape<kHeadK, kHeadV, BV, KG>;
     const dim3 grid(static_cast<unsigned>(units * TS::NV));
-    gdn::gdn_decode_kernel<kHeadK, kHeadV, BV, KG><<<grid, TS::THREADS, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_ex(gdn::gdn_decode_kernel<kHeadK, kHeadV, BV, KG>, grid, dim3(TS::THREADS), 0, stream, pdl, p);
 }
 
 constexpr int kPipeStages = 3;
@@ -193,7 +210,7 @@ struct PipeDevice {
     bool ready = false;
 };
 
-cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream)
+cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl)
 {
     static PipeDevice devices[64];
     int dev = 0;
@@ -215,9 +232,8 @@ cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStre
         d.ready = true;
     }
     const int64_t grid = units < d.sms ? units : d.sms;
-    gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>
-        <<<static_cast<unsigned>(grid), gdn::pipe::THREADS, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_ex(gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>, dim3(static_cast<unsigned>(grid)),
+                     dim3(gdn::pipe::THREADS), smem, stream, pdl, p);
 }
 
 }  // namespace
@@ -250,7 +266,8 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
                               const gdn_tensor *out, float scale, uint32_t flags, const gdn_extra *extra)
 {
     // ---- scalars and flags
-    const uint32_t known = GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES;
+    const uint32_t known =
+        GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES | GDN_LAUNCH_PDL;
     if ((flags & ~known) != 0 || !std::isfinite(scale) || !(scale > 0.f))
         return GDN_ERR_ARG;
     const int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
@@ -471,17 +488,18 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
 
     // Library choice: the per-tile schedule (measured faster on every
     // workload shape); the pipelined one only on request.
+    const bool pdl = (flags & GDN_LAUNCH_PDL) != 0;
     cudaError_t err;
     if (schedule == GDN_SCHEDULE_PIPELINED) {
-        err = launch_pipelined(p, units, stream);
+        err = launch_pipelined(p, units, stream, pdl);
     } else {
         // KG (row groups per tile) = K / tile_rows
         switch (tile_v * 100 + tile_rows) {
-        case 1616: err = launch<16, 8>(p, units, stream); break;
-        case 3216: err = launch<32, 8>(p, units, stream); break;
-        case 3232: err = launch<32, 4>(p, units, stream); break;
-        case 6416: err = launch<64, 8>(p, units, stream); break;
-        default: err = launch<64, 4>(p, units, stream); break;
+        case 1616: err = launch<16, 8>(p, units, stream, pdl); break;
+        case 3216: err = launch<32, 8>(p, units, stream, pdl); break;
+        case 3232: err = launch<32, 4>(p, units, stream, pdl); break;
+        case 6416: err = launch<64, 8>(p, units, stream, pdl); break;
+        default: err = launch<64, 4>(p, units, stream, pdl); break;
         }
     }
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

@@ -74,6 +74,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return l | (h << 16);
 }
 
+// Programmatic dependent launch: let the next kernel on the stream be
+// scheduled as soon as every CTA of this grid has started, then wait until the
+// previous kernel has completed (and its writes are visible) before touching
+// any input.  Both are no-ops when the grid was launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_prologue()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(uint32_t *status, uint32_t bit)
 {
     if (status)
@@ -102,6 +113,8 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
     constexpr int VG = TS::VG, WARPS = TS::WARPS, R = TS::R, NV = TS::NV, XW = TS::XW;
 
     __shared__ __align__(16) float xch[2][WARPS > 1 ? WARPS : 1][WARPS > 1 ? XW : 4];
+
+    pdl_prologue();
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;

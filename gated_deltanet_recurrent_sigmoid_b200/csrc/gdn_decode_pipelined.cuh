@@ -212,6 +212,7 @@ __device__ __forceinline__ Unit classify(const DecodeParams &p, int unit)
 template <int STAGES>
 __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const __grid_constant__ DecodeParams p)
 {
+    pdl_prologue();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem<STAGES> &sm = *reinterpret_cast<Smem<STAGES> *>(smem_raw);
     volatile int *failed = &sm.failed;

@@ -63,7 +63,8 @@
  * Errors.  The call returns GDN_OK or a negative gdn_status.  Every argument
  * check happens on the host before anything is enqueued; on any error
  * nothing is launched and no memory is touched.  The call is asynchronous
- * on extra->stream (NULL: the legacy default stream).  N = 0 or T_tot = 0 is
+ * on extra->stream (NULL: the legacy default stream) and can be captured in
+ * a CUDA graph (unless GDN_CHECK_INDICES is set).  N = 0 or T_tot = 0 is
  * GDN_OK with no launch.  Problems only the device can see (a slot index
  * < -1 or >= num_slots, cu_seqlens not monotone or past T_tot) are reported
  * by OR-ing GDN_DEV_* bits into *extra->device_status (when given); the
@@ -98,6 +99,12 @@ extern "C" {
 #define GDN_CHECK_INDICES      (1u << 3) /* host check of indices / cu_seqlens
                                             (copies them to the host and
                                             synchronises extra->stream) */
+#define GDN_LAUNCH_PDL         (1u << 4) /* programmatic dependent launch: the
+                                            kernel may be scheduled while the
+                                            previous kernel on the stream is
+                                            still running; it waits for that
+                                            kernel to complete before reading
+                                            any input, so results are unchanged */
 
 /* status codes returned by the host call */
 #define GDN_OK               0

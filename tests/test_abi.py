@@ -58,6 +58,7 @@ def test_header_constants_match_binding():
     assert define("GDN_WRITE_INTERMEDIATE") == binding.WRITE_INTERMEDIATE
     assert define("GDN_NO_FINAL_WRITEBACK") == binding.NO_FINAL_WRITEBACK
     assert define("GDN_CHECK_INDICES") == binding.CHECK_INDICES
+    assert define("GDN_LAUNCH_PDL") == binding.LAUNCH_PDL
     for name, val in [("GDN_ERR_NULL_ARG", -1), ("GDN_ERR_DTYPE", -2), ("GDN_ERR_SHAPE", -3),
                       ("GDN_ERR_ALIGN", -4), ("GDN_ERR_ALIAS", -5), ("GDN_ERR_UNSUPPORTED", -6),
                       ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9)]:

@@ -364,3 +364,73 @@ def test_validation_on_device_tensors():
         with pytest.raises(binding.GdnError) as e:
             binding.decode_update(*args(**kw))
         assert e.value.status == code
+
+
+@pytest.mark.parametrize("spec", [wl.TINY, wl.shrink(wl.SPEC_B128_T4, 16)], ids=lambda s: s.name)
+def test_host_staged_decode_matches_device_call(spec):
+    """One packed host-to-device copy, one launch, one copy back: same bits
+    as the device-resident call."""
+    w = wl.generate(spec)
+    ref, _, _ = run_gpu(w)
+    d = to_device(w)
+    varlen = w.cu_seqlens is not None
+    staged = binding.HostStagedDecode(d["q"].shape[:-2], spec.H, spec.HV, spec.K, spec.V, spec.N, d["A_log"],
+                                      d["dt_bias"], d["state_pool"], varlen=varlen)
+    for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
+        if d.get(name) is not None:
+            getattr(staged, name).copy_(d[name].cpu())
+    out = staged.step()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref["out"].cpu())
+    assert torch.equal(d["state_pool"], ref["state_pool"])
+    assert staged.h2d_bytes >= sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v", "a", "b"))
+
+
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_cuda_graph_capture_replays_the_same_update(kernel):
+    """The launch is capturable: a graph of two chained updates replays to
+    the same bits as the same two updates run eagerly."""
+    w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 12))
+    kw = kw_of(kernel)
+    eager = to_device(w)
+    for _ in range(2):
+        binding.decode_update(eager["q"], eager["k"], eager["v"], eager["a"], eager["b"], eager["A_log"],
+                              eager["dt_bias"], eager["state_pool"], eager["state_indices"], eager["cu_seqlens"],
+                              eager["out"], **kw)
+    torch.cuda.synchronize()
+    d = to_device(w)
+    pool0 = d["state_pool"].clone()
+    stream = torch.cuda.Stream()
+    call = binding.PreparedCall(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"],
+                                d["state_indices"], d["cu_seqlens"], d["out"], stream=stream, **kw)
+    call()                                   # warm-up (one-time per-device setup happens outside capture)
+    torch.cuda.synchronize()
+    d["state_pool"].copy_(pool0)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        call()
+        call()
+    d["state_pool"].copy_(pool0)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(d["out"], eager["out"]) and torch.equal(d["state_pool"], eager["state_pool"])
+
+
+@pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
+def test_programmatic_dependent_launch_keeps_results(kernel):
+    """With GDN_LAUNCH_PDL every launch still waits for the previous kernel
+    before reading: a chain of launches over the same pool (each reads the
+    state the previous one wrote) equals the chain without PDL."""
+    w = wl.generate(wl.shrink(wl.DECODE_B512, 200))
+    kw = kw_of(kernel)
+    results = []
+    for flags in (L2, L2 | binding.LAUNCH_PDL):
+        d = to_device(w)
+        for _ in range(6):
+            binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
+                                  d["state_pool"], d["state_indices"], d["cu_seqlens"], d["out"], flags=flags, **kw)
+        torch.cuda.synchronize()
+        results.append((d["out"].clone(), d["state_pool"].clone()))
+    assert torch.equal(results[0][0], results[1][0]) and torch.equal(results[0][1], results[1][1])
