@@ -11,7 +11,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SOURCES = ["gdn_oracle.c", "gdn_oracle_f32.c"]
+SOURCES = ["gdn_oracle.c", "gdn_oracle_f32.c", "gdn_oracle_fin.c"]
 HEADERS = ["gdn_oracle.h"]
 LIB_PATH = os.path.join(HERE, "libgdn_oracle.so")
 

@@ -6,8 +6,9 @@
  * The loop nest is the definition written out: sequence -> value head ->
  * token -> (gating, q/k normalisation, decay, S^T k, delta, rank-1 update,
  * output, optional intermediate copy).  No step is fused, reordered or
- * blocked.  The file is compiled twice: as-is for the fp64 oracle, and from
- * gdn_oracle_f32.c with GDN_ORACLE_REAL=float for the fp32 drift study.
+ * blocked.  The file is compiled three times: as-is for the fp64 oracle,
+ * from gdn_oracle_f32.c with GDN_ORACLE_REAL=float for the fp32 drift study,
+ * and from gdn_oracle_fin.c with fp32 (instead of bf16-pattern) inputs.
  * <tgmath.h> makes exp/log1p/sqrt follow the working type.
  */
 #include <stddef.h>
@@ -17,13 +18,22 @@
 
 #include "gdn_oracle.h"
 
+/* Three builds of this file: fp64 with bf16-pattern inputs (the oracle),
+ * fp32 with bf16-pattern inputs (drift study), fp64 with fp32 inputs. */
 #ifndef GDN_ORACLE_REAL
 #define GDN_ORACLE_REAL double
 #define GDN_ORACLE_FN gdn_oracle_update
+#define GDN_ORACLE_GATING_FN gdn_oracle_gating
+#endif
+#ifndef GDN_ORACLE_IN_T
+#define GDN_ORACLE_IN_T uint16_t
+#define GDN_ORACLE_IN_BF16 1
 #endif
 
 typedef GDN_ORACLE_REAL real;
+typedef GDN_ORACLE_IN_T in_t;
 
+#ifdef GDN_ORACLE_IN_BF16
 /* A bf16 value is the upper half of an IEEE binary32 pattern. */
 static real bf16_bits_to_real(uint16_t bits)
 {
@@ -32,6 +42,13 @@ static real bf16_bits_to_real(uint16_t bits)
     memcpy(&f, &u, sizeof f);
     return (real)f;
 }
+#else
+/* fp32 inputs: the value itself. */
+static real bf16_bits_to_real(float x)
+{
+    return (real)x;
+}
+#endif
 
 /* softplus(x) = ln(1 + e^x); above 20 the correction e^-x is below 2e-9
  * relative and the function returns x (reading: threshold 20). */
@@ -48,9 +65,26 @@ static real sigmoid(real x)
     return (real)1 / ((real)1 + exp(-x));
 }
 
-int GDN_ORACLE_FN(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                  const uint16_t *a, const uint16_t *b,
+/* g, beta = -exp(A_log) softplus(a + dt_bias), sigmoid(b), per (token, value
+ * head): the gating step on its own (the pages' fused_gdn_gating). */
+int GDN_ORACLE_GATING_FN(const in_t *a, const in_t *b, const float *A_log, const float *dt_bias,
+                         int32_t T_tot, int32_t HV, real *g_out, real *beta_out)
+{
+    if (!a || !b || !A_log || !dt_bias || !g_out || !beta_out || T_tot < 0 || HV <= 0)
+        return GDN_ORACLE_BAD_ARGUMENT;
+    for (int64_t tok = 0; tok < T_tot; ++tok)
+        for (int32_t hv = 0; hv < HV; ++hv) {
+            const real x = bf16_bits_to_real(a[(size_t)tok * HV + hv]) + (real)dt_bias[hv];
+            g_out[(size_t)tok * HV + hv] = -exp((real)A_log[hv]) * softplus(x);
+            beta_out[(size_t)tok * HV + hv] = sigmoid(bf16_bits_to_real(b[(size_t)tok * HV + hv]));
+        }
+    return 0;
+}
+
+int GDN_ORACLE_FN(const in_t *q, const in_t *k, const in_t *v,
+                  const in_t *a, const in_t *b,
                   const float *A_log, const float *dt_bias,
+                  const float *g_in, const float *beta_in,
                   const float *state_in, const int32_t *state_indices,
                   const int32_t *cu_seqlens,
                   int32_t N, int32_t T_fixed, int32_t T_tot,
@@ -64,8 +98,11 @@ int GDN_ORACLE_FN(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     const int final_write = (flags & GDN_ORACLE_NO_FINAL_WRITEBACK) == 0;
     int status = 0;
 
-    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state_in ||
-        !state_indices || !out || !state_out)
+    /* Gates: from (a, b, A_log, dt_bias), or given as (g, beta) arrays. */
+    const int given_gates = g_in != NULL || beta_in != NULL;
+    if (given_gates ? (!g_in || !beta_in) : (!a || !b || !A_log || !dt_bias))
+        return GDN_ORACLE_BAD_ARGUMENT;
+    if (!q || !k || !v || !state_in || !state_indices || !out || !state_out)
         return GDN_ORACLE_BAD_ARGUMENT;
     if (N < 0 || T_tot < 0 || H <= 0 || HV <= 0 || K <= 0 || V <= 0 ||
         num_slots < 0 || HV % H != 0)
@@ -129,14 +166,20 @@ int GDN_ORACLE_FN(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 S[e] = (real)S_in[e];
 
             for (int64_t tok = bos; tok < eos; ++tok) {
-                /* Gating: g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b). */
-                const real x = bf16_bits_to_real(a[(size_t)tok * HV + hv]) + (real)dt_bias[hv];
-                const real g = -exp((real)A_log[hv]) * softplus(x);
-                const real beta = sigmoid(bf16_bits_to_real(b[(size_t)tok * HV + hv]));
+                real g, beta;
+                if (given_gates) {
+                    g = (real)g_in[(size_t)tok * HV + hv];
+                    beta = (real)beta_in[(size_t)tok * HV + hv];
+                } else {
+                    /* Gating: g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b). */
+                    const real x = bf16_bits_to_real(a[(size_t)tok * HV + hv]) + (real)dt_bias[hv];
+                    g = -exp((real)A_log[hv]) * softplus(x);
+                    beta = sigmoid(bf16_bits_to_real(b[(size_t)tok * HV + hv]));
+                }
 
                 /* q and k of key head h, L2-normalised; q scaled. */
-                const uint16_t *k_row = k + ((size_t)tok * H + h) * K;
-                const uint16_t *q_row = q + ((size_t)tok * H + h) * K;
+                const in_t *k_row = k + ((size_t)tok * H + h) * K;
+                const in_t *q_row = q + ((size_t)tok * H + h) * K;
                 real sum_kk = 0, sum_qq = 0;
                 for (int32_t r = 0; r < K; ++r) {
                     const real kr = bf16_bits_to_real(k_row[r]);
@@ -165,7 +208,7 @@ int GDN_ORACLE_FN(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 }
 
                 /* delta = beta (v - kv). */
-                const uint16_t *v_row = v + ((size_t)tok * HV + hv) * V;
+                const in_t *v_row = v + ((size_t)tok * HV + hv) * V;
                 for (int32_t c = 0; c < V; ++c)
                     delta[c] = beta * (bf16_bits_to_real(v_row[c]) - kv[c]);
 

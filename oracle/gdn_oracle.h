@@ -72,10 +72,16 @@ extern "C" {
 #define GDN_ORACLE_BAD_SEQLENS  2
 #define GDN_ORACLE_BAD_ARGUMENT (-1)
 
-/* fp64 oracle: every step in double precision. */
+/* fp64 oracle: every step in double precision.  Gates come from (a, b,
+ * A_log, dt_bias), or -- when g and beta are given (both non-NULL; a, b,
+ * A_log and dt_bias are then ignored and may be NULL) -- from the per
+ * (token, value head) arrays g [T_tot, HV] (S <- exp(g) S) and beta
+ * [T_tot, HV]: the recurrence of the unfused pair (the pages'
+ * fused_recurrent_gated_delta_rule with precomputed gates). */
 int gdn_oracle_update(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                       const uint16_t *a, const uint16_t *b,
                       const float *A_log, const float *dt_bias,
+                      const float *g, const float *beta,
                       const float *state_in, const int32_t *state_indices,
                       const int32_t *cu_seqlens,
                       int32_t N, int32_t T_fixed, int32_t T_tot,
@@ -88,12 +94,34 @@ int gdn_oracle_update(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 int gdn_oracle_update_f32(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           const uint16_t *a, const uint16_t *b,
                           const float *A_log, const float *dt_bias,
+                          const float *g, const float *beta,
                           const float *state_in, const int32_t *state_indices,
                           const int32_t *cu_seqlens,
                           int32_t N, int32_t T_fixed, int32_t T_tot,
                           int32_t H, int32_t HV, int32_t K, int32_t V,
                           int32_t num_slots, double scale, uint32_t flags,
                           float *out, float *state_out, float *inter);
+
+/* The fp64 oracle with q, k, v, a, b given as fp32 values. */
+int gdn_oracle_update_fin(const float *q, const float *k, const float *v,
+                          const float *a, const float *b,
+                          const float *A_log, const float *dt_bias,
+                          const float *g, const float *beta,
+                          const float *state_in, const int32_t *state_indices,
+                          const int32_t *cu_seqlens,
+                          int32_t N, int32_t T_fixed, int32_t T_tot,
+                          int32_t H, int32_t HV, int32_t K, int32_t V,
+                          int32_t num_slots, double scale, uint32_t flags,
+                          double *out, double *state_out, double *inter);
+
+/* The gating step alone: g = -exp(A_log) softplus(a + dt_bias) and
+ * beta = sigmoid(b) for every (token, value head), [T_tot, HV] each. */
+int gdn_oracle_gating(const uint16_t *a, const uint16_t *b, const float *A_log, const float *dt_bias,
+                      int32_t T_tot, int32_t HV, double *g, double *beta);
+int gdn_oracle_gating_f32(const uint16_t *a, const uint16_t *b, const float *A_log, const float *dt_bias,
+                          int32_t T_tot, int32_t HV, float *g, float *beta);
+int gdn_oracle_gating_fin(const float *a, const float *b, const float *A_log, const float *dt_bias,
+                          int32_t T_tot, int32_t HV, double *g, double *beta);
 
 #ifdef __cplusplus
 }

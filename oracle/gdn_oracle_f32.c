@@ -5,4 +5,5 @@
  */
 #define GDN_ORACLE_REAL float
 #define GDN_ORACLE_FN gdn_oracle_update_f32
+#define GDN_ORACLE_GATING_FN gdn_oracle_gating_f32
 #include "gdn_oracle.c"

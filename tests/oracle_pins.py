@@ -396,10 +396,97 @@ def pin_softplus_large_argument(library=None):
         np.testing.assert_allclose(st[s], np.exp(-25.0) * p["state_pool"][s].astype(np.float64), rtol=1e-15)
 
 
+# --------------------------------------------------------------------------
+# The unfused pair (gating alone; recurrence with given g, beta) and fp32 inputs
+# --------------------------------------------------------------------------
+
+def _pin_golden_given(name, g_value, library):
+    """A golden case through the given-gates recurrence: g and beta passed
+    as arrays with the values the case derives."""
+    case = load_golden(name)
+    p = golden_arrays(case)
+    T = len(case["tokens"])
+    g = np.full((T, 1), g_value, dtype=np.float32)
+    beta = np.full((T, 1), 0.5, dtype=np.float32)
+    flags = INTER | (L2 if case["l2norm"] else 0)
+    scale = None if case["l2norm"] else case["scale"]
+    status, out, st, inter = oracle.update(p["q"], p["k"], p["v"], None, None, None, None, p["state_pool"],
+                                           p["state_indices"], None, scale=scale, flags=flags, g=g, beta=beta,
+                                           library=library)
+    assert status == 0
+    tol = case["tolerance_abs"]
+    np.testing.assert_allclose(out.reshape(T, -1), np.array(case["expected_out"]), rtol=0, atol=tol)
+    np.testing.assert_allclose(inter.reshape(T, case["K"], case["V"]), np.array(case["expected_inter"]),
+                               rtol=0, atol=tol)
+
+
+def pin_given_gates_golden(library=None):
+    """decay 1/4 is g = ln(1/4) (rounded to fp32: 4e-9 relative), beta 1/2;
+    no decay is g = 0."""
+    _pin_golden_given("k4v4_two_tokens_decay_quarter.json", np.log(0.25), library)
+    _pin_golden_given("k4v4_l2norm_no_decay.json", 0.0, library)
+
+
+def pin_gating_closed_forms(library=None):
+    """softplus(0) = ln 2 (a = -dt_bias), softplus(2) = ln(1 + e^2),
+    softplus(-inf) = 0, the threshold branch (x = 25), sigmoid(0) = 1/2,
+    sigmoid(+-inf) = 1 / 0."""
+    a = np.stack([bf16([1.0, 1.0, 24.0]), np.array([BF16_NEG_INF, bf16(1.0), bf16(1.0)], dtype=np.uint16)])
+    b = np.stack([np.array([0, BF16_POS_INF, BF16_NEG_INF], dtype=np.uint16), bf16([0.0, 0.0, 0.0])])
+    A_log = np.array([0.0, np.log(2.0), 0.0], dtype=np.float32)
+    dt_bias = np.array([-1.0, -1.0, 1.0], dtype=np.float32)
+    g, beta = oracle.gating(a, b, A_log, dt_bias, library=library)
+    e2 = float(np.exp(np.float64(np.float32(np.log(2.0)))))
+    np.testing.assert_allclose(g[0], [-np.log(2.0), -e2 * np.log(2.0), -25.0], rtol=1e-15)
+    assert g[1, 0] == 0.0
+    np.testing.assert_allclose(g[1, 1:], [-e2 * np.log(2.0), -np.log(1.0 + np.e ** 2)], rtol=1e-15)
+    assert list(beta[0]) == [0.5, 1.0, 0.0] and list(beta[1]) == [0.5, 0.5, 0.5]
+
+
+def pin_fused_equals_gating_then_given(library=None):
+    """The fused update equals the unfused pair: gates from the gating step
+    (rounded to fp32, as the pair stores them), then the recurrence with
+    given gates."""
+    rng = np.random.default_rng(24)
+    p = random_problem(rng, lens=[3, 1, 4], H=2, HV=4, K=8, V=8, pad=(1,))
+    _, o_f, s_f, i_f = _run(p, library, flags=L2 | INTER)
+    g, beta = oracle.gating(p["a"], p["b"], p["A_log"], p["dt_bias"], library=library)
+    status, o_u, s_u, i_u = oracle.update(p["q"], p["k"], p["v"], None, None, None, None, p["state_pool"],
+                                          p["state_indices"], p["cu_seqlens"], flags=L2 | INTER,
+                                          g=g.astype(np.float32), beta=beta.astype(np.float32), library=library)
+    assert status == 0
+    np.testing.assert_allclose(o_u, o_f, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(s_u, s_f, rtol=1e-5, atol=1e-6)
+    assert np.array_equal(np.isnan(i_u), np.isnan(i_f))
+
+
+def pin_fp32_inputs_equal_bf16_inputs(library=None):
+    """The same values given as fp32 instead of bf16 patterns give the same
+    bits (the arithmetic is fp64 either way)."""
+    rng = np.random.default_rng(25)
+    p = random_problem(rng, lens=[2, 3], H=2, HV=4, K=8, V=8)
+    ref = _run(p, library, flags=L2 | INTER)
+    pf = dict(p)
+    for n in ("q", "k", "v", "a", "b"):
+        pf[n] = bf16_bits_to_f32(p[n])
+    got = _run(pf, library, flags=L2 | INTER)
+    for x, y in zip(ref[1:], got[1:]):
+        assert np.array_equal(x, y, equal_nan=True)
+    g1, b1 = oracle.gating(p["a"], p["b"], p["A_log"], p["dt_bias"], library=library)
+    g2, b2 = oracle.gating(pf["a"], pf["b"], p["A_log"], p["dt_bias"], library=library)
+    assert np.array_equal(g1, g2) and np.array_equal(b1, b2)
+    # fp32 values that are not bf16 values go through unrounded
+    pf["v"] = pf["v"] + np.float32(1.0 / 3.0)
+    _, o3, _, _ = _run(pf, library, flags=L2 | INTER)
+    assert not np.array_equal(o3, got[1])
+
+
 ALL_PINS = [
     pin_golden_decay_quarter, pin_golden_l2norm_no_decay, pin_gating_pattern,
     pin_unit_k_recall, pin_no_decay_rows, pin_zero_state_one_token,
     pin_chain_equals_multi_token, pin_intermediate_prefix, pin_gqa_decomposition,
     pin_heads_independent, pin_slot_permutation, pin_padding_and_untouched,
     pin_invalid_and_empty, pin_no_final_writeback, pin_softplus_large_argument,
+    pin_given_gates_golden, pin_gating_closed_forms, pin_fused_equals_gating_then_given,
+    pin_fp32_inputs_equal_bf16_inputs,
 ]

@@ -32,10 +32,17 @@ MUTANTS = [
     ("scale_on_k_too", "k_hat[r] = bf16_bits_to_real(k_row[r]) * k_norm;",
      "k_hat[r] = bf16_bits_to_real(k_row[r]) * k_norm * (real)scale;"),
     ("decay_dropped", "S[e] *= decay;", "S[e] *= 1;"),
-    ("g_sign", "const real g = -exp((real)A_log[hv]) * softplus(x);",
-     "const real g = exp((real)A_log[hv]) * softplus(x);"),
-    ("A_log_not_exponentiated", "const real g = -exp((real)A_log[hv]) * softplus(x);",
-     "const real g = -(real)A_log[hv] * softplus(x);"),
+    ("g_sign", "g = -exp((real)A_log[hv]) * softplus(x);",
+     "g = exp((real)A_log[hv]) * softplus(x);"),
+    ("A_log_not_exponentiated", "g = -exp((real)A_log[hv]) * softplus(x);",
+     "g = -(real)A_log[hv] * softplus(x);"),
+    ("given_g_sign", "g = (real)g_in[(size_t)tok * HV + hv];", "g = -(real)g_in[(size_t)tok * HV + hv];"),
+    ("given_beta_ignored", "beta = (real)beta_in[(size_t)tok * HV + hv];", "beta = 1;"),
+    ("given_g_indexed_by_head_only", "g = (real)g_in[(size_t)tok * HV + hv];", "g = (real)g_in[hv];"),
+    ("gating_beta_complement", "beta_out[(size_t)tok * HV + hv] = sigmoid(", "beta_out[(size_t)tok * HV + hv] = 1 - sigmoid("),
+    ("gating_g_unscaled", "g_out[(size_t)tok * HV + hv] = -exp((real)A_log[hv]) * softplus(x);",
+     "g_out[(size_t)tok * HV + hv] = -softplus(x);"),
+    ("fp32_inputs_truncated", "    return (real)x;", "    return (real)(int)x;"),
     ("dt_bias_dropped", "+ (real)dt_bias[hv];", ";"),
     ("softplus_is_identity", "return log1p(exp(x));", "return log(exp(x));"),
     ("sigmoid_sign", "return (real)1 / ((real)1 + exp(-x));", "return (real)1 / ((real)1 + exp(x));"),
@@ -54,7 +61,7 @@ MUTANTS = [
 def _build_mutant(tmpdir, name, old, new):
     d = os.path.join(tmpdir, name)
     os.makedirs(d)
-    for f in ("gdn_oracle.c", "gdn_oracle_f32.c", "gdn_oracle.h"):
+    for f in ("gdn_oracle.c", "gdn_oracle_f32.c", "gdn_oracle_fin.c", "gdn_oracle.h"):
         shutil.copy(os.path.join(SRC, f), d)
     path = os.path.join(d, "gdn_oracle.c")
     text = open(path).read()
@@ -62,7 +69,8 @@ def _build_mutant(tmpdir, name, old, new):
     open(path, "w").write(text.replace(old, new))
     lib = os.path.join(d, "libmutant.so")
     subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-w",
-                    "-o", lib, os.path.join(d, "gdn_oracle.c"), os.path.join(d, "gdn_oracle_f32.c"), "-lm"],
+                    "-o", lib, os.path.join(d, "gdn_oracle.c"), os.path.join(d, "gdn_oracle_f32.c"),
+                    os.path.join(d, "gdn_oracle_fin.c"), "-lm"],
                    check=True)
     return lib
 
