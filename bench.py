@@ -255,6 +255,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the two-kernel pair (gating, then the recurrence) instead of the fused update")
     ap.add_argument("--no-pdl", dest="pdl", action="store_false",
                     help="launch in plain stream order instead of with programmatic dependent launch")
     args = ap.parse_args()
@@ -292,11 +294,20 @@ def main():
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
     if args.pdl:
         flags |= binding.LAUNCH_PDL
-    calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"], c["state_pool"],
-                                  c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
-                                  intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
-                                  schedule=schedule, tile_rows=args.tile_rows)
-             for c in copies]
+    if args.unfused:
+        # the two-kernel baseline the fused update replaces (gating, then the
+        # recurrence reading g and beta back from HBM)
+        calls = [binding.PreparedUnfusedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
+                                             c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"],
+                                             flags=flags, intermediate_states=c.get("inter"), stream=stream,
+                                             tile_v=args.tile_v, tile_rows=args.tile_rows)
+                 for c in copies]
+    else:
+        calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
+                                      c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
+                                      intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
+                                      schedule=schedule, tile_rows=args.tile_rows)
+                 for c in copies]
     nbytes = wl.algorithmic_bytes(w)
     torch.cuda.synchronize(device)
 
@@ -373,7 +384,7 @@ def main():
         peak, peak_src = hbm_peak()
         achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
         traffic = None
-        if NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash():
+        if NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash() and not args.unfused:
             traffic = NCU_TRAFFIC["bytes_per_launch"]
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -386,11 +397,12 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
-                         "kernel": kernel_name(schedule, args.tile_v, args.tile_rows,
+                         "kernel": ("gdn::gdn_gating_kernel + " if args.unfused else "") +
+                                   kernel_name(schedule, args.tile_v, args.tile_rows,
                                                w.T_tot == w.spec.N and not w.spec.intermediate,
                                                w.spec.N * w.spec.HV)},
             "e2e": e2e,
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * (2 if args.unfused else 1),
             "clocks": clocks,
         }
         if world == 1 and not args.skip_cpu_baseline:

@@ -9,14 +9,15 @@ missing: there is no CPU or library fallback.
 """
 from __future__ import annotations
 
-__all__ = ["decode_update", "binding", "workloads"]
+__all__ = ["decode_update", "recurrent_update", "gating", "binding", "workloads"]
 
 
 def __getattr__(name):
     # Lazy: importing the package (e.g. for ``workloads``) must not need the
     # CUDA library; calling into it must.
-    if name in ("decode_update", "decode_update_host", "GdnError", "L2NORM_QK",
-                "WRITE_INTERMEDIATE", "NO_FINAL_WRITEBACK", "CHECK_INDICES"):
+    if name in ("decode_update", "decode_update_host", "recurrent_update", "gating", "PreparedCall",
+                "HostStagedDecode", "GdnError", "L2NORM_QK", "WRITE_INTERMEDIATE", "NO_FINAL_WRITEBACK",
+                "CHECK_INDICES", "LAUNCH_PDL"):
         from . import binding
         return getattr(binding, name)
     if name in ("binding", "workloads", "build"):

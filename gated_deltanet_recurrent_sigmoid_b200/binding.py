@@ -76,6 +76,10 @@ def load() -> ctypes.CDLL:
         P = ctypes.POINTER(GdnTensor)
         lib.gdn_decode_update.restype = ctypes.c_int
         lib.gdn_decode_update.argtypes = [P] * 11 + [ctypes.c_float, ctypes.c_uint32, ctypes.POINTER(GdnExtra)]
+        lib.gdn_recurrent_update.restype = ctypes.c_int
+        lib.gdn_recurrent_update.argtypes = [P] * 9 + [ctypes.c_float, ctypes.c_uint32, ctypes.POINTER(GdnExtra)]
+        lib.gdn_gating.restype = ctypes.c_int
+        lib.gdn_gating.argtypes = [P] * 6 + [ctypes.POINTER(GdnExtra)]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_version.restype = ctypes.c_int
@@ -145,6 +149,54 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     if status != OK:
         raise GdnError(status, status_string(status))
     return out
+
+
+def recurrent_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                     state_pool: torch.Tensor, state_indices: torch.Tensor, cu_seqlens: Optional[torch.Tensor],
+                     out: torch.Tensor, scale: Optional[float] = None, flags: int = L2NORM_QK,
+                     intermediate_states: Optional[torch.Tensor] = None,
+                     device_status: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                     tile_v: int = 0, schedule: int = SCHEDULE_AUTO, tile_rows: int = 0) -> torch.Tensor:
+    """The recurrence of the unfused pair with precomputed gates
+    (``gdn_recurrent_update``): decay = exp(g), beta given per (token, value
+    head).  Arguments otherwise as ``decode_update``."""
+    lib = load()
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if intermediate_states is not None:
+        flags |= WRITE_INTERMEDIATE
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    descs = [describe(t) for t in (q, k, v, g, beta, state_pool, state_indices, cu_seqlens, out)]
+    inter = describe(intermediate_states)
+    extra = GdnExtra()
+    extra.stream = stream.cuda_stream if stream is not None else None
+    extra.intermediate_states = ctypes.pointer(inter) if inter is not None else None
+    extra.device_status = device_status.data_ptr() if device_status is not None else None
+    extra.tile_v = int(tile_v)
+    extra.tile_rows = int(tile_rows)
+    extra.schedule = int(schedule)
+    status = lib.gdn_recurrent_update(*[_ref(d) for d in descs], ctypes.c_float(scale), ctypes.c_uint32(flags),
+                                      ctypes.byref(extra))
+    if status != OK:
+        raise GdnError(status, status_string(status))
+    return out
+
+
+def gating(A_log: torch.Tensor, a: torch.Tensor, dt_bias: torch.Tensor, b: torch.Tensor, g: torch.Tensor,
+           beta: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> tuple:
+    """The gating step alone (``gdn_gating``): g = -exp(A_log) softplus(a +
+    dt_bias) (fp32) and beta = sigmoid(b) into the given [T_tot, HV] tensors."""
+    lib = load()
+    if stream is None:
+        stream = torch.cuda.current_stream(a.device) if a.is_cuda else None
+    descs = [describe(t) for t in (A_log, a, dt_bias, b, g, beta)]
+    extra = GdnExtra()
+    extra.stream = stream.cuda_stream if stream is not None else None
+    status = lib.gdn_gating(*[_ref(d) for d in descs], ctypes.byref(extra))
+    if status != OK:
+        raise GdnError(status, status_string(status))
+    return g, beta
 
 
 def decode_update_host(host: dict, device: dict, *, scale: Optional[float] = None, flags: int = L2NORM_QK,
@@ -272,3 +324,53 @@ class HostStagedDecode:
             self._call()
             self.out_host.copy_(self.out_device, non_blocking=True)
         return self.out_host
+
+
+class PreparedUnfusedCall:
+    """The unfused pair as one prepared step: the gating kernel writes g and
+    beta (fp32, [T_tot, HV], owned here) and the recurrence reads them --
+    two launches and one round trip of the gates through HBM, which is what
+    the fused update saves.  Arguments as ``PreparedCall``."""
+
+    def __init__(self, q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
+                 scale: Optional[float] = None, flags: int = L2NORM_QK, intermediate_states=None,
+                 device_status=None, stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
+                 tile_rows: int = 0):
+        lib = load()
+        lead = q.shape[:-2]
+        HV = v.shape[-2]
+        self.g = torch.empty(math.prod(lead), HV, dtype=torch.float32, device=q.device)
+        self.beta = torch.empty_like(self.g)
+        a2, b2 = a.reshape(-1, HV), b.reshape(-1, HV)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(q.device)
+        if scale is None:
+            scale = 1.0 / math.sqrt(q.shape[-1])
+        if intermediate_states is not None:
+            flags |= WRITE_INTERMEDIATE
+        self._keep = (q, k, v, a2, b2, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
+                      intermediate_states, device_status)
+        self._gd = [describe(t) for t in (A_log, a2, dt_bias, b2, self.g, self.beta)]
+        g_view, beta_view = self.g.view(*lead, HV), self.beta.view(*lead, HV)
+        self._keep2 = (g_view, beta_view)
+        self._rd = [describe(t) for t in (q, k, v, g_view, beta_view, state_pool, state_indices, cu_seqlens, out)]
+        self._inter = describe(intermediate_states)
+        self._gx = GdnExtra()
+        self._gx.stream = self.stream.cuda_stream
+        self._rx = GdnExtra()
+        self._rx.stream = self.stream.cuda_stream
+        self._rx.intermediate_states = ctypes.pointer(self._inter) if self._inter is not None else None
+        self._rx.device_status = device_status.data_ptr() if device_status is not None else None
+        self._rx.tile_v = int(tile_v)
+        self._rx.tile_rows = int(tile_rows)
+        self._gargs = [_ref(d) for d in self._gd] + [ctypes.byref(self._gx)]
+        self._rargs = [_ref(d) for d in self._rd] + [ctypes.c_float(scale), ctypes.c_uint32(flags),
+                                                     ctypes.byref(self._rx)]
+        self._gating = lib.gdn_gating
+        self._recurrent = lib.gdn_recurrent_update
+
+    def __call__(self) -> None:
+        status = self._gating(*self._gargs)
+        if status == OK:
+            status = self._recurrent(*self._rargs)
+        if status != OK:
+            raise GdnError(status, status_string(status))

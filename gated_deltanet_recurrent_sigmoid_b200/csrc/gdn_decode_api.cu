@@ -63,12 +63,13 @@ bool overlap(const Span &x, const Span &y)
 }
 
 // Basic descriptor sanity: rank, non-negative shape and strides, and a data
-// pointer unless the tensor has no elements.
-int check_desc(const gdn_tensor *t, int32_t dtype)
+// pointer unless the tensor has no elements.  `dtype2` is a second accepted
+// element type (0: none).
+int check_desc(const gdn_tensor *t, int32_t dtype, int32_t dtype2 = 0)
 {
     if (!t)
         return GDN_ERR_NULL_ARG;
-    if (t->dtype != dtype)
+    if (t->dtype != dtype && (dtype2 == 0 || t->dtype != dtype2))
         return GDN_ERR_DTYPE;
     if (t->ndim < 1 || t->ndim > 4)
         return GDN_ERR_SHAPE;
@@ -193,12 +194,27 @@ cudaError_t launch_ex(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStr
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <int BV, int KG>
+template <int BV, int KG, typename TAct, bool GIVEN>
 cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl)
 {
     using TS = gdn::TileShape<kHeadK, kHeadV, BV, KG>;
     const dim3 grid(static_cast<unsigned>(units * TS::NV));
-    return launch_ex(gdn::gdn_decode_kernel<kHeadK, kHeadV, BV, KG>, grid, dim3(TS::THREADS), 0, stream, pdl, p);
+    return launch_ex(gdn::gdn_decode_kernel<kHeadK, kHeadV, BV, KG, TAct, GIVEN>, grid, dim3(TS::THREADS), 0,
+                     stream, pdl, p);
+}
+
+// The tile table: (V-tile width, rows per thread) -> (BV, KG = K / rows).
+template <typename TAct, bool GIVEN>
+cudaError_t launch_tile(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, int tile_v,
+                        int tile_rows)
+{
+    switch (tile_v * 100 + tile_rows) {
+    case 1616: return launch<16, 8, TAct, GIVEN>(p, units, stream, pdl);
+    case 3216: return launch<32, 8, TAct, GIVEN>(p, units, stream, pdl);
+    case 3232: return launch<32, 4, TAct, GIVEN>(p, units, stream, pdl);
+    case 6416: return launch<64, 8, TAct, GIVEN>(p, units, stream, pdl);
+    default: return launch<64, 4, TAct, GIVEN>(p, units, stream, pdl);
+    }
 }
 
 constexpr int kPipeStages = 3;
@@ -236,39 +252,31 @@ cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStre
                      dim3(gdn::pipe::THREADS), smem, stream, pdl, p);
 }
 
-}  // namespace
+// Everything one update call needs; the fused and the given-gate entry
+// points differ only in where decay and beta come from.
+struct UpdateArgs {
+    const gdn_tensor *q, *k, *v, *out;
+    bool given_gates;
+    const gdn_tensor *gate_a, *gate_b;   // fused: a, b; given: g, beta
+    const gdn_tensor *A_log, *dt_bias;   // fused only
+    const gdn_tensor *state_pool, *state_indices, *cu_seqlens;
+    float scale;
+    uint32_t flags;
+    const gdn_extra *extra;
+};
 
-extern "C" {
-
-GDN_API int gdn_version(void) { return GDN_DECODE_ABI_VERSION; }
-
-GDN_API const char *gdn_status_string(int status)
+int run_update(const UpdateArgs &c)
 {
-    switch (status) {
-    case GDN_OK: return "GDN_OK: success";
-    case GDN_ERR_NULL_ARG: return "GDN_ERR_NULL_ARG: a required tensor or pointer is NULL";
-    case GDN_ERR_DTYPE: return "GDN_ERR_DTYPE: a tensor has the wrong dtype";
-    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: a tensor has the wrong rank, shape or strides";
-    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: a pointer or stride breaks an alignment rule";
-    case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: a written tensor overlaps another tensor";
-    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: head size or V-tile not built";
-    case GDN_ERR_ARG: return "GDN_ERR_ARG: bad scalar argument or flag";
-    case GDN_ERR_INDICES: return "GDN_ERR_INDICES: bad or repeated state index, or bad cu_seqlens";
-    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: the CUDA runtime refused the launch or copy";
-    default: return "unknown gdn status";
-    }
-}
+    const gdn_tensor *q = c.q, *k = c.k, *v = c.v, *out = c.out, *ga = c.gate_a, *gb = c.gate_b;
+    const gdn_tensor *A_log = c.A_log, *dt_bias = c.dt_bias, *state_pool = c.state_pool;
+    const gdn_tensor *state_indices = c.state_indices, *cu_seqlens = c.cu_seqlens;
+    const gdn_extra *extra = c.extra;
+    const uint32_t flags = c.flags;
 
-GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
-                              const gdn_tensor *a, const gdn_tensor *b, const gdn_tensor *A_log,
-                              const gdn_tensor *dt_bias, const gdn_tensor *state_pool,
-                              const gdn_tensor *state_indices, const gdn_tensor *cu_seqlens,
-                              const gdn_tensor *out, float scale, uint32_t flags, const gdn_extra *extra)
-{
     // ---- scalars and flags
     const uint32_t known =
         GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES | GDN_LAUNCH_PDL;
-    if ((flags & ~known) != 0 || !std::isfinite(scale) || !(scale > 0.f))
+    if ((flags & ~known) != 0 || !std::isfinite(c.scale) || !(c.scale > 0.f))
         return GDN_ERR_ARG;
     const int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
     if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED)
@@ -281,21 +289,28 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         return GDN_ERR_NULL_ARG;
 
     // ---- descriptors and dtypes
-    GDN_TRY(check_desc(q, GDN_DTYPE_BF16));
-    GDN_TRY(check_desc(k, GDN_DTYPE_BF16));
-    GDN_TRY(check_desc(v, GDN_DTYPE_BF16));
-    GDN_TRY(check_desc(a, GDN_DTYPE_BF16));
-    GDN_TRY(check_desc(b, GDN_DTYPE_BF16));
-    GDN_TRY(check_desc(A_log, GDN_DTYPE_F32));
-    GDN_TRY(check_desc(dt_bias, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(q, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+    const int32_t act = q->dtype;
+    GDN_TRY(check_desc(k, act));
+    GDN_TRY(check_desc(v, act));
+    GDN_TRY(check_desc(out, act));
+    if (c.given_gates) {
+        GDN_TRY(check_desc(ga, GDN_DTYPE_F32));
+        GDN_TRY(check_desc(gb, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+    } else {
+        GDN_TRY(check_desc(ga, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+        GDN_TRY(check_desc(gb, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+        GDN_TRY(check_desc(A_log, GDN_DTYPE_F32));
+        GDN_TRY(check_desc(dt_bias, GDN_DTYPE_F32));
+    }
     GDN_TRY(check_desc(state_pool, GDN_DTYPE_F32));
     GDN_TRY(check_desc(state_indices, GDN_DTYPE_I32));
-    GDN_TRY(check_desc(out, GDN_DTYPE_BF16));
     if (cu_seqlens)
         GDN_TRY(check_desc(cu_seqlens, GDN_DTYPE_I32));
     if (want_inter)
         GDN_TRY(check_desc(inter, GDN_DTYPE_F32));
     const bool varlen = cu_seqlens != nullptr;
+    const int64_t act_size = elem_size(act);
 
     // ---- shapes
     if (state_indices->ndim != 1 || q->ndim < 3 || q->ndim > 4)
@@ -313,10 +328,10 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     GDN_TRY(token_layout(k, 2, varlen, N, &Lk));
     GDN_TRY(token_layout(v, 2, varlen, N, &Lv));
     GDN_TRY(token_layout(out, 2, varlen, N, &Lo));
-    if (a->ndim != q->ndim - 1 || b->ndim != q->ndim - 1 || out->ndim != q->ndim || k->ndim != q->ndim)
+    if (ga->ndim != q->ndim - 1 || gb->ndim != q->ndim - 1 || out->ndim != q->ndim || k->ndim != q->ndim)
         return GDN_ERR_SHAPE;
-    GDN_TRY(token_layout(a, 1, varlen, N, &La));
-    GDN_TRY(token_layout(b, 1, varlen, N, &Lb));
+    GDN_TRY(token_layout(ga, 1, varlen, N, &La));
+    GDN_TRY(token_layout(gb, 1, varlen, N, &Lb));
     const int64_t T_tot = Lq.T_tot;
     if (Lk.T_tot != T_tot || Lv.T_tot != T_tot || Lo.T_tot != T_tot || La.T_tot != T_tot || Lb.T_tot != T_tot)
         return GDN_ERR_SHAPE;
@@ -324,9 +339,10 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         return GDN_ERR_SHAPE;
     if (out->shape[out->ndim - 2] != HV || out->shape[out->ndim - 1] != V)
         return GDN_ERR_SHAPE;
-    if (a->shape[a->ndim - 1] != HV || b->shape[b->ndim - 1] != HV)
+    if (ga->shape[ga->ndim - 1] != HV || gb->shape[gb->ndim - 1] != HV)
         return GDN_ERR_SHAPE;
-    if (A_log->ndim != 1 || A_log->shape[0] != HV || dt_bias->ndim != 1 || dt_bias->shape[0] != HV)
+    if (!c.given_gates &&
+        (A_log->ndim != 1 || A_log->shape[0] != HV || dt_bias->ndim != 1 || dt_bias->shape[0] != HV))
         return GDN_ERR_SHAPE;
     if (state_pool->ndim != 4 || state_pool->shape[1] != HV || state_pool->shape[2] != K ||
         state_pool->shape[3] != V)
@@ -341,7 +357,8 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         (!varlen && Lq.T > INT32_MAX))
         return GDN_ERR_SHAPE;
 
-    // ---- contiguity and alignment
+    // ---- contiguity and alignment: q/k rows are read 16 bytes at a time,
+    // v/out 4 elements at a time, the state 16 bytes at a time
     if (q->stride[q->ndim - 1] != 1 || k->stride[k->ndim - 1] != 1 || v->stride[v->ndim - 1] != 1 ||
         out->stride[out->ndim - 1] != 1)
         return GDN_ERR_SHAPE;
@@ -353,18 +370,21 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         return GDN_ERR_SHAPE;
     if (varlen && cu_seqlens->stride[0] != 1)
         return GDN_ERR_SHAPE;
+    const int64_t qk_mult = 16 / act_size;
     for (const gdn_tensor *t : {q, k}) {
-        if (!aligned(t->data, 16) || !stride_ok(T_tot, t == q ? Lq.tok : Lk.tok, 8) ||
-            !stride_ok(H, t->stride[t->ndim - 2], 8))
+        if (!aligned(t->data, 16) || !stride_ok(T_tot, t == q ? Lq.tok : Lk.tok, qk_mult) ||
+            !stride_ok(H, t->stride[t->ndim - 2], qk_mult))
             return GDN_ERR_ALIGN;
     }
     for (const gdn_tensor *t : {v, out}) {
-        if (!aligned(t->data, 8) || !stride_ok(T_tot, t == v ? Lv.tok : Lo.tok, 4) ||
+        if (!aligned(t->data, static_cast<uintptr_t>(4 * act_size)) || !stride_ok(T_tot, t == v ? Lv.tok : Lo.tok, 4) ||
             !stride_ok(HV, t->stride[t->ndim - 2], 4))
             return GDN_ERR_ALIGN;
     }
-    if (!aligned(a->data, 2) || !aligned(b->data, 2) || !aligned(A_log->data, 4) || !aligned(dt_bias->data, 4) ||
+    if (!aligned(ga->data, elem_size(ga->dtype)) || !aligned(gb->data, elem_size(gb->dtype)) ||
         !aligned(state_indices->data, 4) || (varlen && !aligned(cu_seqlens->data, 4)))
+        return GDN_ERR_ALIGN;
+    if (!c.given_gates && (!aligned(A_log->data, 4) || !aligned(dt_bias->data, 4)))
         return GDN_ERR_ALIGN;
     if (!aligned(state_pool->data, 16) || !stride_ok(num_slots, state_pool->stride[0], 4) ||
         !stride_ok(HV, state_pool->stride[1], 4))
@@ -378,7 +398,8 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     // ---- aliasing: nothing written may overlap anything else
     {
         const Span s_out = span_of(out), s_pool = span_of(state_pool), s_inter = want_inter ? span_of(inter) : Span{};
-        const gdn_tensor *inputs[] = {q, k, v, a, b, A_log, dt_bias, state_indices, cu_seqlens};
+        const gdn_tensor *inputs[] = {q, k, v, ga, gb, c.given_gates ? nullptr : A_log,
+                                      c.given_gates ? nullptr : dt_bias, state_indices, cu_seqlens};
         for (const gdn_tensor *t : inputs) {
             if (!t)
                 continue;
@@ -420,6 +441,12 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
         tile_v = 16;
         tile_rows = 16;
     }
+    if (act == GDN_DTYPE_F32) {
+        // fp32 q/k rows double the prefetch registers: 16 rows per thread
+        // keep every fp32 tile free of spills
+        tile_v = one_token ? 32 : 16;
+        tile_rows = 16;
+    }
     if (extra && extra->tile_v) {
         tile_v = extra->tile_v;
         tile_rows = extra->tile_rows ? extra->tile_rows : 16;
@@ -429,6 +456,10 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     const bool tile_ok = (tile_v == 16 && tile_rows == 16) || (tile_v == 32 && (tile_rows == 16 || tile_rows == 32)) ||
                          (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
     if (!tile_ok)
+        return GDN_ERR_UNSUPPORTED;
+    // The pipelined schedule is built for bf16 activations and fused bf16 gates.
+    if (schedule == GDN_SCHEDULE_PIPELINED &&
+        (act != GDN_DTYPE_BF16 || c.given_gates || ga->dtype != GDN_DTYPE_BF16 || gb->dtype != GDN_DTYPE_BF16))
         return GDN_ERR_UNSUPPORTED;
     const int64_t units = N * HV;
     if (units * (kHeadV / tile_v) > INT32_MAX)
@@ -446,17 +477,17 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     // ---- parameters
     gdn::DecodeParams p;
     std::memset(&p, 0, sizeof p);
-    p.q = static_cast<const __nv_bfloat16 *>(q->data);
-    p.k = static_cast<const __nv_bfloat16 *>(k->data);
-    p.v = static_cast<const __nv_bfloat16 *>(v->data);
-    p.a = static_cast<const __nv_bfloat16 *>(a->data);
-    p.b = static_cast<const __nv_bfloat16 *>(b->data);
-    p.A_log = static_cast<const float *>(A_log->data);
-    p.dt_bias = static_cast<const float *>(dt_bias->data);
+    p.q = q->data;
+    p.k = k->data;
+    p.v = v->data;
+    p.a = ga->data;
+    p.b = gb->data;
+    p.A_log = c.given_gates ? nullptr : static_cast<const float *>(A_log->data);
+    p.dt_bias = c.given_gates ? nullptr : static_cast<const float *>(dt_bias->data);
     p.state = static_cast<float *>(state_pool->data);
     p.indices = static_cast<const int32_t *>(state_indices->data);
     p.cu_seqlens = varlen ? static_cast<const int32_t *>(cu_seqlens->data) : nullptr;
-    p.out = static_cast<__nv_bfloat16 *>(out->data);
+    p.out = out->data;
     p.inter = want_inter ? static_cast<float *>(inter->data) : nullptr;
     p.status = extra ? extra->device_status : nullptr;
     p.q_tok = Lq.tok;
@@ -468,11 +499,11 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     p.o_tok = Lo.tok;
     p.o_head = out->stride[out->ndim - 2];
     p.a_tok = La.tok;
-    p.a_head = a->stride[a->ndim - 1];
+    p.a_head = ga->stride[ga->ndim - 1];
     p.b_tok = Lb.tok;
-    p.b_head = b->stride[b->ndim - 1];
-    p.A_stride = A_log->stride[0];
-    p.dt_stride = dt_bias->stride[0];
+    p.b_head = gb->stride[gb->ndim - 1];
+    p.A_stride = c.given_gates ? 0 : A_log->stride[0];
+    p.dt_stride = c.given_gates ? 0 : dt_bias->stride[0];
     p.s_slot = state_pool->stride[0];
     p.s_head = state_pool->stride[1];
     p.i_tok = want_inter ? inter->stride[0] : 0;
@@ -483,25 +514,132 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
     p.HV = static_cast<int32_t>(HV);
     p.G = static_cast<int32_t>(HV / H);
     p.num_slots = static_cast<int32_t>(num_slots);
-    p.scale = scale;
+    p.a_f32 = ga->dtype == GDN_DTYPE_F32;
+    p.b_f32 = gb->dtype == GDN_DTYPE_F32;
+    p.scale = c.scale;
     p.flags = flags;
 
-    // Library choice: the per-tile schedule (measured faster on every
-    // workload shape); the pipelined one only on request.
     const bool pdl = (flags & GDN_LAUNCH_PDL) != 0;
     cudaError_t err;
-    if (schedule == GDN_SCHEDULE_PIPELINED) {
+    if (schedule == GDN_SCHEDULE_PIPELINED)
         err = launch_pipelined(p, units, stream, pdl);
-    } else {
-        // KG (row groups per tile) = K / tile_rows
-        switch (tile_v * 100 + tile_rows) {
-        case 1616: err = launch<16, 8>(p, units, stream, pdl); break;
-        case 3216: err = launch<32, 8>(p, units, stream, pdl); break;
-        case 3232: err = launch<32, 4>(p, units, stream, pdl); break;
-        case 6416: err = launch<64, 8>(p, units, stream, pdl); break;
-        default: err = launch<64, 4>(p, units, stream, pdl); break;
-        }
+    else if (act == GDN_DTYPE_BF16)
+        err = c.given_gates ? launch_tile<__nv_bfloat16, true>(p, units, stream, pdl, tile_v, tile_rows)
+                            : launch_tile<__nv_bfloat16, false>(p, units, stream, pdl, tile_v, tile_rows);
+    else
+        err = c.given_gates ? launch_tile<float, true>(p, units, stream, pdl, tile_v, tile_rows)
+                            : launch_tile<float, false>(p, units, stream, pdl, tile_v, tile_rows);
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+GDN_API int gdn_version(void) { return GDN_DECODE_ABI_VERSION; }
+
+GDN_API const char *gdn_status_string(int status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK: success";
+    case GDN_ERR_NULL_ARG: return "GDN_ERR_NULL_ARG: a required tensor or pointer is NULL";
+    case GDN_ERR_DTYPE: return "GDN_ERR_DTYPE: a tensor has the wrong dtype";
+    case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE: a tensor has the wrong rank, shape or strides";
+    case GDN_ERR_ALIGN: return "GDN_ERR_ALIGN: a pointer or stride breaks an alignment rule";
+    case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: a written tensor overlaps another tensor";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: head size, tile or schedule not built for this call";
+    case GDN_ERR_ARG: return "GDN_ERR_ARG: bad scalar argument or flag";
+    case GDN_ERR_INDICES: return "GDN_ERR_INDICES: bad or repeated state index, or bad cu_seqlens";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: the CUDA runtime refused the launch or copy";
+    default: return "unknown gdn status";
     }
+}
+
+GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                              const gdn_tensor *a, const gdn_tensor *b, const gdn_tensor *A_log,
+                              const gdn_tensor *dt_bias, const gdn_tensor *state_pool,
+                              const gdn_tensor *state_indices, const gdn_tensor *cu_seqlens,
+                              const gdn_tensor *out, float scale, uint32_t flags, const gdn_extra *extra)
+{
+    UpdateArgs c{q, k, v, out, false, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, scale, flags, extra};
+    return run_update(c);
+}
+
+GDN_API int gdn_recurrent_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                                 const gdn_tensor *g, const gdn_tensor *beta, const gdn_tensor *state_pool,
+                                 const gdn_tensor *state_indices, const gdn_tensor *cu_seqlens,
+                                 const gdn_tensor *out, float scale, uint32_t flags, const gdn_extra *extra)
+{
+    UpdateArgs c{q, k, v, out, true, g, beta, nullptr, nullptr, state_pool, state_indices, cu_seqlens, scale, flags,
+                 extra};
+    return run_update(c);
+}
+
+GDN_API int gdn_gating(const gdn_tensor *A_log, const gdn_tensor *a, const gdn_tensor *dt_bias,
+                       const gdn_tensor *b, const gdn_tensor *g, const gdn_tensor *beta, const gdn_extra *extra)
+{
+    GDN_TRY(check_desc(A_log, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(dt_bias, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(a, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(b, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(g, GDN_DTYPE_F32));
+    GDN_TRY(check_desc(beta, GDN_DTYPE_BF16, GDN_DTYPE_F32));
+    if (extra && (extra->schedule != 0 || extra->reserved != 0))
+        return GDN_ERR_ARG;
+    // a, b, g, beta: the same shape [T_tot, HV] (any leading dims that
+    // flatten to tokens are passed as rank 2 here)
+    const gdn_tensor *pt[] = {a, b, g, beta};
+    for (const gdn_tensor *t : pt)
+        if (t->ndim != 2 || t->shape[0] != a->shape[0] || t->shape[1] != a->shape[1])
+            return GDN_ERR_SHAPE;
+    const int64_t T_tot = a->shape[0], HV = a->shape[1];
+    if (HV <= 0 || HV > INT32_MAX || A_log->ndim != 1 || A_log->shape[0] != HV || dt_bias->ndim != 1 ||
+        dt_bias->shape[0] != HV)
+        return GDN_ERR_SHAPE;
+    for (const gdn_tensor *t : {A_log, dt_bias, a, b, g, beta})
+        if (!aligned(t->data, elem_size(t->dtype)))
+            return GDN_ERR_ALIGN;
+    const Span sg = span_of(g), sb = span_of(beta);
+    if (overlap(sg, sb))
+        return GDN_ERR_ALIAS;
+    for (const gdn_tensor *t : {A_log, dt_bias, a, b}) {
+        const Span s = span_of(t);
+        if (overlap(s, sg) || overlap(s, sb))
+            return GDN_ERR_ALIAS;
+    }
+    if (T_tot == 0)
+        return GDN_OK;
+
+    gdn::GatingParams p;
+    std::memset(&p, 0, sizeof p);
+    p.a = a->data;
+    p.b = b->data;
+    p.A_log = static_cast<const float *>(A_log->data);
+    p.dt_bias = static_cast<const float *>(dt_bias->data);
+    p.g = static_cast<float *>(g->data);
+    p.beta = beta->data;
+    p.a_tok = a->stride[0];
+    p.a_head = a->stride[1];
+    p.b_tok = b->stride[0];
+    p.b_head = b->stride[1];
+    p.g_tok = g->stride[0];
+    p.g_head = g->stride[1];
+    p.beta_tok = beta->stride[0];
+    p.beta_head = beta->stride[1];
+    p.A_stride = A_log->stride[0];
+    p.dt_stride = dt_bias->stride[0];
+    p.n = T_tot * HV;
+    p.HV = static_cast<int32_t>(HV);
+    p.a_f32 = a->dtype == GDN_DTYPE_F32;
+    p.b_f32 = b->dtype == GDN_DTYPE_F32;
+    p.beta_f32 = beta->dtype == GDN_DTYPE_F32;
+    cudaStream_t stream = extra ? static_cast<cudaStream_t>(extra->stream) : nullptr;
+    const int64_t blocks = (p.n + 255) / 256;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks < 4096 ? blocks : 4096));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, gdn::gdn_gating_kernel, p);
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -1,27 +1,33 @@
-// gdn_decode_kernel.cuh -- sm_100a kernel of the fused sigmoid-gating Gated
-// DeltaNet decode / speculative-decode state update (the operation is
-// stated in include/gdn_decode.h).
+// gdn_decode_kernel.cuh -- sm_100a kernels of the Gated DeltaNet decode /
+// speculative-decode state update (the operation is stated in
+// include/gdn_decode.h): the per-tile update kernel and the gating kernel.
 //
 // Work decomposition.  One CTA owns one (sequence i, value head hv, V-tile)
 // unit: a [K, BV] slab of the fp32 state S = pool[slot_i, hv].  The slab is
 // split over the CTA's threads as a (KG x VG) grid: thread (kg, vq) holds
 // rows kg*R .. kg*R+R-1 (R = K/KG) and the four columns vq*4 .. vq*4+3, i.e.
-// R float4 registers.  Each warp-wide load touches whole 128-byte rows, so
-// the state moves with 128-bit, fully coalesced loads and stores, once per
-// sequence; the slab stays in registers across all tokens of the sequence
-// (the speculative-decode path).
+// R float4 registers.  Each warp-wide load touches whole row segments of
+// 64-256 bytes, so the state moves with 128-bit, fully coalesced streaming
+// loads and stores, once per sequence; the slab stays in registers across
+// all tokens of the sequence (the speculative-decode path).
 //
 // Per token the two contractions over K that the update needs -- u = S^T k
 // and w = S^T q on the state before this token -- are done in ONE pass over
 // the registers, together with |k|^2, |q|^2 and k.q (for the rsqrt
 // normalisation, which is a per-token scalar and therefore commutes with the
-// sums).  Partial sums are reduced with xor-shuffles inside the warp and
-// one shared-memory exchange across warps (one __syncthreads per token,
-// double-buffered by token parity).  Then, with decay = exp(g):
+// sums).  Partial sums are reduced with xor-shuffles inside the warp and,
+// for multi-warp tiles, one shared-memory exchange across warps (one
+// __syncthreads per token, double-buffered by token parity).  Then, with
+// decay = exp(g):
 //     delta = beta * (v - decay * u * rk)                (S^T k^ on the decayed S)
 //     o     = decay * w * qs + (k^ . q^) * delta         (= S'^T q^ after the update)
 //     S'    = decay * S + k^ delta^T
 // which is the update of the header rearranged so that S is read once.
+//
+// Template parameters: the activation element type TAct (q, k, v, out:
+// bf16 or fp32) and GIVEN_GATES (false: decay and beta come from A_log, a,
+// b, dt_bias -- the fused sigmoid gating; true: from per-token g and beta
+// arrays -- the recurrence of the unfused pair).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,12 +38,13 @@
 namespace gdn {
 
 struct DecodeParams {
-    const __nv_bfloat16 *q, *k, *v, *a, *b;
+    const void *q, *k, *v;      // TAct
+    const void *a, *b;          // fused: a, b; given gates: g (fp32), beta
     const float *A_log, *dt_bias;
     float *state;
     const int32_t *indices;
     const int32_t *cu_seqlens;  // nullptr: fixed length T_fixed
-    __nv_bfloat16 *out;
+    void *out;                  // TAct
     float *inter;               // nullptr unless GDN_WRITE_INTERMEDIATE
     uint32_t *status;           // nullptr: device errors are not reported
     // strides in elements
@@ -46,6 +53,7 @@ struct DecodeParams {
     int64_t A_stride, dt_stride;
     int64_t s_slot, s_head, i_tok, i_head;
     int32_t N, T_fixed, T_tot, HV, G, num_slots;
+    int32_t a_f32, b_f32;       // element type of a / b (fused) or g / beta (given): 1 = fp32, 0 = bf16
     float scale;
     uint32_t flags;
 };
@@ -73,6 +81,54 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
     return l | (h << 16);
 }
+
+// A scalar gate input stored as fp32 or bf16: fetch its raw bits now, widen
+// them when the value is needed (so the load stays in flight meanwhile).
+__device__ __forceinline__ uint32_t gate_raw(const void *base, int64_t idx, int32_t is_f32)
+{
+    return is_f32 ? __ldg(static_cast<const unsigned int *>(base) + idx)
+                  : static_cast<uint32_t>(__ldg(static_cast<const unsigned short *>(base) + idx));
+}
+
+__device__ __forceinline__ float gate_value(uint32_t raw, int32_t is_f32)
+{
+    return __uint_as_float(is_f32 ? raw : raw << 16);
+}
+
+// Element-type traits of the activations.
+template <typename T>
+struct Act;
+
+template <>
+struct Act<__nv_bfloat16> {
+    static constexpr int PER16 = 8;   // elements per 16-byte load
+    using Raw4 = uint2;               // four elements
+    __device__ static void unpack16(const uint4 u, float *f) { unpack8(u, f); }
+    __device__ static float4 unpack4(const uint2 r)
+    {
+        return make_float4(bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y));
+    }
+    __device__ static void store4(__nv_bfloat16 *p, float a, float b, float c, float d)
+    {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+    }
+};
+
+template <>
+struct Act<float> {
+    static constexpr int PER16 = 4;
+    using Raw4 = float4;
+    __device__ static void unpack16(const uint4 u, float *f)
+    {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+    __device__ static float4 unpack4(const float4 r) { return r; }
+    __device__ static void store4(float *p, float a, float b, float c, float d)
+    {
+        *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+    }
+};
 
 // Programmatic dependent launch: let the next kernel on the stream be
 // scheduled as soon as every CTA of this grid has started, then wait until the
@@ -102,19 +158,26 @@ struct TileShape {
     static_assert(BV % 4 == 0 && V % BV == 0, "V must split into BV-wide tiles");
     static_assert(VG <= 32 && 32 % VG == 0, "a warp must hold whole k-groups");
     static_assert(THREADS % 32 == 0 && THREADS <= 1024, "whole warps");
-    static_assert(K % KG == 0 && R % 8 == 0, "q/k rows are loaded 8 bf16 (16 bytes) at a time");
+    static_assert(K % KG == 0 && R % 8 == 0, "q/k rows are loaded 16 bytes at a time");
 };
 
-template <int K, int V, int BV, int KG>
+template <int K, int V, int BV, int KG, typename TAct, bool GIVEN_GATES>
 __global__ void __launch_bounds__(TileShape<K, V, BV, KG>::THREADS)
 gdn_decode_kernel(const __grid_constant__ DecodeParams p)
 {
     using TS = TileShape<K, V, BV, KG>;
+    using A = Act<TAct>;
     constexpr int VG = TS::VG, WARPS = TS::WARPS, R = TS::R, NV = TS::NV, XW = TS::XW;
+    constexpr int QK_LOADS = R / A::PER16;
 
     __shared__ __align__(16) float xch[2][WARPS > 1 ? WARPS : 1][WARPS > 1 ? XW : 4];
 
     pdl_prologue();
+
+    const TAct *q = static_cast<const TAct *>(p.q);
+    const TAct *k = static_cast<const TAct *>(p.k);
+    const TAct *v = static_cast<const TAct *>(p.v);
+    TAct *out = static_cast<TAct *>(p.out);
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -157,8 +220,7 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
         // Padded sequence: zero output rows of this tile, no state access.
         if (kg == 0)
             for (int t = 0; t < len; ++t)
-                *reinterpret_cast<uint2 *>(p.out + (bos + t) * p.o_tok + hv * p.o_head + col0) =
-                    make_uint2(0u, 0u);
+                A::store4(out + (bos + t) * p.o_tok + hv * p.o_head + col0, 0.f, 0.f, 0.f, 0.f);
         return;
     }
     if (len == 0)
@@ -173,27 +235,30 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
         s[j] = __ldcs(reinterpret_cast<const float4 *>(s_ptr + j * V));
 
     const int h = hv / p.G;
-    const float neg_A = -expf(__ldg(p.A_log + hv * p.A_stride));
-    const float dt_b = __ldg(p.dt_bias + hv * p.dt_stride);
+    float neg_A = 0.f, dt_b = 0.f;
+    if constexpr (!GIVEN_GATES) {
+        neg_A = -expf(__ldg(p.A_log + hv * p.A_stride));
+        dt_b = __ldg(p.dt_bias + hv * p.dt_stride);
+    }
     const bool l2norm = (p.flags & GDN_L2NORM_QK) != 0;
     const bool write_inter = (p.flags & GDN_WRITE_INTERMEDIATE) != 0;
 
-    // Token inputs are software-pipelined: the raw bf16 words of token t+1
-    // are in flight while token t is computed.
-    uint4 k_nx[R / 8], q_nx[R / 8];
-    uint2 v_nx;
-    unsigned short a_nx, b_nx;
+    // Token inputs are software-pipelined: the raw words of token t+1 are
+    // in flight while token t is computed.
+    uint4 k_nx[QK_LOADS], q_nx[QK_LOADS];
+    typename A::Raw4 v_nx;
+    uint32_t a_nx, b_nx;
     auto fetch = [&](int64_t tok) {
-        const uint4 *kp = reinterpret_cast<const uint4 *>(p.k + tok * p.k_tok + h * p.k_head + row0);
-        const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + tok * p.q_tok + h * p.q_head + row0);
+        const uint4 *kp = reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + row0);
+        const uint4 *qp = reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + row0);
 #pragma unroll
-        for (int c = 0; c < R / 8; ++c) {
+        for (int c = 0; c < QK_LOADS; ++c) {
             k_nx[c] = __ldg(kp + c);
             q_nx[c] = __ldg(qp + c);
         }
-        v_nx = __ldg(reinterpret_cast<const uint2 *>(p.v + tok * p.v_tok + hv * p.v_head + col0));
-        a_nx = __ldg(reinterpret_cast<const unsigned short *>(p.a + tok * p.a_tok + hv * p.a_head));
-        b_nx = __ldg(reinterpret_cast<const unsigned short *>(p.b + tok * p.b_tok + hv * p.b_head));
+        v_nx = __ldg(reinterpret_cast<const typename A::Raw4 *>(v + tok * p.v_tok + hv * p.v_head + col0));
+        a_nx = gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32);
+        b_nx = gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32);
     };
     fetch(bos);
 
@@ -203,13 +268,13 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
         // ---- inputs: this thread's R rows of q and k, 4 columns of v
         float kr[R], qr[R];
 #pragma unroll
-        for (int c = 0; c < R / 8; ++c) {
-            unpack8(k_nx[c], kr + 8 * c);
-            unpack8(q_nx[c], qr + 8 * c);
+        for (int c = 0; c < QK_LOADS; ++c) {
+            A::unpack16(k_nx[c], kr + A::PER16 * c);
+            A::unpack16(q_nx[c], qr + A::PER16 * c);
         }
-        const uint2 v_raw = v_nx;
-        const float a_t = __uint_as_float(static_cast<uint32_t>(a_nx) << 16);
-        const float b_t = __uint_as_float(static_cast<uint32_t>(b_nx) << 16);
+        const float4 v_t = A::unpack4(v_nx);
+        const float a_t = gate_value(a_nx, p.a_f32);   // a, or g with given gates
+        const float b_t = gate_value(b_nx, p.b_f32);   // b, or beta with given gates
         if (t + 1 < len)
             fetch(tok + 1);
 
@@ -246,48 +311,54 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             W = make_float4(w0, w1, w2, w3);
             SKK = skk; SQQ = sqq; SKQ = skq;
         } else {
-        const int buf = t & 1;
-        if (lane < VG) {
-            *reinterpret_cast<float4 *>(&xch[buf][warp][vq * 4]) = make_float4(u0, u1, u2, u3);
-            *reinterpret_cast<float4 *>(&xch[buf][warp][BV + vq * 4]) = make_float4(w0, w1, w2, w3);
-            if (lane == 0) {
-                xch[buf][warp][2 * BV + 0] = skk;
-                xch[buf][warp][2 * BV + 1] = sqq;
-                xch[buf][warp][2 * BV + 2] = skq;
+            const int buf = t & 1;
+            if (lane < VG) {
+                *reinterpret_cast<float4 *>(&xch[buf][warp][vq * 4]) = make_float4(u0, u1, u2, u3);
+                *reinterpret_cast<float4 *>(&xch[buf][warp][BV + vq * 4]) = make_float4(w0, w1, w2, w3);
+                if (lane == 0) {
+                    xch[buf][warp][2 * BV + 0] = skk;
+                    xch[buf][warp][2 * BV + 1] = sqq;
+                    xch[buf][warp][2 * BV + 2] = skq;
+                }
             }
-        }
-        __syncthreads();
-        U = make_float4(0.f, 0.f, 0.f, 0.f);
-        W = U;
-        SKK = 0.f; SQQ = 0.f; SKQ = 0.f;
+            __syncthreads();
+            U = make_float4(0.f, 0.f, 0.f, 0.f);
+            W = U;
+            SKK = 0.f; SQQ = 0.f; SKQ = 0.f;
 #pragma unroll
-        for (int wi = 0; wi < WARPS; ++wi) {
-            const float4 uu = *reinterpret_cast<const float4 *>(&xch[buf][wi][vq * 4]);
-            const float4 ww = *reinterpret_cast<const float4 *>(&xch[buf][wi][BV + vq * 4]);
-            U.x += uu.x; U.y += uu.y; U.z += uu.z; U.w += uu.w;
-            W.x += ww.x; W.y += ww.y; W.z += ww.z; W.w += ww.w;
-            SKK += xch[buf][wi][2 * BV + 0];
-            SQQ += xch[buf][wi][2 * BV + 1];
-            SKQ += xch[buf][wi][2 * BV + 2];
-        }
+            for (int wi = 0; wi < WARPS; ++wi) {
+                const float4 uu = *reinterpret_cast<const float4 *>(&xch[buf][wi][vq * 4]);
+                const float4 ww = *reinterpret_cast<const float4 *>(&xch[buf][wi][BV + vq * 4]);
+                U.x += uu.x; U.y += uu.y; U.z += uu.z; U.w += uu.w;
+                W.x += ww.x; W.y += ww.y; W.z += ww.z; W.w += ww.w;
+                SKK += xch[buf][wi][2 * BV + 0];
+                SQQ += xch[buf][wi][2 * BV + 1];
+                SKQ += xch[buf][wi][2 * BV + 2];
+            }
         }
 
         // ---- gates and norms (scalars, computed by every thread) ----
         const float rk = l2norm ? rsqrtf(SKK + 1e-6f) : 1.f;
         const float qs = (l2norm ? rsqrtf(SQQ + 1e-6f) : 1.f) * p.scale;
-        const float x = a_t + dt_b;
-        const float sp = x > 20.f ? x : log1pf(expf(x));
-        const float decay = expf(neg_A * sp);
-        const float beta = 1.f / (1.f + expf(-b_t));
+        float decay, beta;
+        if constexpr (GIVEN_GATES) {
+            decay = expf(a_t);
+            beta = b_t;
+        } else {
+            const float x = a_t + dt_b;
+            const float sp = x > 20.f ? x : log1pf(expf(x));
+            decay = expf(neg_A * sp);
+            beta = 1.f / (1.f + expf(-b_t));
+        }
         const float kq = SKQ * rk * qs;
 
         // ---- delta and output ----------------------------------
         const float dku = decay * rk;
         const float dwq = decay * qs;
-        const float d0 = beta * (bf16_lo(v_raw.x) - dku * U.x);
-        const float d1 = beta * (bf16_hi(v_raw.x) - dku * U.y);
-        const float d2 = beta * (bf16_lo(v_raw.y) - dku * U.z);
-        const float d3 = beta * (bf16_hi(v_raw.y) - dku * U.w);
+        const float d0 = beta * (v_t.x - dku * U.x);
+        const float d1 = beta * (v_t.y - dku * U.y);
+        const float d2 = beta * (v_t.z - dku * U.z);
+        const float d3 = beta * (v_t.w - dku * U.w);
 
         // ---- S <- decay S + k^ delta^T -----------------------------
 #pragma unroll
@@ -299,14 +370,9 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             s[j].w = fmaf(kh, d3, decay * s[j].w);
         }
 
-        if (kg == 0) {
-            const float o0 = fmaf(kq, d0, dwq * W.x);
-            const float o1 = fmaf(kq, d1, dwq * W.y);
-            const float o2 = fmaf(kq, d2, dwq * W.z);
-            const float o3 = fmaf(kq, d3, dwq * W.w);
-            *reinterpret_cast<uint2 *>(p.out + tok * p.o_tok + hv * p.o_head + col0) =
-                make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
-        }
+        if (kg == 0)
+            A::store4(out + tok * p.o_tok + hv * p.o_head + col0, fmaf(kq, d0, dwq * W.x),
+                      fmaf(kq, d1, dwq * W.y), fmaf(kq, d2, dwq * W.z), fmaf(kq, d3, dwq * W.w));
 
         // ---- optional per-token state ------------------------------
         if (write_inter) {
@@ -322,6 +388,42 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
 #pragma unroll
         for (int j = 0; j < R; ++j)
             __stcs(reinterpret_cast<float4 *>(s_ptr + j * V), s[j]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The gating step alone (the first kernel of the unfused pair):
+//     g[t,hv]    = -exp(A_log[hv]) * softplus(a[t,hv] + dt_bias[hv])   (fp32)
+//     beta[t,hv] = sigmoid(b[t,hv])                                    (fp32 or bf16)
+// One thread per (token, value head), grid-stride over T_tot * HV.
+// ---------------------------------------------------------------------------
+struct GatingParams {
+    const void *a, *b;
+    const float *A_log, *dt_bias;
+    float *g;
+    void *beta;
+    int64_t a_tok, a_head, b_tok, b_head, g_tok, g_head, beta_tok, beta_head, A_stride, dt_stride;
+    int64_t n;                  // T_tot * HV
+    int32_t HV, a_f32, b_f32, beta_f32;
+};
+
+__global__ void __launch_bounds__(256) gdn_gating_kernel(const __grid_constant__ GatingParams p)
+{
+    pdl_prologue();
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < p.n;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t tok = e / p.HV;
+        const int hv = static_cast<int>(e - tok * p.HV);
+        const float a_t = gate_value(gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32), p.a_f32);
+        const float b_t = gate_value(gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32), p.b_f32);
+        const float x = a_t + __ldg(p.dt_bias + hv * p.dt_stride);
+        const float sp = x > 20.f ? x : log1pf(expf(x));
+        p.g[tok * p.g_tok + hv * p.g_head] = -expf(__ldg(p.A_log + hv * p.A_stride)) * sp;
+        const float beta = 1.f / (1.f + expf(-b_t));
+        if (p.beta_f32)
+            static_cast<float *>(p.beta)[tok * p.beta_tok + hv * p.beta_head] = beta;
+        else
+            static_cast<__nv_bfloat16 *>(p.beta)[tok * p.beta_tok + hv * p.beta_head] = __float2bfloat16_rn(beta);
     }
 }
 

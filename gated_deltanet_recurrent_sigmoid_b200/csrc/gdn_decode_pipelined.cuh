@@ -1,6 +1,7 @@
 // gdn_decode_pipelined.cuh -- persistent, bulk-copy-pipelined sm_100a kernel
 // of the fused sigmoid-gating Gated DeltaNet decode update (operation in
-// include/gdn_decode.h; same arithmetic as gdn_decode_kernel.cuh).
+// include/gdn_decode.h; same arithmetic as gdn_decode_kernel.cuh), for bf16
+// activations and the fused sigmoid gating.
 //
 // One CTA per SM walks a static list of (sequence, value head) units: unit
 // u = blockIdx.x + n * gridDim.x.  A unit's whole fp32 state S (K x V =
@@ -304,6 +305,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
     const int col0 = g * GROUP_COLS + vq * 4;
     const bool l2norm = (p.flags & GDN_L2NORM_QK) != 0;
     const bool write_inter = (p.flags & GDN_WRITE_INTERMEDIATE) != 0;
+    // This schedule takes bf16 activations and bf16 a, b (the host checks).
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
+    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
+    const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(p.a);
+    const __nv_bfloat16 *b = static_cast<const __nv_bfloat16 *>(p.b);
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
 
     uint32_t tcount = 0;  // tokens this group has processed: picks the exchange buffer
     for (int j = 0; j < n_mine; ++j) {
@@ -321,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
         } else if (u.kind == 1) {
             if (kg == 0)
                 for (int t = 0; t < u.len; ++t)
-                    *reinterpret_cast<uint2 *>(p.out + (u.bos + t) * p.o_tok + u.hv * p.o_head + col0) =
+                    *reinterpret_cast<uint2 *>(out + (u.bos + t) * p.o_tok + u.hv * p.o_head + col0) =
                         make_uint2(0u, 0u);
         } else if (u.kind == 0 && ok) {
             float *tile = sm.tile[s];
@@ -336,12 +344,12 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
             for (int t = 0; t < u.len; ++t) {
                 const int64_t tok = u.bos + t;
                 float kr[R], qr[R];
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(p.k + tok * p.k_tok + h * p.k_head + row0)), kr);
-                unpack8(__ldg(reinterpret_cast<const uint4 *>(p.q + tok * p.q_tok + h * p.q_head + row0)), qr);
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + row0)), kr);
+                unpack8(__ldg(reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + row0)), qr);
                 const uint2 v_raw =
-                    __ldg(reinterpret_cast<const uint2 *>(p.v + tok * p.v_tok + u.hv * p.v_head + col0));
-                const float a_t = load_bf16(p.a + tok * p.a_tok + u.hv * p.a_head);
-                const float b_t = load_bf16(p.b + tok * p.b_tok + u.hv * p.b_head);
+                    __ldg(reinterpret_cast<const uint2 *>(v + tok * p.v_tok + u.hv * p.v_head + col0));
+                const float a_t = load_bf16(a + tok * p.a_tok + u.hv * p.a_head);
+                const float b_t = load_bf16(b + tok * p.b_tok + u.hv * p.b_head);
 
                 float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
                 float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f;
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
                     const float o1 = fmaf(kq, d1, dwq * W.y);
                     const float o2 = fmaf(kq, d2, dwq * W.z);
                     const float o3 = fmaf(kq, d3, dwq * W.w);
-                    *reinterpret_cast<uint2 *>(p.out + tok * p.o_tok + u.hv * p.o_head + col0) =
+                    *reinterpret_cast<uint2 *>(out + tok * p.o_tok + u.hv * p.o_head + col0) =
                         make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
                 }
                 if (write_inter) {

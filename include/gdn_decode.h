@@ -32,14 +32,16 @@
  * The caller owns all memory; the library allocates no device memory and
  * keeps no pointer after the call returns.  Strides must be >= 0.
  *
- *   argument        dtype  shape                                  layout rules
- *   q, k            bf16   [T_tot, H, K] | [1, T_tot, H, K]       K contiguous; token and
- *                          (varlen) or [N, T, H, K] (fixed T)     head strides % 8 == 0;
- *                                                                 data 16-byte aligned
- *   v, out          bf16   same leading dims, [.., HV, V]         V contiguous; strides % 4
- *                                                                 == 0; data 8-byte aligned
- *   a, b            bf16   [T_tot, HV] | [1, T_tot, HV] | [N,T,HV] any strides (packed `ba`
- *                                                                 projections are fine)
+ *   argument        dtype      shape                              layout rules
+ *   q, k            bf16|fp32  [T_tot, H, K] | [1, T_tot, H, K]   K contiguous; token and
+ *                              (varlen) or [N, T, H, K] (fixed T) head strides x element
+ *                                                                 size % 16 == 0; data
+ *                                                                 16-byte aligned
+ *   v, out          as q       same leading dims, [.., HV, V]     V contiguous; strides % 4
+ *                                                                 == 0; data aligned to 4
+ *                                                                 elements
+ *   a, b            bf16|fp32  [T_tot, HV] | [1, T_tot, HV] |     any strides (packed `ba`
+ *                              [N, T, HV]                         projections are fine)
  *   A_log, dt_bias  fp32   [HV]                                   any stride
  *   state_pool      fp32   [num_slots, HV, K, V]                  K, V contiguous (strides
  *                                                                 V, 1); slot/head strides
@@ -113,7 +115,7 @@ extern "C" {
 #define GDN_ERR_SHAPE       (-3) /* wrong rank, shape or inconsistent sizes */
 #define GDN_ERR_ALIGN       (-4) /* pointer or stride breaks an alignment rule */
 #define GDN_ERR_ALIAS       (-5) /* a written tensor overlaps another tensor */
-#define GDN_ERR_UNSUPPORTED (-6) /* head size or tile not built */
+#define GDN_ERR_UNSUPPORTED (-6) /* head size, tile or schedule not built */
 #define GDN_ERR_ARG         (-7) /* bad scalar: scale <= 0 or not finite, unknown flag */
 #define GDN_ERR_INDICES     (-8) /* GDN_CHECK_INDICES found a bad or repeated slot,
                                     or bad cu_seqlens */
@@ -127,7 +129,8 @@ extern "C" {
                                     64x16, 64x32.  Library choice: 64x32 when
                                     every sequence has one token, else 32x32
                                     with >= 4096 (sequence, value head) pairs,
-                                    else 16x16 */
+                                    else 16x16; with fp32 activations 32x16
+                                    for one token, else 16x16 */
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
                                     tiles stream through a shared-memory ring of
                                     bulk async copies (cp.async.bulk) */
@@ -172,6 +175,43 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
                       float scale, uint32_t flags, const gdn_extra *extra);
 
 /* Static text for a gdn_status value (never NULL). */
+/*
+ * The recurrence of the unfused pair: the pages name the two kernels the
+ * fused op replaces, fused_gdn_gating then fused_recurrent_gated_delta_rule
+ * (vLLM PR 35777 summary, 执行摘要 / 实现拆解), and the sglang variant
+ * with precomputed gates, fused_recurrent_gated_delta_rule_update_fwd
+ * ("[Qwen3Next] Optimize ...", Code Review).  Same as gdn_decode_update,
+ * except that each token's decay and beta come from arrays:
+ *     S <- exp(g[t,hv]) * S;   S <- S + k^ (beta[t,hv] * (v - S^T k^))^T
+ *   g     fp32       [tokens..., HV] (same leading dims as a would have)
+ *   beta  bf16|fp32  [tokens..., HV]
+ * Every other argument, flag, error and the extra struct are as for
+ * gdn_decode_update.  GDN_SCHEDULE_PIPELINED is not built for this entry
+ * point (GDN_ERR_UNSUPPORTED).
+ */
+GDN_API int gdn_recurrent_update(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                                 const gdn_tensor *g, const gdn_tensor *beta,
+                                 const gdn_tensor *state_pool, const gdn_tensor *state_indices,
+                                 const gdn_tensor *cu_seqlens, const gdn_tensor *out,
+                                 float scale, uint32_t flags, const gdn_extra *extra);
+
+/*
+ * The gating step alone (the pages' fused_gdn_gating, the first kernel of
+ * the unfused pair): for every (token, value head)
+ *     g[t,hv]    = -exp(A_log[hv]) * softplus(a[t,hv] + dt_bias[hv])
+ *     beta[t,hv] = sigmoid(b[t,hv])
+ *   A_log, dt_bias  fp32       [HV]
+ *   a, b            bf16|fp32  [T_tot, HV]   (rank 2, any strides)
+ *   g               fp32       [T_tot, HV]
+ *   beta            bf16|fp32  [T_tot, HV]
+ * g and beta must not overlap each other or any input.  extra: only the
+ * stream is used (NULL: default stream; schedule and reserved must be 0).
+ * Asynchronous; T_tot = 0 is GDN_OK with no launch.
+ */
+GDN_API int gdn_gating(const gdn_tensor *A_log, const gdn_tensor *a, const gdn_tensor *dt_bias,
+                       const gdn_tensor *b, const gdn_tensor *g, const gdn_tensor *beta,
+                       const gdn_extra *extra);
+
 GDN_API const char *gdn_status_string(int status);
 
 /* GDN_DECODE_ABI_VERSION of the loaded library. */

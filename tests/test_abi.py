@@ -23,7 +23,8 @@ def declared_functions():
 
 
 def test_header_declares_the_abi():
-    assert set(declared_functions()) == {"gdn_decode_update", "gdn_status_string", "gdn_version"}
+    assert set(declared_functions()) == {"gdn_decode_update", "gdn_recurrent_update", "gdn_gating",
+                                         "gdn_status_string", "gdn_version"}
 
 
 def test_library_exports_every_declared_symbol(gdn_lib):
