@@ -210,6 +210,8 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs):
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
+    if schedule == binding.SCHEDULE_CHUNKED:
+        return "gdn::chunk::gdn_chunk_kernel<true>"
     if tile_v:
         bv, rows = tile_v, tile_rows or 16
     else:
@@ -251,7 +253,7 @@ def main():
     ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
     ap.add_argument("--tile-v", type=int, default=0)
     ap.add_argument("--tile-rows", type=int, default=0)
-    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -288,7 +290,7 @@ def main():
     binding.load()
 
     schedule = {"auto": binding.SCHEDULE_AUTO, "per_tile": binding.SCHEDULE_PER_TILE,
-                "pipelined": binding.SCHEDULE_PIPELINED}[args.schedule]
+                "pipelined": binding.SCHEDULE_PIPELINED, "chunked": binding.SCHEDULE_CHUNKED}[args.schedule]
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)

@@ -30,6 +30,7 @@ DEV_TIMEOUT = 4
 SCHEDULE_AUTO = 0
 SCHEDULE_PER_TILE = 1
 SCHEDULE_PIPELINED = 2
+SCHEDULE_CHUNKED = 3
 
 OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5

@@ -14,6 +14,7 @@
 
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
+#include "gdn_chunk_kernel.cuh"
 #include "gdn_decode_pipelined.cuh"
 
 namespace {
@@ -203,6 +204,29 @@ cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t strea
                      stream, pdl, p);
 }
 
+// Chunked schedule: one CTA per (sequence, value head), dynamic shared
+// memory opted in once per device.
+cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
+{
+    static bool ready[64][2];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    const size_t smem = sizeof(gdn::chunk::Smem);
+    if (!ready[dev][l2norm]) {
+        err = cudaFuncSetAttribute(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (err != cudaSuccess)
+            return err;
+        ready[dev][l2norm] = true;
+    }
+    return launch_ex(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
+                     dim3(static_cast<unsigned>(units)), dim3(gdn::chunk::THREADS), smem, stream, pdl, p);
+}
+
 // The tile table: (V-tile width, rows per thread) -> (BV, KG = K / rows).
 template <typename TAct, bool GIVEN>
 cudaError_t launch_tile(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, int tile_v,
@@ -279,7 +303,8 @@ int run_update(const UpdateArgs &c)
     if ((flags & ~known) != 0 || !std::isfinite(c.scale) || !(c.scale > 0.f))
         return GDN_ERR_ARG;
     const int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
-    if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED)
+    if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED &&
+        schedule != GDN_SCHEDULE_CHUNKED)
         return GDN_ERR_ARG;
     if (extra && extra->reserved != 0)
         return GDN_ERR_ARG;
@@ -457,10 +482,18 @@ int run_update(const UpdateArgs &c)
                          (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
     if (!tile_ok)
         return GDN_ERR_UNSUPPORTED;
-    // The pipelined schedule is built for bf16 activations and fused bf16 gates.
+    // The pipelined schedule is built for bf16 activations and fused bf16
+    // gates; the chunked one for bf16 activations, fused gates and no
+    // per-token states.
     if (schedule == GDN_SCHEDULE_PIPELINED &&
         (act != GDN_DTYPE_BF16 || c.given_gates || ga->dtype != GDN_DTYPE_BF16 || gb->dtype != GDN_DTYPE_BF16))
         return GDN_ERR_UNSUPPORTED;
+    if (schedule == GDN_SCHEDULE_CHUNKED && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
+        return GDN_ERR_UNSUPPORTED;
+    // the chunked kernel reads v rows 16 bytes at a time, like q and k
+    if (schedule == GDN_SCHEDULE_CHUNKED &&
+        (!aligned(v->data, 16) || !stride_ok(T_tot, Lv.tok, 8) || !stride_ok(HV, v->stride[v->ndim - 2], 8)))
+        return GDN_ERR_ALIGN;
     const int64_t units = N * HV;
     if (units * (kHeadV / tile_v) > INT32_MAX)
         return GDN_ERR_SHAPE;
@@ -523,6 +556,8 @@ int run_update(const UpdateArgs &c)
     cudaError_t err;
     if (schedule == GDN_SCHEDULE_PIPELINED)
         err = launch_pipelined(p, units, stream, pdl);
+    else if (schedule == GDN_SCHEDULE_CHUNKED)
+        err = launch_chunked(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (act == GDN_DTYPE_BF16)
         err = c.given_gates ? launch_tile<__nv_bfloat16, true>(p, units, stream, pdl, tile_v, tile_rows)
                             : launch_tile<__nv_bfloat16, false>(p, units, stream, pdl, tile_v, tile_rows);

@@ -37,9 +37,12 @@
 
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
+#include "mbarrier_sm100.cuh"
 
 namespace gdn {
 namespace pipe {
+
+using namespace gdn::sync;
 
 constexpr int K = 128;
 constexpr int V = 128;
@@ -53,7 +56,6 @@ constexpr int XW = 2 * GROUP_COLS + 4;               // exchange floats per warp
 constexpr uint32_t TILE_BYTES = K * V * 4;           // 65536
 constexpr int CHUNKS = 4;                            // bulk copies per tile
 constexpr uint32_t CHUNK_BYTES = TILE_BYTES / CHUNKS;
-constexpr uint64_t WAIT_LIMIT_NS = 500ull * 1000ull * 1000ull;   // 0.5 s
 
 template <int STAGES>
 struct Smem {
@@ -63,62 +65,6 @@ struct Smem {
     unsigned long long done[STAGES];
     int failed;
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(unsigned long long *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(unsigned long long *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait on an mbarrier phase.  Gives up (returns false) after
-// WAIT_LIMIT_NS, or at once when another thread of the CTA has given up.
-__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *failed)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity))
-            return true;
-        if ((n & 63u) == 0u && (*failed || global_ns() - t0 > WAIT_LIMIT_NS))
-            return false;
-    }
-}
 
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, uint32_t bytes,
                                           unsigned long long *bar)
@@ -140,10 +86,6 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void fence_barrier_init()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
 
 __device__ __forceinline__ void group_sync(int group)
 {

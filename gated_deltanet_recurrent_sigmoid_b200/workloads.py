@@ -49,7 +49,8 @@ class WorkloadSpec:
     num_slots: int              # state-pool slots
     seed: int
     T: Optional[int] = 1        # fixed tokens per sequence, or None for varlen
-    max_len: int = 64           # varlen: lengths drawn U{1..max_len}
+    max_len: int = 64           # varlen: lengths drawn U{min_len..max_len}
+    min_len: int = 1
     pad_frac: float = 0.0       # fraction of state_indices set to -1
     varlen: bool = False        # pass cu_seqlens (also used for uniform T)
     intermediate: bool = False  # write per-token states
@@ -92,7 +93,7 @@ def generate(spec: WorkloadSpec) -> Workload:
     rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([spec.seed, spec.N])))
     N, H, HV, K, V = spec.N, spec.H, spec.HV, spec.K, spec.V
     if spec.T is None:
-        lens = rng.integers(1, spec.max_len + 1, size=N).astype(np.int32)
+        lens = rng.integers(spec.min_len, spec.max_len + 1, size=N).astype(np.int32)
     else:
         lens = np.full(N, spec.T, dtype=np.int32)
     T_tot = int(lens.sum())
@@ -136,7 +137,14 @@ def sweep_spec(N: int) -> WorkloadSpec:
                         T=None, max_len=64, pad_frac=0.10)
 
 
-ALL_SPECS = [TINY, DECODE_B512, FULLHEAD_B256, SPEC_B128_T4] + [sweep_spec(n) for n in SWEEP_NS]
+# Prefill-style: few sequences, long and ragged (the chunked schedule's workload).
+PREFILL_B8 = WorkloadSpec("prefill_b8_t2k", N=8, H=4, HV=8, num_slots=16, seed=5, T=None, min_len=1024,
+                          max_len=2048)
+PREFILL_B64 = WorkloadSpec("prefill_b64_t512", N=64, H=4, HV=8, num_slots=128, seed=6, T=None, min_len=256,
+                           max_len=768)
+
+ALL_SPECS = [TINY, DECODE_B512, FULLHEAD_B256, SPEC_B128_T4] + [sweep_spec(n) for n in SWEEP_NS] + [PREFILL_B8,
+                                                                                                   PREFILL_B64]
 BY_NAME = {s.name: s for s in ALL_SPECS}
 
 

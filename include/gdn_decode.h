@@ -134,6 +134,12 @@ extern "C" {
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
                                     tiles stream through a shared-memory ring of
                                     bulk async copies (cp.async.bulk) */
+#define GDN_SCHEDULE_CHUNKED   3 /* one CTA per (sequence, value head); tokens in
+                                    chunks of 64 through the closed form of the
+                                    delta rule over a chunk, every matrix product
+                                    on the tcgen05 tensor cores (prefill-style);
+                                    bf16 activations, gates from A_log/a/b/dt_bias,
+                                    no GDN_WRITE_INTERMEDIATE; v aligned like q */
 
 /* bits OR-ed into *device_status by the kernel */
 #define GDN_DEV_BAD_SLOT    1u

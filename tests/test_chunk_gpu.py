@@ -1,0 +1,128 @@
+"""The chunked (tensor-core) schedule against the oracle.
+
+Same update, same tolerances as the per-token kernels: state max abs 1e-4,
+output 1e-2 + 1e-2 |o_ref|, slots and status exact.  Sequences span several
+64-token chunks with ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_recurrent_sigmoid_b200 import binding
+from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl
+from gpu_helpers import (assert_out_close, assert_state_close, oracle_on, out_as_f32, run_gpu, run_oracle,
+                         sample_subproblem, to_device)
+from helpers import random_problem
+
+pytestmark = pytest.mark.gpu
+
+CHUNKED = binding.SCHEDULE_CHUNKED
+L2 = binding.L2NORM_QK
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(gdn_lib):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return gdn_lib
+
+
+def check(w, flags=L2, scale=None):
+    d, status, _ = run_gpu(w, flags=flags, schedule=CHUNKED, scale=scale)
+    ost, o_ref, s_ref, _ = run_oracle(w, flags=flags, scale=scale)
+    assert status == ost
+    assert_out_close(out_as_f32(d["out"]), o_ref)
+    pool = d["state_pool"].cpu().numpy()
+    live = w.state_indices[(w.state_indices >= 0) & (w.seq_lens > 0)] if not flags & binding.NO_FINAL_WRITEBACK \
+        else np.zeros(0, np.int64)
+    touched = np.zeros(w.spec.num_slots, bool)
+    touched[live] = True
+    assert np.array_equal(pool[~touched], w.state_pool[~touched])
+    if touched.any():
+        assert_state_close(pool[touched], s_ref[touched])
+    return d
+
+
+def problem(lens, pad=(), H=4, HV=8, seed=0):
+    rng = np.random.default_rng(seed)
+    p = random_problem(rng, lens=lens, H=H, HV=HV, K=128, V=128, pad=pad)
+    spec = wl.WorkloadSpec("chunk_case", N=len(lens), H=H, HV=HV, num_slots=p["state_pool"].shape[0], seed=seed,
+                           T=None)
+    return wl.Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
+                       p["state_indices"], p["cu_seqlens"])
+
+
+@pytest.mark.parametrize("lens", [[1], [64], [65], [200, 7, 130], [3, 64, 128, 1, 300]],
+                         ids=["1", "64", "65", "ragged3", "ragged5"])
+def test_chunked_matches_oracle(lens):
+    check(problem(lens, seed=len(lens)))
+
+
+def test_chunked_padding_empty_and_gqa():
+    check(problem([70, 0, 33, 129], pad=(2,), H=2, HV=6, seed=9))
+
+
+def test_chunked_l2norm_off_and_scale():
+    w = problem([90, 40], seed=3)
+    # L2 off: unit-length k keeps the state O(1)
+    k = wl.bf16_bits_to_f32(w.k)
+    w.k = wl.f32_to_bf16_bits(k / np.linalg.norm(k, axis=-1, keepdims=True))
+    check(w, flags=0)
+    check(problem([90, 40], seed=4), scale=0.2)
+
+
+def test_chunked_no_final_writeback_and_fixed_layout():
+    check(problem([77, 12], seed=5), flags=L2 | binding.NO_FINAL_WRITEBACK)
+    check(wl.generate(wl.shrink(wl.SPEC_B128_T4, 16)))         # T = 4, one partial chunk each
+    check(wl.generate(wl.TINY))                                 # fixed [N, 1] layout
+
+
+@pytest.mark.parametrize("spec", [wl.sweep_spec(8), wl.sweep_spec(64)], ids=lambda s: s.name)
+def test_chunked_full_size_sweeps(spec):
+    check(wl.generate(spec))
+
+
+def test_chunked_prefill_b64_sampled():
+    """Full-size prefill-style batch in the benchmark's launch configuration;
+    the oracle recomputes a sample of sequences."""
+    w = wl.generate(wl.PREFILL_B64)
+    d, status, _ = run_gpu(w, schedule=CHUNKED)
+    assert status == 0
+    rng = np.random.default_rng(0)
+    seqs = np.sort(rng.choice(w.spec.N, size=6, replace=False))
+    arrays, rows, slots = sample_subproblem(w, seqs)
+    _, o_ref, s_ref, _ = oracle_on(arrays)
+    out = d["out"].view(w.T_tot, w.spec.HV, w.spec.V)
+    assert_out_close(out[torch.from_numpy(rows).cuda()].float().cpu().numpy(), o_ref, "sampled out")
+    live = slots >= 0
+    got = d["state_pool"][torch.from_numpy(slots[live].astype(np.int64)).cuda()].cpu().numpy()
+    assert_state_close(got, s_ref, "sampled state")
+
+
+def test_chunked_agrees_with_per_token_kernel():
+    w = wl.generate(wl.shrink(wl.sweep_spec(64), 24))
+    a, _, _ = run_gpu(w, schedule=CHUNKED)
+    b, _, _ = run_gpu(w, schedule=binding.SCHEDULE_PER_TILE, tile_v=16, tile_rows=16)
+    assert (a["state_pool"] - b["state_pool"]).abs().max().item() <= 1e-4
+    assert (a["out"].float() - b["out"].float()).abs().max().item() <= 3e-2
+
+
+def test_chunked_rejects_unbuilt_modes():
+    w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 4))
+    d = to_device(w)
+    inter = torch.empty((w.T_tot, w.spec.HV, 128, 128), device="cuda")
+    with pytest.raises(binding.GdnError) as e:
+        binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"],
+                              d["state_indices"], d["cu_seqlens"], d["out"], intermediate_states=inter,
+                              schedule=CHUNKED)
+    assert e.value.status == binding.ERR_UNSUPPORTED
+
+
+def test_chunked_device_status():
+    w = problem([70, 20, 5], seed=11)
+    w.state_indices = w.state_indices.copy()
+    w.state_indices[1] = w.spec.num_slots           # out of range
+    d, status, _ = run_gpu(w, schedule=CHUNKED)
+    ost, o_ref, s_ref, _ = run_oracle(w)
+    assert status == ost == oracle.BAD_SLOT
+    assert_out_close(out_as_f32(d["out"]), o_ref)

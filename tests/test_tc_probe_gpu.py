@@ -1,0 +1,39 @@
+"""The tcgen05 wrappers (descriptors, TMEM layout, MMA, commit, TMEM loads)
+checked through a test-only one-tile probe against a plain matrix product."""
+import ctypes
+import os
+import sys
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+sys.path.insert(0, os.path.join(os.path.dirname(os.path.abspath(__file__)), "tc_probe"))
+
+
+@pytest.fixture(scope="module")
+def probe():
+    import build as probe_build
+    lib = ctypes.CDLL(probe_build.build())
+    lib.tc_gemm_probe.restype = ctypes.c_int
+    lib.tc_gemm_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
+    return lib
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 64, 128), (128, 128, 64), (128, 256, 128), (128, 16, 16),
+                                   (64, 64, 128), (64, 128, 64)])
+@pytest.mark.parametrize("negate,twice", [(0, 0), (1, 1)], ids=["plain", "neg_acc"])
+def test_tile_product_matches_matmul(probe, M, N, K, negate, twice):
+    g = torch.Generator().manual_seed(M * 1000 + N * 10 + K)
+    A = torch.randn(M, K, generator=g).bfloat16().cuda()
+    B = torch.randn(N, K, generator=g).bfloat16().cuda()
+    D = torch.full((M, N), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = probe.tc_gemm_probe(A.data_ptr(), B.data_ptr(), D.data_ptr(), M, N, K, negate, twice, status.data_ptr(),
+                             torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == 0 and int(status.item()) == 0
+    ref = (A.double() @ B.double().T) * (-1.0 if negate else 1.0) * (2.0 if twice else 1.0)
+    err = (D.double() - ref).abs().max().item()
+    assert err <= 1e-4 * max(1.0, ref.abs().max().item()), err
