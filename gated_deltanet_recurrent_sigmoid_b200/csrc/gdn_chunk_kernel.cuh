@@ -65,6 +65,11 @@ struct Smem {
     // each); before both, the fp32 matrix A [64][64] for the solve.
     alignas(1024) unsigned char wd[2][128 * 64 * 2];
     float rk[C], rqs[C], gam[C], beta[C], g[C];
+    // per-token factors of the chunk (computed once after the scan)
+    float fa[C];   // beta_j rk_j          (row factor of A)
+    float fw[C];   // beta_i e^gamma_i rk_i (column factor of T for W)
+    float fo[C];   // e^gamma_j rqs_j      (factor of S0^T q_j in the output)
+    float fd[C];   // e^(gamma_last - gamma_i) rk_i (factor of Delta_i in the state update)
     unsigned long long mbar;
     uint32_t tmem_base;
     int failed;
@@ -95,6 +100,32 @@ __device__ __forceinline__ void st_row8(unsigned char *tile, uint32_t r, uint32_
         w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
     }
     *reinterpret_cast<uint4 *>(tile + tc::kmajor_offset(r, c0, cols)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// fp32 64 x 64 matrices in shared memory (A and T of the solve): row-major
+// with the column XOR-swizzled by the row, so that both a row and a column
+// are spread over all 32 banks.
+__device__ __forceinline__ int sw64(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+
+// Transpose an 8 x 8 block of bf16 held as 8 rows of 16 bytes: out[c] holds
+// column c of the input (8 rows, as bf16 pairs).
+__device__ __forceinline__ void transpose8x8(const uint4 (&in)[8], uint4 (&out)[8])
+{
+    uint32_t pw[8][4];
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) {
+        const uint32_t a[4] = {in[2 * s2].x, in[2 * s2].y, in[2 * s2].z, in[2 * s2].w};
+        const uint32_t b[4] = {in[2 * s2 + 1].x, in[2 * s2 + 1].y, in[2 * s2 + 1].z, in[2 * s2 + 1].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            pw[2 * s2][w] = __byte_perm(a[w], b[w], 0x5410);       // column 2w of rows 2s2, 2s2+1
+            pw[2 * s2 + 1][w] = __byte_perm(a[w], b[w], 0x7632);   // column 2w+1
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        out[c] = make_uint4(pw[c & 1][c >> 1], pw[2 + (c & 1)][c >> 1], pw[4 + (c & 1)][c >> 1],
+                            pw[6 + (c & 1)][c >> 1]);
 }
 
 // Issue a product over `slices` 16-column k-slices: D (+)= A * B^T.
@@ -218,42 +249,69 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
         const bool last = c0 + C >= len;
 
         // ---- step 1: raw q, k, v of the chunk into the operand tiles ----
+        // thread (tg, kg): tokens 8 tg .. 8 tg + 7, columns 8 kg .. 8 kg + 7
         {
-            const int j = tid >> 1;             // token of the chunk
-            const int half = tid & 1;           // columns [64 half, 64 half + 64)
-            const bool live = j < n;
-            const int64_t tok = bos + c0 + j;
-            float kk = 0.f, qq = 0.f;
+            const int tg = tid >> 4, kg = tid & 15, col = 8 * kg;
+            uint4 kr[8], qr[8], vr[8];
+            float kk[8], qq[8];
+            // all 24 loads in flight before any is used
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int col = 64 * half + 8 * m;
-                uint4 kr = make_uint4(0u, 0u, 0u, 0u), qr = kr, vr = kr;
-                if (live) {
-                    kr = __ldg(reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + col));
-                    qr = __ldg(reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + col));
-                    vr = __ldg(reinterpret_cast<const uint4 *>(v + tok * p.v_tok + hv * p.v_head + col));
-                }
-                *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(j, col, K)) = kr;
-                *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(64 + j, col, K)) = qr;
-                float kf[8], qf[8], vf[8];
-                unpack8(kr, kf);
-                unpack8(qr, qf);
-                unpack8(vr, vf);
+            for (int r = 0; r < 8; ++r) {
+                const int j = 8 * tg + r;
+                const int64_t tok = bos + c0 + (j < n ? j : 0);
+                kr[r] = __ldg(reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + col));
+                qr[r] = __ldg(reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + col));
+                vr[r] = __ldg(reinterpret_cast<const uint4 *>(v + tok * p.v_tok + hv * p.v_head + col));
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int j = 8 * tg + r;
+                if (j >= n)
+                    kr[r] = qr[r] = vr[r] = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(j, col, K)) = kr[r];
+                *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(64 + j, col, K)) = qr[r];
+                float kf[8], qf[8];
+                unpack8(kr[r], kf);
+                unpack8(qr[r], qf);
+                kk[r] = 0.f;
+                qq[r] = 0.f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    kk = fmaf(kf[e], kf[e], kk);
-                    qq = fmaf(qf[e], qf[e], qq);
-                    st_bf16(sm.kt, col + e, j, C, __float2bfloat16_rn(kf[e]));
-                    st_bf16(sm.vt, col + e, j, C, __float2bfloat16_rn(vf[e]));
+                    kk[r] = fmaf(kf[e], kf[e], kk[r]);
+                    qq[r] = fmaf(qf[e], qf[e], qq[r]);
                 }
             }
-            kk += __shfl_xor_sync(0xffffffffu, kk, 1);
-            qq += __shfl_xor_sync(0xffffffffu, qq, 1);
-            if (half == 0) {
+            uint4 tr[8];
+            transpose8x8(kr, tr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                *reinterpret_cast<uint4 *>(sm.kt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
+            transpose8x8(vr, tr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                *reinterpret_cast<uint4 *>(sm.vt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
+            // sum the 16 column groups of each token (lanes differing in bits 0..3)
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1)
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    kk[r] += __shfl_xor_sync(0xffffffffu, kk[r], off);
+                    qq[r] += __shfl_xor_sync(0xffffffffu, qq[r], off);
+                }
+            if (kg < 8) {
+                const int j = 8 * tg + kg;
+                const int64_t tok = bos + c0 + j;
                 float rk = 0.f, rq = 0.f, g = 0.f, be = 0.f;
-                if (live) {
-                    rk = L2NORM ? rsqrtf(kk + 1e-6f) : 1.f;
-                    rq = (L2NORM ? rsqrtf(qq + 1e-6f) : 1.f) * p.scale;
+                float kk_j = kk[0], qq_j = qq[0];
+#pragma unroll
+                for (int r = 1; r < 8; ++r)
+                    if (kg == r) {
+                        kk_j = kk[r];
+                        qq_j = qq[r];
+                    }
+                if (j < n) {
+                    rk = L2NORM ? rsqrtf(kk_j + 1e-6f) : 1.f;
+                    rq = (L2NORM ? rsqrtf(qq_j + 1e-6f) : 1.f) * p.scale;
                     const float a_t = gate_value(gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32), p.a_f32);
                     const float b_t = gate_value(gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32), p.b_f32);
                     const float x = a_t + dt_b;
@@ -282,6 +340,14 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
             sm.gam[tid] = a0;
             sm.gam[32 + tid] = a1 + total0;
         }
+        __syncthreads();
+        if (tid < C) {      // per-token factors, once
+            const float gl = sm.gam[n - 1], gj = sm.gam[tid];
+            sm.fa[tid] = sm.beta[tid] * sm.rk[tid];
+            sm.fw[tid] = sm.beta[tid] * expf(gj) * sm.rk[tid];
+            sm.fo[tid] = expf(gj) * sm.rqs[tid];
+            sm.fd[tid] = expf(gl - gj) * sm.rk[tid];
+        }
         publish_smem();
 
         // ---- step 2: [K;Q] K^T and S0^T Q^T --------------------------------
@@ -297,7 +363,8 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
             break;
 
         // ---- step 3: A (rows 0..63) and P (rows 64..127) --------------------
-        float *Amat = reinterpret_cast<float *>(sm.wd[0]);     // [64][64] fp32
+        float *Amat = reinterpret_cast<float *>(sm.wd[0]);     // [64][64] fp32, swizzled
+        float *Tmat = reinterpret_cast<float *>(sm.wd[1]);     // [64][64] fp32, swizzled
         {
             float row[64];
 #pragma unroll
@@ -306,11 +373,11 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
             tc::tmem_wait_ld();
             if (tid < 64) {
                 const int j = tid;
-                const float fj = sm.beta[j] * sm.rk[j];
+                const float fj = sm.fa[j];
                 const float gj = sm.gam[j];
 #pragma unroll
                 for (int c = 0; c < 64; ++c)
-                    Amat[j * 64 + c] = (c < j) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
+                    Amat[sw64(j, c)] = (c < j) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
             } else {
                 const int j = tid - 64;
                 const float fj = sm.rqs[j];
@@ -327,29 +394,75 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
         }
         __syncthreads();
 
-        // ---- step 4: T = (I + A)^-1 by forward substitution, column per thread
+        // ---- step 4: T = (I + A)^-1, blocked by 16 x 16 ---------------------
+        // T_II = (I + A_II)^-1 (forward substitution, one column per thread);
+        // then T_IJ = -T_II sum_{M=J}^{I-1} A_IM T_MJ, one block diagonal at a
+        // time (each level is two small products spread over all threads).
+        float *X = reinterpret_cast<float *>(sm.tw[0]);        // scratch [3][16][16]
         if (tid < 64) {
-            const int col = tid;
-            float tcol[64];
+            const int I = tid >> 4, cc = tid & 15, c = 16 * I + cc;
+            float x[16];
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                float acc = (r == col) ? 1.f : 0.f;
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
                 for (int m = 0; m < r; ++m)
-                    acc = fmaf(-Amat[r * 64 + m], tcol[m], acc);
-                tcol[r] = (r < col) ? 0.f : acc;
+                    acc = fmaf(-Amat[sw64(16 * I + r, 16 * I + m)], x[m], acc);
+                x[r] = (r < cc) ? 0.f : acc;
+                Tmat[sw64(16 * I + r, c)] = x[r];
             }
-            const float fw = sm.beta[col] * expf(sm.gam[col]) * sm.rk[col];
-            const float fu = sm.beta[col];
+        } else {
+            // the strictly upper blocks of T are zero
+            for (int e = tid - 64; e < 6 * 256; e += 64) {
+                const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                Tmat[sw64(16 * I + r, 16 * J + cc)] = 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {           // block diagonal I - J = d
+            const int nb = 4 - d;               // blocks (J + d, J), J = 0 .. nb - 1
+            // X_J = sum_{M=J}^{J+d-1} A_{J+d,M} T_{M,J}
+            for (int e = tid; e < nb * 256; e += THREADS) {
+                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
+                float acc = 0.f;
+                for (int M = J; M < I; ++M)
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                __nv_bfloat16 hi, lo;
-                split2(tcol[r] * fw, hi, lo);
-                st_bf16(sm.tw[0], r, col, C, hi);
-                st_bf16(sm.tw[1], r, col, C, lo);
-                split2(tcol[r] * fu, hi, lo);
-                st_bf16(sm.tu[0], r, col, C, hi);
-                st_bf16(sm.tu[1], r, col, C, lo);
+                    for (int m = 0; m < 16; ++m)
+                        acc = fmaf(Amat[sw64(16 * I + r, 16 * M + m)], Tmat[sw64(16 * M + m, 16 * J + cc)], acc);
+                X[e] = acc;
+            }
+            __syncthreads();
+            // T_{I,J} = -T_{I,I} X_J
+            for (int e = tid; e < nb * 256; e += THREADS) {
+                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Tmat[sw64(16 * I + r, 16 * I + m)], X[(J << 8) + (m << 4) + cc], acc);
+                Tmat[sw64(16 * I + r, 16 * J + cc)] = -acc;
+            }
+            __syncthreads();
+        }
+        // T' = T diag(fw), T'' = T diag(beta): thread = (row, half of the columns)
+        {
+            const int r = tid >> 1, cbase = 32 * (tid & 1);
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                float tw8[8], tu8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int col = cbase + c + e;
+                    const float t = Tmat[sw64(r, col)];
+                    tw8[e] = t * sm.fw[col];
+                    tu8[e] = t * sm.beta[col];
+                }
+                st_row8(sm.tw[0], r, cbase + c, C, tw8, false);
+                st_row8(sm.tw[1], r, cbase + c, C, tw8, true);
+                st_row8(sm.tu[0], r, cbase + c, C, tu8, false);
+                st_row8(sm.tu[1], r, cbase + c, C, tu8, true);
             }
         }
         publish_smem();
@@ -394,82 +507,79 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
         if (!ok)
             break;
 
-        // ---- step 8: Delta^T (thread = v) into the hi / lo tiles [v][i] -------
+        // ---- step 8: Delta^T (thread = v) into the hi / lo tiles [v][i] of wd;
+        // Delta'^T = Delta^T diag(e^(gamma_last - gamma_i) rk_i) into the tw / tu
+        // area (free since W and U are done); the state in TMEM decayed ------
+        unsigned char *dp_hi = sm.tw[0];     // 128 x 64 bf16 (tw[0..1] contiguous)
+        unsigned char *dp_lo = sm.tu[0];     // 128 x 64 bf16 (tu[0..1] contiguous)
         {
-            float drow[64];
-#pragma unroll
-            for (int c = 0; c < 64; c += 16)
-                tc::tmem_ld16(my_lane + COL_DT + c, drow + c);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-                st_row8(sm.wd[0], tid, c, C, drow + c, false);
-                st_row8(sm.wd[1], tid, c, C, drow + c, true);
-            }
-        }
-        publish_smem();
-
-        // ---- step 9: O2^T = Delta^T P^T (3 split products) --------------------
-        if (tid == 0) {
-            mma_tiles(tmem + COL_O2, sm.wd[0], C, sm.p[0], C, C / 16, ID_M128_N64, false);
-            mma_tiles(tmem + COL_O2, sm.wd[0], C, sm.p[1], C, C / 16, ID_M128_N64, true);
-            mma_tiles(tmem + COL_O2, sm.wd[1], C, sm.p[0], C, C / 16, ID_M128_N64, true);
-            tc::mma_commit(&sm.mbar);
-        }
-        wait_mma();
-        if (!ok)
-            break;
-
-        // ---- step 10: outputs; Delta' for the state; decay the state ----------
-        {
-            const float gl = sm.gam[n - 1];
 #pragma unroll
             for (int cb = 0; cb < 64; cb += 16) {
-                float o1[16], o2[16], d[16];
-                tc::tmem_ld16(my_lane + COL_O1 + cb, o1);
-                tc::tmem_ld16(my_lane + COL_O2 + cb, o2);
+                float d[16];
                 tc::tmem_ld16(my_lane + COL_DT + cb, d);
                 tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int j = cb + e;
-                    if (j < n) {
-                        const float f = expf(sm.gam[j]) * sm.rqs[j];
-                        out[(bos + c0 + j) * p.o_tok + hv * p.o_head + tid] =
-                            __float2bfloat16_rn(fmaf(f, o1[e], o2[e]));
-                    }
-                    d[e] *= expf(gl - sm.gam[j]) * sm.rk[j];     // Delta' = Delta e^(gamma_last - gamma_i) rk_i
-                }
                 st_row8(sm.wd[0], tid, cb, C, d, false);
                 st_row8(sm.wd[0], tid, cb + 8, C, d + 8, false);
                 st_row8(sm.wd[1], tid, cb, C, d, true);
                 st_row8(sm.wd[1], tid, cb + 8, C, d + 8, true);
-            }
-            const float decay = expf(gl);
-            for (int k0 = 0; k0 < K; k0 += 16) {
-                float x[16];
-                tc::tmem_ld16(my_lane + COL_S + k0, x);
-                tc::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
+                    d[e] *= sm.fd[cb + e];
+                st_row8(dp_hi, tid, cb, C, d, false);
+                st_row8(dp_hi, tid, cb + 8, C, d + 8, false);
+                st_row8(dp_lo, tid, cb, C, d, true);
+                st_row8(dp_lo, tid, cb + 8, C, d + 8, true);
+            }
+            const float decay = expf(sm.gam[n - 1]);
+#pragma unroll
+            for (int k0 = 0; k0 < K; k0 += 64) {
+                float x[64];
+#pragma unroll
+                for (int e = 0; e < 64; e += 16)
+                    tc::tmem_ld16(my_lane + COL_S + k0 + e, x + e);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
                     x[e] *= decay;
-                tc::tmem_st16(my_lane + COL_S + k0, x);
+#pragma unroll
+                for (int e = 0; e < 64; e += 16)
+                    tc::tmem_st16(my_lane + COL_S + k0 + e, x + e);
             }
             tc::tmem_wait_st();
         }
         publish_smem();
 
-        // ---- step 11: S^T += Delta'^T K (2 split products, K exact) -----------
+        // ---- step 9: O2^T = Delta^T P^T (3 split products) and
+        //      S^T += Delta'^T K (2 split products, K exact), one batch ------
         if (tid == 0) {
-            mma_tiles(tmem + COL_S, sm.wd[0], C, sm.kt, C, C / 16, ID_M128_N128, true);
-            mma_tiles(tmem + COL_S, sm.wd[1], C, sm.kt, C, C / 16, ID_M128_N128, true);
+            mma_tiles(tmem + COL_O2, sm.wd[0], C, sm.p[0], C, C / 16, ID_M128_N64, false);
+            mma_tiles(tmem + COL_O2, sm.wd[0], C, sm.p[1], C, C / 16, ID_M128_N64, true);
+            mma_tiles(tmem + COL_O2, sm.wd[1], C, sm.p[0], C, C / 16, ID_M128_N64, true);
+            mma_tiles(tmem + COL_S, dp_hi, C, sm.kt, C, C / 16, ID_M128_N128, true);
+            mma_tiles(tmem + COL_S, dp_lo, C, sm.kt, C, C / 16, ID_M128_N128, true);
             tc::mma_commit(&sm.mbar);
         }
         wait_mma();
         if (!ok)
             break;
 
-        // ---- step 12: the next chunk's S^T tiles, or the final write-back -----
+        // ---- step 10: outputs o_j = fo_j (S0^T q_j) + (Delta^T P^T)_j ----------
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+            float o1[16], o2[16];
+            tc::tmem_ld16(my_lane + COL_O1 + cb, o1);
+            tc::tmem_ld16(my_lane + COL_O2 + cb, o2);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = cb + e;
+                if (j < n)
+                    out[(bos + c0 + j) * p.o_tok + hv * p.o_head + tid] =
+                        __float2bfloat16_rn(fmaf(sm.fo[j], o1[e], o2[e]));
+            }
+        }
+
+        // ---- step 11: the next chunk's S^T tiles, or the final write-back -----
         for (int k0 = 0; k0 < K; k0 += 16) {
             float x[16];
             tc::tmem_ld16(my_lane + COL_S + k0, x);
