@@ -598,6 +598,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_kernel(const __grid_cons
         publish_smem();
     }
 
+    pdl_trigger();
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0)

@@ -130,16 +130,16 @@ struct Act<float> {
     }
 };
 
-// Programmatic dependent launch: let the next kernel on the stream be
-// scheduled as soon as every CTA of this grid has started, then wait until the
-// previous kernel has completed (and its writes are visible) before touching
-// any input.  Both are no-ops when the grid was launched without the
-// programmatic-serialization attribute.
-__device__ __forceinline__ void pdl_prologue()
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
+// Programmatic dependent launch.  pdl_prologue: wait until the previous
+// kernel on the stream has completed (and its writes are visible) before
+// touching any input.  pdl_trigger: this CTA's main work is done -- once
+// every CTA of the grid has triggered or exited, the next kernel may be
+// scheduled (it still waits for this grid to complete before it reads).
+// Triggering late keeps the next grid's CTAs from occupying SM slots while
+// this grid still needs them.  Both are no-ops when the grid was launched
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_prologue() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void report(uint32_t *status, uint32_t bit)
 {
@@ -383,6 +383,8 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
         }
     }
 
+    pdl_trigger();
+
     // ---- write the slab back in place ------------------------------
     if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
 #pragma unroll
@@ -425,6 +427,7 @@ __global__ void __launch_bounds__(256) gdn_gating_kernel(const __grid_constant__
         else
             static_cast<__nv_bfloat16 *>(p.beta)[tok * p.beta_tok + hv * p.beta_head] = __float2bfloat16_rn(beta);
     }
+    pdl_trigger();
 }
 
 }  // namespace gdn

@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
             for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
                 mbar_wait(&sm.full[j % STAGES], (j / STAGES) & 1, &never);
         }
+        pdl_trigger();
         bulk_wait_all();
         return;
     }
