@@ -47,8 +47,8 @@ ROTATING_COPIES = 4
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": "842fcb401f4fe707c1ee3911332621979904277adacbc512894ea50c169da894",
-               "bytes_per_launch": 257372928 + 201082880}
+NCU_TRAFFIC = {"kernel_sha256": "c08e45ebe87627abb7984eca8562f11be4b413190b5c22dca9968bc6236879a8",
+               "workload": "decode_b512_hv8", "bytes_per_launch": 257378816 + 197948416}
 
 
 def kernel_source_hash() -> str:
@@ -129,9 +129,9 @@ class ClockSampler:
 # CPU oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_subset_seconds(w, seqs):
-    """Wall time of the oracle on a subset of sequences (its own inputs)."""
-    import oracle
+def oracle_subset_args(w, seqs):
+    """The oracle's inputs for a subset of sequences (a compact pool holding
+    only their live slots)."""
     lens = w.seq_lens
     starts = np.concatenate([[0], np.cumsum(lens)])
     rows = np.concatenate([np.arange(starts[i], starts[i] + lens[i]) for i in seqs])
@@ -144,6 +144,13 @@ def oracle_subset_seconds(w, seqs):
     cu[1:] = np.cumsum(lens[seqs])
     args = (flat(w.q, 2), flat(w.k, 2), flat(w.v, 2), flat(w.a, 1), flat(w.b, 1), w.A_log, w.dt_bias,
             np.ascontiguousarray(w.state_pool[slots[live]]), idx, cu)
+    return args
+
+
+def oracle_subset_seconds(w, seqs):
+    """Wall time of the oracle on a subset of sequences (its own inputs)."""
+    import oracle
+    args = oracle_subset_args(w, seqs)
     t0 = time.perf_counter()
     oracle.update(*args)
     return time.perf_counter() - t0
@@ -164,6 +171,7 @@ def cpu_baseline(w, budget_s=10.0):
     """The oracle as it stands, single-threaded, over the whole workload
     repeated until about ``budget_s`` seconds of CPU work."""
     seqs = np.arange(w.spec.N)
+    oracle_subset_seconds(w, seqs[:1])   # untimed: loads the oracle library
     total_t, reps = 0.0, 0
     while reps == 0 or total_t < budget_s:
         total_t += oracle_subset_seconds(w, seqs)
@@ -175,10 +183,36 @@ def cpu_baseline(w, budget_s=10.0):
                       f"{total_t:.1f} s single-threaded fp64 C loop nest"}
 
 
+def cpu_baseline_all_cores(w, budget_s=10.0):
+    """The same oracle, unchanged, run on all host cores: the sequences are
+    split into one contiguous group per core and each group is one oracle
+    call on its own thread (the C loop nest runs without the interpreter
+    lock)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    cores = max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
+    groups = [g for g in np.array_split(np.arange(w.spec.N), cores) if len(g)]
+    args = [oracle_subset_args(w, g) for g in groups]
+    total_t, reps = 0.0, 0
+    oracle_subset_seconds(w, groups[0][:1])   # untimed: loads the oracle library
+    with ThreadPoolExecutor(len(groups)) as pool:
+        while reps == 0 or total_t < budget_s:
+            t0 = time.perf_counter()
+            list(pool.map(lambda a: oracle.update(*a), args))
+            total_t += time.perf_counter() - t0
+            reps += 1
+    per = total_t / reps
+    return {"value": round(wl.algorithmic_bytes(w) / per / 1e9, 4), "unit": "GB/s", "cores": len(groups),
+            "kind": "oracle", "us_per_call": round(per * 1e6, 1),
+            "sample": f"whole {w.spec.name} workload split into {len(groups)} sequence groups, one thread each, "
+                      f"{reps} repetitions, {total_t:.1f} s"}
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle on bounded per-step samples."""
     N = w.spec.N
     rng = np.random.default_rng(0)
+    oracle_subset_seconds(w, np.arange(1))   # untimed: loads the oracle library
     t1 = oracle_subset_seconds(w, np.arange(min(8, N))) / min(8, N)
     budget = 120.0
     per_step = max(1, min(N, int(budget / max(1, args.steps + args.warmup) / max(t1, 1e-6))))
@@ -347,6 +381,21 @@ def main():
     ms_per_step = max_region_ms / args.steps
     value = nbytes * world * args.steps / (max_region_ms * 1e-3) / 1e9
 
+    # per-launch distribution: isolated launches, each bracketed by its own
+    # events (so programmatic dependent launch cannot overlap neighbours)
+    dist_n = min(args.steps, 300)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(dist_n)]
+    for s_, (a_, b_) in enumerate(ev):
+        a_.record(stream)
+        calls[s_ % len(calls)]()
+        b_.record(stream)
+    torch.cuda.synchronize(device)
+    per_launch = np.array([a_.elapsed_time(b_) * 1e3 for a_, b_ in ev])
+    launch_us = {"p10": round(float(np.percentile(per_launch, 10)), 3),
+                 "p50": round(float(np.percentile(per_launch, 50)), 3),
+                 "p90": round(float(np.percentile(per_launch, 90)), 3), "launches": dist_n,
+                 "how": "isolated launches, CUDA events around each, inputs rotating over the copies"}
+
     # end to end through the public API with pinned host buffers: each step
     # copies its inputs host -> device (one packed copy), launches, copies the
     # output back and synchronises on it
@@ -387,7 +436,9 @@ def main():
         peak, peak_src = hbm_peak()
         achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
         traffic = None
-        if NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash() and not args.unfused:
+        if (NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.spec.name
+                and not args.unfused and args.schedule in ("auto", "per_tile") and not args.tile_v
+                and not args.tile_rows):
             traffic = NCU_TRAFFIC["bytes_per_launch"]
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -395,6 +446,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(w, world, args.pdl),
             "us_per_call": round(avg_kernel_ms * 1e3, 3),
+            "launch_us": launch_us,
             "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                          "peak_source": peak_src},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
@@ -406,10 +458,12 @@ def main():
                                                w.spec.N * w.spec.HV)},
             "e2e": e2e,
             "gpu_launches": args.steps * (2 if args.unfused else 1),
+            "gpu_launches_note": "launches inside the timed region; the per-launch distribution and e2e run after it",
             "clocks": clocks,
         }
         if world == 1 and not args.skip_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
+            line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w)
         print(json.dumps(line), flush=True)
 
     del calls
