@@ -43,22 +43,30 @@ METRIC = "µs/call and state GB/s (% of B200 HBM peak) at B=512, HV=8, K=V=128"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 ROTATING_COPIES = 4
+# the library's GDN_SCHEDULE_AUTO thresholds (mean tokens per sequence) for
+# the chunked kernel, as documented in include/gdn_decode.h
+
+
+def chunked_min_mean_tokens(pairs):
+    return 128 if pairs <= 1024 else 256
 
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": "c08e45ebe87627abb7984eca8562f11be4b413190b5c22dca9968bc6236879a8",
+NCU_TRAFFIC = {"kernel_sha256": "f6b891eb3ef14a8b7d52962a1f3d8ee3936fd0e76d342ecfa9ca84115a87cc36",
                "workload": "decode_b512_hv8", "bytes_per_launch": 257378816 + 197948416}
 
 
 def kernel_source_hash() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "gated_deltanet_recurrent_sigmoid_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
-    return h.hexdigest()
+    """Hash of the per-tile kernel's device code (the kernel the traffic figure
+    belongs to)."""
+    with open(os.path.join(ROOT, "gated_deltanet_recurrent_sigmoid_b200", "csrc", "gdn_decode_kernel.cuh"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+# fp32 CUDA-core bound of the per-token arithmetic: 148 SMs x 128 fp32 lanes x
+# 2 flops per FMA x the 1965 MHz maximum SM clock (B200 unit counts).
+ALU_F32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def hbm_peak():
@@ -239,10 +247,13 @@ def run_reference(args, w):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def kernel_name(schedule, tile_v, tile_rows, one_token, pairs):
+def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, chunk_ok=False):
     """Name of the kernel the library launches for these settings (mirrors
     the library's documented choice)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
+    if (schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok
+            and mean_tokens >= chunked_min_mean_tokens(pairs)):
+        schedule = binding.SCHEDULE_CHUNKED
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
     if schedule == binding.SCHEDULE_CHUNKED:
@@ -257,7 +268,8 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs):
 
 def workload_config(w, world, pdl=False):
     s = w.spec
-    return {"workload": s.name, "B": s.N, "T": s.T if s.T is not None else "U{1..64}", "H": s.H, "HV": s.HV,
+    return {"workload": s.name, "B": s.N, "T": s.T if s.T is not None else f"U{{{s.min_len}..{s.max_len}}}",
+            "H": s.H, "HV": s.HV,
             "K": s.K, "V": s.V, "num_slots": s.num_slots, "padded": int((w.state_indices < 0).sum()),
             "state_dtype": "f32", "activation_dtype": "bf16",
             "l2": f"inputs larger than L2: steps rotate over {ROTATING_COPIES} input copies",
@@ -435,6 +447,8 @@ def main():
     if rank == 0:
         peak, peak_src = hbm_peak()
         achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
+        nflops = wl.algorithmic_flops(w)
+        alu_bound = nflops / (ALU_F32_PEAK_TFLOPS * 1e12) > nbytes / (peak * 1e9)
         traffic = None
         if (NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.spec.name
                 and not args.unfused and args.schedule in ("auto", "per_tile") and not args.tile_v
@@ -449,13 +463,20 @@ def main():
             "launch_us": launch_us,
             "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                          "peak_source": peak_src},
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
+            "roofline": ({"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                          "frac": round(achieved / peak, 4)} if not alu_bound else
+                         {"bound": "alu", "achieved": round(nflops / (avg_kernel_ms * 1e-3) / 1e12, 3),
+                          "peak": round(ALU_F32_PEAK_TFLOPS, 2), "unit": "TFLOP/s",
+                          "frac": round(nflops / (avg_kernel_ms * 1e-3) / 1e12 / ALU_F32_PEAK_TFLOPS, 4),
+                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                          "hbm_frac": round(achieved / peak, 4)}) | {
+                         "traffic": traffic, "algorithmic_bytes_per_launch": nbytes,
+                         "algorithmic_flops_per_launch": nflops, "hbm_peak_source": peak_src,
                          "kernel": ("gdn::gdn_gating_kernel + " if args.unfused else "") +
                                    kernel_name(schedule, args.tile_v, args.tile_rows,
                                                w.T_tot == w.spec.N and not w.spec.intermediate,
-                                               w.spec.N * w.spec.HV)},
+                                               w.spec.N * w.spec.HV, w.T_tot / max(1, w.spec.N),
+                                               not args.unfused and not w.spec.intermediate)},
             "e2e": e2e,
             "gpu_launches": args.steps * (2 if args.unfused else 1),
             "gpu_launches_note": "launches inside the timed region; the per-launch distribution and e2e run after it",

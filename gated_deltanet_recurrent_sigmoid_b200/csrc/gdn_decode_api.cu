@@ -21,6 +21,14 @@ namespace {
 
 constexpr int kHeadK = 128;
 constexpr int kHeadV = 128;
+// GDN_SCHEDULE_AUTO takes the chunked kernel when the batch holds at least
+// this many tokens per sequence on average: 128 while there are at most 1024
+// (sequence, value head) pairs, 256 beyond (the measured B200 crossovers:
+// with 64-1024 pairs the chunked kernel is 0.82-0.97 of the per-tile time at
+// ~128 tokens; with 4096 pairs it needs ~250).
+constexpr int64_t kChunkedMinMeanTokensFew = 128;
+constexpr int64_t kChunkedMinMeanTokensMany = 256;
+constexpr int64_t kChunkedFewPairs = 1024;
 
 int64_t elem_size(int32_t dtype)
 {
@@ -302,7 +310,7 @@ int run_update(const UpdateArgs &c)
         GDN_L2NORM_QK | GDN_WRITE_INTERMEDIATE | GDN_NO_FINAL_WRITEBACK | GDN_CHECK_INDICES | GDN_LAUNCH_PDL;
     if ((flags & ~known) != 0 || !std::isfinite(c.scale) || !(c.scale > 0.f))
         return GDN_ERR_ARG;
-    const int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
+    int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
     if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED &&
         schedule != GDN_SCHEDULE_CHUNKED)
         return GDN_ERR_ARG;
@@ -482,6 +490,15 @@ int run_update(const UpdateArgs &c)
                          (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
     if (!tile_ok)
         return GDN_ERR_UNSUPPORTED;
+    // The library's schedule: the chunked tensor-core kernel when the
+    // sequences are long on average (and it is built for the call), else the
+    // per-tile kernel.
+    const bool v_rows_16b =
+        aligned(v->data, 16) && stride_ok(T_tot, Lv.tok, 8) && stride_ok(HV, v->stride[v->ndim - 2], 8);
+    if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
+        act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0 &&
+        T_tot >= (N * HV <= kChunkedFewPairs ? kChunkedMinMeanTokensFew : kChunkedMinMeanTokensMany) * N)
+        schedule = GDN_SCHEDULE_CHUNKED;
     // The pipelined schedule is built for bf16 activations and fused bf16
     // gates; the chunked one for bf16 activations, fused gates and no
     // per-token states.
@@ -491,8 +508,7 @@ int run_update(const UpdateArgs &c)
     if (schedule == GDN_SCHEDULE_CHUNKED && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
         return GDN_ERR_UNSUPPORTED;
     // the chunked kernel reads v rows 16 bytes at a time, like q and k
-    if (schedule == GDN_SCHEDULE_CHUNKED &&
-        (!aligned(v->data, 16) || !stride_ok(T_tot, Lv.tok, 8) || !stride_ok(HV, v->stride[v->ndim - 2], 8)))
+    if (schedule == GDN_SCHEDULE_CHUNKED && !v_rows_16b)
         return GDN_ERR_ALIGN;
     const int64_t units = N * HV;
     if (units * (kHeadV / tile_v) > INT32_MAX)

@@ -122,7 +122,13 @@ extern "C" {
 #define GDN_ERR_CUDA        (-9) /* the CUDA runtime refused the launch or copy */
 
 /* work schedules (gdn_extra.schedule); all compute the same update */
-#define GDN_SCHEDULE_AUTO      0 /* library choice */
+#define GDN_SCHEDULE_AUTO      0 /* library choice: GDN_SCHEDULE_CHUNKED when the
+                                    call qualifies for it (bf16 activations, fused
+                                    gates, no per-token states, v rows 16-byte
+                                    aligned) and holds enough tokens per
+                                    sequence on average: >= 128 when N * HV <=
+                                    1024, else >= 256 (total tokens >= 128 N or
+                                    256 N); else GDN_SCHEDULE_PER_TILE */
 #define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
                                     state tile moves through registers.  Tiles
                                     (tile_v x tile_rows): 16x16, 32x16, 32x32,

@@ -126,3 +126,27 @@ def test_chunked_device_status():
     ost, o_ref, s_ref, _ = run_oracle(w)
     assert status == ost == oracle.BAD_SLOT
     assert_out_close(out_as_f32(d["out"]), o_ref)
+
+
+def _bits_equal(a, b):
+    return torch.equal(a["state_pool"], b["state_pool"]) and torch.equal(a["out"], b["out"])
+
+
+def test_auto_schedule_picks_chunked_for_long_sequences():
+    """GDN_SCHEDULE_AUTO: mean length >= 128 with few (sequence, head) pairs
+    runs the chunked kernel (bit-identical to asking for it); short
+    sequences, or a call with per-token states, run the per-tile kernel."""
+    long_w = problem([200, 150, 300], seed=21)
+    auto, _, _ = run_gpu(long_w)
+    chunked, _, _ = run_gpu(long_w, schedule=CHUNKED)
+    per_tile, _, _ = run_gpu(long_w, schedule=binding.SCHEDULE_PER_TILE)
+    assert _bits_equal(auto, chunked) and not _bits_equal(auto, per_tile)
+
+    short_w = problem([3, 60, 10], seed=22)
+    auto, _, _ = run_gpu(short_w)
+    per_tile, _, _ = run_gpu(short_w, schedule=binding.SCHEDULE_PER_TILE)
+    assert _bits_equal(auto, per_tile)
+
+    auto_d, _, auto_i = run_gpu(long_w, inter=True)
+    pt_d, _, pt_i = run_gpu(long_w, inter=True, schedule=binding.SCHEDULE_PER_TILE)
+    assert _bits_equal(auto_d, pt_d) and torch.equal(auto_i, pt_i)
