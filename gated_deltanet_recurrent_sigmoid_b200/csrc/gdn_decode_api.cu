@@ -467,7 +467,7 @@ int run_update(const UpdateArgs &c)
     if (one_token) {
         tile_v = 64;
         tile_rows = 32;
-    } else if (pairs >= 4096) {
+    } else if (pairs >= 2048) {
         tile_v = 32;
         tile_rows = 32;
     } else {

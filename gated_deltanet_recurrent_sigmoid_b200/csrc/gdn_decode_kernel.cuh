@@ -22,7 +22,9 @@
 //     delta = beta * (v - decay * u * rk)                (S^T k^ on the decayed S)
 //     o     = decay * w * qs + (k^ . q^) * delta         (= S'^T q^ after the update)
 //     S'    = decay * S + k^ delta^T
-// which is the update of the header rearranged so that S is read once.
+// which is the update of the header rearranged so that S is read once.  The
+// registers hold S / cs for a per-CTA scale cs that absorbs the decays, so
+// the update costs one FMA per element (see the token loop).
 //
 // Template parameters: the activation element type TAct (q, k, v, out:
 // bf16 or fp32) and GIVEN_GATES (false: decay and beta come from A_log, a,
@@ -262,6 +264,14 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
     };
     fetch(bos);
 
+    // The registers hold the state divided by a per-CTA scale cs (S = cs * s),
+    // so that a token's decay multiplies cs instead of every element: the
+    // update becomes s += k (rk / cs') delta^T with cs' = cs decay, one FMA
+    // per element.  When cs' leaves [2^-60, 2^60] the decay is applied to
+    // the elements instead and cs returns to 1, so s never overflows and
+    // 1 / cs' stays finite (this also covers decays that underflow to 0).
+    float cs = 1.f;
+
     for (int t = 0; t < len; ++t) {
         const int64_t tok = bos + t;
 
@@ -348,26 +358,43 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             const float x = a_t + dt_b;
             const float sp = x > 20.f ? x : log1pf(expf(x));
             decay = expf(neg_A * sp);
-            beta = 1.f / (1.f + expf(-b_t));
+            beta = __fdividef(1.f, 1.f + expf(-b_t));   // 0 for b = -inf
         }
         const float kq = SKQ * rk * qs;
 
         // ---- delta and output ----------------------------------
-        const float dku = decay * rk;
-        const float dwq = decay * qs;
+        const float cn = cs * decay;        // scale of the decayed state
+        const float dku = cn * rk;
+        const float dwq = cn * qs;
         const float d0 = beta * (v_t.x - dku * U.x);
         const float d1 = beta * (v_t.y - dku * U.y);
         const float d2 = beta * (v_t.z - dku * U.z);
         const float d3 = beta * (v_t.w - dku * U.w);
 
         // ---- S <- decay S + k^ delta^T -----------------------------
+        if (cn >= 0x1p-60f && cn <= 0x1p60f) {
+            // s <- s + k (rk / cs') delta^T; the scale becomes cs'
+            const float f = rk * __fdividef(1.f, cn);
+            const float e0 = d0 * f, e1 = d1 * f, e2 = d2 * f, e3 = d3 * f;
 #pragma unroll
-        for (int j = 0; j < R; ++j) {
-            const float kh = kr[j] * rk;
-            s[j].x = fmaf(kh, d0, decay * s[j].x);
-            s[j].y = fmaf(kh, d1, decay * s[j].y);
-            s[j].z = fmaf(kh, d2, decay * s[j].z);
-            s[j].w = fmaf(kh, d3, decay * s[j].w);
+            for (int j = 0; j < R; ++j) {
+                s[j].x = fmaf(kr[j], e0, s[j].x);
+                s[j].y = fmaf(kr[j], e1, s[j].y);
+                s[j].z = fmaf(kr[j], e2, s[j].z);
+                s[j].w = fmaf(kr[j], e3, s[j].w);
+            }
+            cs = cn;
+        } else {
+            // apply the scale to the elements: s <- cs' s + k^ delta^T, cs = 1
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                const float kh = kr[j] * rk;
+                s[j].x = fmaf(kh, d0, cn * s[j].x);
+                s[j].y = fmaf(kh, d1, cn * s[j].y);
+                s[j].z = fmaf(kh, d2, cn * s[j].z);
+                s[j].w = fmaf(kh, d3, cn * s[j].w);
+            }
+            cs = 1.f;
         }
 
         if (kg == 0)
@@ -379,7 +406,7 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
             float *ip = p.inter + tok * p.i_tok + hv * p.i_head + static_cast<int64_t>(row0) * V + col0;
 #pragma unroll
             for (int j = 0; j < R; ++j)
-                __stcs(reinterpret_cast<float4 *>(ip + j * V), s[j]);
+                __stcs(reinterpret_cast<float4 *>(ip + j * V), make_float4(cs * s[j].x, cs * s[j].y, cs * s[j].z, cs * s[j].w));
         }
     }
 
@@ -389,7 +416,7 @@ gdn_decode_kernel(const __grid_constant__ DecodeParams p)
     if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
 #pragma unroll
         for (int j = 0; j < R; ++j)
-            __stcs(reinterpret_cast<float4 *>(s_ptr + j * V), s[j]);
+            __stcs(reinterpret_cast<float4 *>(s_ptr + j * V), make_float4(cs * s[j].x, cs * s[j].y, cs * s[j].z, cs * s[j].w));
     }
 }
 

@@ -134,7 +134,7 @@ extern "C" {
                                     (tile_v x tile_rows): 16x16, 32x16, 32x32,
                                     64x16, 64x32.  Library choice: 64x32 when
                                     every sequence has one token, else 32x32
-                                    with >= 4096 (sequence, value head) pairs,
+                                    with >= 2048 (sequence, value head) pairs,
                                     else 16x16; with fp32 activations 32x16
                                     for one token, else 16x16 */
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
