@@ -253,7 +253,9 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if (schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok
             and mean_tokens >= chunked_min_mean_tokens(pairs)):
-        schedule = binding.SCHEDULE_CHUNKED
+        schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
+    if schedule == binding.SCHEDULE_CHUNKED_SPLIT:
+        return "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
     if schedule == binding.SCHEDULE_CHUNKED:
@@ -300,7 +302,7 @@ def main():
     ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
     ap.add_argument("--tile-v", type=int, default=0)
     ap.add_argument("--tile-rows", type=int, default=0)
-    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -337,7 +339,8 @@ def main():
     binding.load()
 
     schedule = {"auto": binding.SCHEDULE_AUTO, "per_tile": binding.SCHEDULE_PER_TILE,
-                "pipelined": binding.SCHEDULE_PIPELINED, "chunked": binding.SCHEDULE_CHUNKED}[args.schedule]
+                "pipelined": binding.SCHEDULE_PIPELINED, "chunked": binding.SCHEDULE_CHUNKED,
+                "split": binding.SCHEDULE_CHUNKED_SPLIT}[args.schedule]
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
@@ -454,6 +457,9 @@ def main():
                 and not args.unfused and args.schedule in ("auto", "per_tile") and not args.tile_v
                 and not args.tile_rows):
             traffic = NCU_TRAFFIC["bytes_per_launch"]
+        kname = ("gdn::gdn_gating_kernel + " if args.unfused else "") + kernel_name(
+            schedule, args.tile_v, args.tile_rows, w.T_tot == w.spec.N and not w.spec.intermediate,
+            w.spec.N * w.spec.HV, w.T_tot / max(1, w.spec.N), not args.unfused and not w.spec.intermediate)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
@@ -472,13 +478,9 @@ def main():
                           "hbm_frac": round(achieved / peak, 4)}) | {
                          "traffic": traffic, "algorithmic_bytes_per_launch": nbytes,
                          "algorithmic_flops_per_launch": nflops, "hbm_peak_source": peak_src,
-                         "kernel": ("gdn::gdn_gating_kernel + " if args.unfused else "") +
-                                   kernel_name(schedule, args.tile_v, args.tile_rows,
-                                               w.T_tot == w.spec.N and not w.spec.intermediate,
-                                               w.spec.N * w.spec.HV, w.T_tot / max(1, w.spec.N),
-                                               not args.unfused and not w.spec.intermediate)},
+                         "kernel": kname},
             "e2e": e2e,
-            "gpu_launches": args.steps * (2 if args.unfused else 1),
+            "gpu_launches": args.steps * (2 if args.unfused or "+" in kname else 1),
             "gpu_launches_note": "launches inside the timed region; the per-launch distribution and e2e run after it",
             "clocks": clocks,
         }

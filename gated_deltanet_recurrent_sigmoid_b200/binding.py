@@ -31,6 +31,7 @@ SCHEDULE_AUTO = 0
 SCHEDULE_PER_TILE = 1
 SCHEDULE_PIPELINED = 2
 SCHEDULE_CHUNKED = 3
+SCHEDULE_CHUNKED_SPLIT = 4
 
 OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5
@@ -55,7 +56,8 @@ class GdnTensor(ctypes.Structure):
 class GdnExtra(ctypes.Structure):
     _fields_ = [("stream", ctypes.c_void_p), ("intermediate_states", ctypes.POINTER(GdnTensor)),
                 ("device_status", ctypes.c_void_p), ("tile_v", ctypes.c_int32),
-                ("tile_rows", ctypes.c_int32), ("schedule", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("tile_rows", ctypes.c_int32), ("schedule", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64)]
 
 
 _LIB = None
@@ -85,6 +87,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_version.restype = ctypes.c_int
         lib.gdn_version.argtypes = []
+        lib.gdn_chunked_workspace_bytes.restype = ctypes.c_uint64
+        lib.gdn_chunked_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
         _LIB = lib
     return _LIB
 
@@ -113,6 +117,33 @@ def _ref(d: Optional[GdnTensor]):
     return None if d is None else ctypes.byref(d)
 
 
+def chunked_workspace_bytes(T_tot: int, HV: int) -> int:
+    """Workspace bytes of GDN_SCHEDULE_CHUNKED_SPLIT (gdn_chunked_workspace_bytes)."""
+    return int(load().gdn_chunked_workspace_bytes(int(T_tot), int(HV)))
+
+
+def _workspace_for(workspace, schedule: int, q: torch.Tensor, v: torch.Tensor, N: int):
+    """The workspace to pass: the caller's tensor, or (workspace="auto") one
+    allocated here when the split chunked schedule is asked for, or when the
+    library may choose it (AUTO with at least 128 tokens per sequence on
+    average -- the library's lowest threshold for the chunked kernels)."""
+    if workspace is None or isinstance(workspace, torch.Tensor):
+        return workspace
+    if workspace != "auto":
+        raise ValueError("workspace must be a tensor, None or 'auto'")
+    T_tot = v.numel() // (v.shape[-1] * v.shape[-2]) if v.dim() >= 2 else 0
+    HV = v.shape[-2] if v.dim() >= 2 else 0
+    if not (schedule == SCHEDULE_CHUNKED_SPLIT or (schedule == SCHEDULE_AUTO and N > 0 and T_tot >= 128 * N)):
+        return None
+    nbytes = chunked_workspace_bytes(T_tot, HV)
+    return torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+
+
+def _set_workspace(extra: GdnExtra, ws: Optional[torch.Tensor]) -> None:
+    extra.workspace = ws.data_ptr() if ws is not None and ws.numel() else None
+    extra.workspace_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+
+
 def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
                   A_log: torch.Tensor, dt_bias: torch.Tensor, state_pool: torch.Tensor,
                   state_indices: torch.Tensor, cu_seqlens: Optional[torch.Tensor], out: torch.Tensor,
@@ -120,14 +151,17 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
                   intermediate_states: Optional[torch.Tensor] = None,
                   device_status: Optional[torch.Tensor] = None,
                   stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
-                  schedule: int = SCHEDULE_AUTO, tile_rows: int = 0) -> torch.Tensor:
+                  schedule: int = SCHEDULE_AUTO, tile_rows: int = 0, workspace="auto") -> torch.Tensor:
     """Fused sigmoid-gating GDN decode update, in place on ``state_pool``.
 
     Shapes, dtypes and semantics are those of ``gdn_decode_update`` in
     include/gdn_decode.h.  ``scale`` defaults to 1/sqrt(K).  ``flags`` gets
     WRITE_INTERMEDIATE added automatically when ``intermediate_states`` is
     given.  Runs asynchronously on ``stream`` (default: the current torch
-    stream).  Returns ``out``.  Raises GdnError on a non-zero status.
+    stream).  ``workspace``: a uint8 device tensor for the split chunked
+    schedule, None, or "auto" (allocated here with torch when that schedule
+    is asked for or may be chosen).  Returns ``out``.  Raises GdnError on a
+    non-zero status.
     """
     lib = load()
     if scale is None:
@@ -145,6 +179,8 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     extra.tile_v = int(tile_v)
     extra.tile_rows = int(tile_rows)
     extra.schedule = int(schedule)
+    ws = _workspace_for(workspace, schedule, q, v, state_indices.shape[0])
+    _set_workspace(extra, ws)
     status = lib.gdn_decode_update(*[_ref(d) for d in descs], ctypes.c_float(scale), ctypes.c_uint32(flags),
                                    ctypes.byref(extra))
     if status != OK:
@@ -239,7 +275,7 @@ class PreparedCall:
     def __init__(self, q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
                  scale: Optional[float] = None, flags: int = L2NORM_QK, intermediate_states=None,
                  device_status=None, stream: Optional[torch.cuda.Stream] = None, tile_v: int = 0,
-                 schedule: int = SCHEDULE_AUTO, tile_rows: int = 0):
+                 schedule: int = SCHEDULE_AUTO, tile_rows: int = 0, workspace="auto"):
         self._lib = load()
         self._keep = (q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out,
                       intermediate_states, device_status)
@@ -257,6 +293,8 @@ class PreparedCall:
         self._extra.tile_v = int(tile_v)
         self._extra.tile_rows = int(tile_rows)
         self._extra.schedule = int(schedule)
+        self.workspace = _workspace_for(workspace, schedule, q, v, state_indices.shape[0])
+        _set_workspace(self._extra, self.workspace)
         self._args = [_ref(d) for d in self._descs] + [ctypes.c_float(scale), ctypes.c_uint32(flags),
                                                        ctypes.byref(self._extra)]
         self._fn = self._lib.gdn_decode_update

@@ -1,0 +1,790 @@
+// gdn_chunk_split.cuh -- the chunked Gated DeltaNet update split into two
+// sm_100a kernels around a caller-provided workspace (GDN_SCHEDULE_CHUNKED_SPLIT).
+//
+// The chunk form of gdn_chunk_kernel.cuh has two kinds of work per chunk:
+// products that need only the chunk's own inputs (the decay scan, A, the
+// triangular solve T = (I + A)^-1, W, U and the masked q.k matrix P -- the
+// pages' chunk_scaled_dot_kkt, solve_tril and recompute_w_u steps) and the
+// recurrence through the state (Delta = U - W S0, the outputs, the state
+// update -- chunk_gated_delta_rule_fwd_h and chunk_fwd_o).  The single-kernel
+// schedule runs both in one CTA per (sequence, head), chunk after chunk, so
+// the state-independent work sits on the sequential critical path.  Here:
+//
+//   gdn_chunk_wy_kernel     one CTA per (64-token block of the packed token
+//                           range, value head), all in parallel: writes the
+//                           block's W, U^T, P, K'^T = (diag(fd) K)^T and raw Q
+//                           into the workspace as the byte images of the
+//                           operand tiles the second kernel feeds to tcgen05.
+//   gdn_chunk_state_kernel  one CTA per (sequence, value head): walks the
+//                           blocks the sequence covers, fetching each block's
+//                           tiles with bulk copies one step ahead, and runs
+//                           only the state-dependent products.
+//
+// Blocks are aligned to the packed token range, not to sequences: a block may
+// hold the end of one sequence and the start of the next.  Each token's
+// quantities are therefore taken within its SEGMENT (the part of its sequence
+// inside the block): the decay scan restarts at the segment start and A, P
+// are masked to the segment, which makes T, W, U block-diagonal by segment.
+// The state kernel processes a sequence as the pieces it has in each block.
+//
+// Within a segment, with gamma_j the running sum of g from the segment start,
+// hats the normalised vectors and S0 the state before the piece:
+//     A[j][i] = beta_j e^(gamma_j - gamma_i) k^_j . k^_i   (i < j, same segment)
+//     T = (I + A)^-1,  W = T diag(beta e^gamma rk) K,  U = T diag(beta) V
+//     Delta  = U - W S0
+//     o_j    = e^gamma_j rqs_j S0^T q_j + sum_i P[j][i] Delta_i,
+//              P[j][i] = e^(gamma_j - gamma_i) rqs_j rk_i q_j . k_i  (i <= j, same segment)
+//     S'     = e^gamma_last S0 + sum_i fd_i k_i Delta_i^T,  fd_i = e^(gamma_last - gamma_i) rk_i
+// Operands that are not exact bf16 are split into bf16 hi + lo parts and
+// multiplied as hi*hi + hi*lo + lo*hi (fp32 accumulators in TMEM), as in the
+// single-kernel schedule.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gdn_chunk_kernel.cuh"
+#include "gdn_decode.h"
+#include "gdn_decode_kernel.cuh"
+#include "mbarrier_sm100.cuh"
+#include "tc_sm100.cuh"
+
+namespace gdn {
+namespace split {
+
+using chunk::mma_tiles;
+using chunk::split2;
+using chunk::st_bf16;
+using chunk::st_row8;
+using chunk::sw64;
+using chunk::transpose8x8;
+
+constexpr int K = 128;
+constexpr int V = 128;
+constexpr int C = 64;            // tokens per block
+constexpr int THREADS = 128;
+
+// One workspace record per (block, value head): byte offsets.  Tiles are in
+// the K-major core-matrix layout of tc_sm100.cuh; [r][c] names the rows and
+// the contraction dimension.
+constexpr uint32_t REC_W_HI = 0;          // W hi              [i][k]   16 KB
+constexpr uint32_t REC_W_LO = 16384;      // W lo              [i][k]   16 KB
+constexpr uint32_t REC_Q = 32768;         // raw q             [j][k]   16 KB
+constexpr uint32_t REC_KP_HI = 49152;     // K'^T hi           [k][i]   16 KB
+constexpr uint32_t REC_KP_LO = 65536;     // K'^T lo           [k][i]   16 KB
+constexpr uint32_t REC_P_HI = 81920;      // P hi              [j][i]    8 KB
+constexpr uint32_t REC_P_LO = 90112;      // P lo              [j][i]    8 KB
+constexpr uint32_t REC_UT = 98304;        // U^T fp32, row-major [v][i]  32 KB
+constexpr uint32_t REC_FO = 131072;       // fo_j = e^gamma_j rqs_j     256 B
+constexpr uint32_t REC_GAM = 131328;      // gamma_j                    256 B
+constexpr uint32_t REC_BYTES = 131584;    // a multiple of 256
+constexpr uint32_t REC_A_BYTES = REC_KP_HI;               // W hi, W lo, Q
+constexpr uint32_t REC_B_BYTES = REC_UT - REC_KP_HI;      // K'^T hi / lo, P hi / lo
+constexpr uint32_t REC_S_BYTES = REC_BYTES - REC_FO;      // fo, gamma
+
+__host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV)
+{
+    return static_cast<uint64_t>((T_tot + C - 1) / C) * static_cast<uint64_t>(HV) * REC_BYTES;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: the state-independent products of one (block, value head).
+// ---------------------------------------------------------------------------
+struct WySmem {
+    // raw k rows 0..63 and q rows 64..127 [r][k]; after the K K^T / Q K^T
+    // product: A and T (fp32 64 x 64 each, swizzled); after the solve: the W
+    // hi / lo tiles staged for the bulk store
+    alignas(1024) unsigned char kq[128 * 128 * 2];
+    alignas(1024) unsigned char kt[128 * 64 * 2];     // raw k^T [k][i]
+    alignas(1024) unsigned char vt[128 * 64 * 2];     // raw v^T [v][i]
+    alignas(1024) unsigned char tw[2][64 * 64 * 2];   // T diag(fw) hi / lo [j][i]; tw[0] first holds solve scratch
+    alignas(1024) unsigned char tu[2][64 * 64 * 2];   // T diag(beta) hi / lo [j][i]
+    float kk[C], qq[C];                                // |k_j|^2, |q_j|^2
+    float rk[C], rqs[C], g[C], beta[C], gam[C];
+    float fa[C], fw[C], fo[C], fd[C];
+    int ss[C], se[C];                                  // segment [ss, se) of row j within the block
+    unsigned long long mbar;
+    uint32_t tmem_base;
+    int failed;
+};
+
+constexpr uint32_t WY_TMEM_COLS = 256;
+constexpr uint32_t WY_COL_KQ = 0;     // [K;Q] K^T  [r][i]   64 columns
+constexpr uint32_t WY_COL_WT = 64;    // W^T        [k][j]   64
+constexpr uint32_t WY_COL_UT = 128;   // U^T        [v][j]   64
+
+template <bool L2NORM>
+__global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_constant__ DecodeParams p,
+                                                                unsigned char *__restrict__ ws)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    WySmem &sm = *reinterpret_cast<WySmem *>(smem_raw);
+
+    pdl_prologue();
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int blk = blockIdx.x / p.HV;
+    const int hv = blockIdx.x - blk * p.HV;
+    const int h = hv / p.G;
+    const int64_t t0 = static_cast<int64_t>(blk) * C;
+    const int n = p.T_tot - t0 < C ? static_cast<int>(p.T_tot - t0) : C;
+    unsigned char *const rec = ws + (static_cast<int64_t>(blk) * p.HV + hv) * REC_BYTES;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
+    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
+
+    if (tid == 0) {
+        sync::mbar_init(&sm.mbar, 1);
+        sm.failed = 0;
+        sync::fence_barrier_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.tmem_base, WY_TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+
+    // ---- step 1: raw q, k, v of the block into the operand tiles; raw q
+    // also straight into the record; squared norms of k and q -------------
+    // thread (tg, kg): rows 8 tg .. 8 tg + 7, columns 8 kg .. 8 kg + 7
+    {
+        const int tg = tid >> 4, kg = tid & 15, col = 8 * kg;
+        uint4 kr[8], qr[8], vr[8];
+        float kk[8], qq[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int j = 8 * tg + r;
+            const int64_t tok = t0 + (j < n ? j : 0);
+            kr[r] = __ldg(reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + col));
+            qr[r] = __ldg(reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + col));
+            vr[r] = __ldg(reinterpret_cast<const uint4 *>(v + tok * p.v_tok + hv * p.v_head + col));
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int j = 8 * tg + r;
+            if (j >= n)
+                kr[r] = qr[r] = vr[r] = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(j, col, K)) = kr[r];
+            *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(64 + j, col, K)) = qr[r];
+            *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[r];
+            float kf[8], qf[8];
+            unpack8(kr[r], kf);
+            unpack8(qr[r], qf);
+            kk[r] = 0.f;
+            qq[r] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                kk[r] = fmaf(kf[e], kf[e], kk[r]);
+                qq[r] = fmaf(qf[e], qf[e], qq[r]);
+            }
+        }
+        uint4 tr[8];
+        transpose8x8(kr, tr);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4 *>(sm.kt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
+        transpose8x8(vr, tr);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4 *>(sm.vt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
+        // sum the 16 column groups of each row (lanes differing in bits 0..3)
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1)
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                kk[r] += __shfl_xor_sync(0xffffffffu, kk[r], off);
+                qq[r] += __shfl_xor_sync(0xffffffffu, qq[r], off);
+            }
+        if (kg == 0) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                sm.kk[8 * tg + r] = kk[r];
+                sm.qq[8 * tg + r] = qq[r];
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t my_lane = tc::tmem_addr(tmem, warp * 32, 0);
+
+    // ---- per-row scalars: gates and norms (threads 0..63), segment of the
+    // row (threads 64..127) -------------------------------------------------
+    if (tid < C) {
+        const int j = tid;
+        float rk = 0.f, rq = 0.f, g = 0.f, be = 0.f;
+        if (j < n) {
+            const int64_t tok = t0 + j;
+            rk = L2NORM ? rsqrtf(sm.kk[j] + 1e-6f) : 1.f;
+            rq = (L2NORM ? rsqrtf(sm.qq[j] + 1e-6f) : 1.f) * p.scale;
+            const float a_t = gate_value(gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32), p.a_f32);
+            const float b_t = gate_value(gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32), p.b_f32);
+            const float x = a_t + __ldg(p.dt_bias + hv * p.dt_stride);
+            g = -expf(__ldg(p.A_log + hv * p.A_stride)) * (x > 20.f ? x : log1pf(expf(x)));
+            be = 1.f / (1.f + expf(-b_t));
+        }
+        sm.rk[j] = rk;
+        sm.rqs[j] = rq;
+        sm.g[j] = g;
+        sm.beta[j] = be;
+    } else {
+        const int j = tid - C;
+        int ss = j, se = j + 1;      // rows past the end: a segment of their own
+        if (j < n) {
+            const int64_t tok = t0 + j;
+            int64_t s_beg, s_end;
+            if (p.cu_seqlens) {
+                // the last sequence starting at or before tok (binary search
+                // over cu_seqlens[0..N]; kept in bounds even if it is invalid)
+                int lo = 0, hi = p.N;            // cu[lo] <= tok < cu[hi] when valid
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (__ldg(p.cu_seqlens + mid) <= tok)
+                        lo = mid;
+                    else
+                        hi = mid;
+                }
+                s_beg = __ldg(p.cu_seqlens + lo);
+                s_end = __ldg(p.cu_seqlens + lo + 1);
+            } else {
+                const int64_t s = tok / p.T_fixed;
+                s_beg = s * p.T_fixed;
+                s_end = s_beg + p.T_fixed;
+            }
+            if (s_beg <= tok && tok < s_end) {
+                ss = static_cast<int>((s_beg > t0 ? s_beg : t0) - t0);
+                se = static_cast<int>((s_end < t0 + n ? s_end : t0 + n) - t0);
+            }
+        }
+        sm.ss[j] = ss;
+        sm.se[j] = se;
+    }
+    __syncthreads();
+    if (tid < C) {
+        // gamma_j: running sum of g over the row's segment
+        const int j = tid;
+        float acc = 0.f;
+        for (int i = sm.ss[j]; i <= j; ++i)
+            acc += sm.g[i];
+        sm.gam[j] = acc;
+    }
+    __syncthreads();
+    if (tid < C) {
+        const int j = tid;
+        const float gj = sm.gam[j], gl = sm.gam[sm.se[j] - 1];
+        sm.fa[j] = sm.beta[j] * sm.rk[j];
+        sm.fw[j] = sm.beta[j] * expf(gj) * sm.rk[j];
+        sm.fo[j] = expf(gj) * sm.rqs[j];
+        sm.fd[j] = expf(gl - gj) * sm.rk[j];
+        reinterpret_cast<float *>(rec + REC_FO)[j] = sm.fo[j];
+        reinterpret_cast<float *>(rec + REC_GAM)[j] = gj;
+    }
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+
+    uint32_t phase = 0;
+    bool ok = true;
+    auto wait_mma = [&]() {
+        bool w = ok && sync::mbar_wait(&sm.mbar, phase, &sm.failed);
+        phase ^= 1u;
+        if (!w && ok) {
+            sm.failed = 1;
+            report(p.status, GDN_DEV_TIMEOUT);
+        }
+        ok = __syncthreads_and(w) != 0;
+        tc::fence_after_sync();
+    };
+    auto publish_smem = [&]() {
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    const uint32_t ID_M128_N64 = tc::idesc_bf16_f32(128, 64);
+
+    // ---- step 2: [K;Q] K^T ---------------------------------------------------
+    if (tid == 0) {
+        mma_tiles(tmem + WY_COL_KQ, sm.kq, K, sm.kq, K, K / 16, ID_M128_N64, false);
+        tc::mma_commit(&sm.mbar);
+    }
+    wait_mma();
+
+    float *Amat = reinterpret_cast<float *>(sm.kq);              // [64][64] fp32, swizzled
+    float *Tmat = reinterpret_cast<float *>(sm.kq + 64 * 64 * 4);
+    if (ok) {
+        // ---- step 3: A (rows 0..63, smem) and P (rows 64..127, to the record)
+        float row[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16)
+            tc::tmem_ld16(my_lane + WY_COL_KQ + c, row + c);
+        tc::tmem_wait_ld();
+        if (tid < 64) {
+            const int j = tid, sj = sm.ss[j];
+            const float fj = sm.fa[j], gj = sm.gam[j];
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                Amat[sw64(j, c)] = (c < j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
+        } else {
+            const int j = tid - 64, sj = sm.ss[j];
+            const float fj = sm.rqs[j], gj = sm.gam[j];
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                row[c] = (c <= j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+                st_row8(rec + REC_P_HI, j, c, C, row + c, false);
+                st_row8(rec + REC_P_LO, j, c, C, row + c, true);
+            }
+        }
+        __syncthreads();
+
+        // ---- step 4: T = (I + A)^-1, blocked by 16 x 16 (as in the
+        // single-kernel schedule) ------------------------------------------
+        float *X = reinterpret_cast<float *>(sm.tw[0]);   // scratch [3][16][16]
+        if (tid < 64) {
+            const int I = tid >> 4, cc = tid & 15, c = 16 * I + cc;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m)
+                    acc = fmaf(-Amat[sw64(16 * I + r, 16 * I + m)], x[m], acc);
+                x[r] = (r < cc) ? 0.f : acc;
+                Tmat[sw64(16 * I + r, c)] = x[r];
+            }
+        } else {
+            for (int e = tid - 64; e < 6 * 256; e += 64) {
+                const int b6 = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int I = b6 < 3 ? 0 : (b6 < 5 ? 1 : 2);
+                const int J = b6 < 3 ? b6 + 1 : (b6 < 5 ? b6 - 1 : 3);
+                Tmat[sw64(16 * I + r, 16 * J + cc)] = 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {
+            const int nb = 4 - d;
+            for (int e = tid; e < nb * 256; e += THREADS) {
+                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
+                float acc = 0.f;
+                for (int M = J; M < I; ++M)
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        acc = fmaf(Amat[sw64(16 * I + r, 16 * M + m)], Tmat[sw64(16 * M + m, 16 * J + cc)], acc);
+                X[e] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nb * 256; e += THREADS) {
+                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Tmat[sw64(16 * I + r, 16 * I + m)], X[(J << 8) + (m << 4) + cc], acc);
+                Tmat[sw64(16 * I + r, 16 * J + cc)] = -acc;
+            }
+            __syncthreads();
+        }
+        // T diag(fw) and T diag(beta) as hi / lo operand tiles
+        {
+            const int r = tid >> 1, cbase = 32 * (tid & 1);
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                float tw8[8], tu8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int col = cbase + c + e;
+                    const float t = Tmat[sw64(r, col)];
+                    tw8[e] = t * sm.fw[col];
+                    tu8[e] = t * sm.beta[col];
+                }
+                st_row8(sm.tw[0], r, cbase + c, C, tw8, false);
+                st_row8(sm.tw[1], r, cbase + c, C, tw8, true);
+                st_row8(sm.tu[0], r, cbase + c, C, tu8, false);
+                st_row8(sm.tu[1], r, cbase + c, C, tu8, true);
+            }
+        }
+        publish_smem();
+
+        // ---- step 5: W^T = K^T T_w^T and U^T = V^T T_u^T ----------------
+        if (tid == 0) {
+            mma_tiles(tmem + WY_COL_WT, sm.kt, C, sm.tw[0], C, C / 16, ID_M128_N64, false);
+            mma_tiles(tmem + WY_COL_WT, sm.kt, C, sm.tw[1], C, C / 16, ID_M128_N64, true);
+            mma_tiles(tmem + WY_COL_UT, sm.vt, C, sm.tu[0], C, C / 16, ID_M128_N64, false);
+            mma_tiles(tmem + WY_COL_UT, sm.vt, C, sm.tu[1], C, C / 16, ID_M128_N64, true);
+            tc::mma_commit(&sm.mbar);
+        }
+        wait_mma();
+    }
+    if (ok) {
+        // ---- step 6: the record's remaining tiles -------------------------
+        // W (thread = k): hi / lo tiles [i][k] staged in the kq area (A and T
+        // are dead), then one bulk store of both
+        unsigned char *w_hi = sm.kq, *w_lo = sm.kq + 64 * 128 * 2;
+        {
+            float wcol[64];
+#pragma unroll
+            for (int c = 0; c < 64; c += 16)
+                tc::tmem_ld16(my_lane + WY_COL_WT + c, wcol + c);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                __nv_bfloat16 hi, lo;
+                split2(wcol[j], hi, lo);
+                st_bf16(w_hi, j, tid, K, hi);
+                st_bf16(w_lo, j, tid, K, lo);
+            }
+        }
+        // U^T (thread = v): one fp32 row of 64
+        {
+            float4 *dst = reinterpret_cast<float4 *>(rec + REC_UT) + tid * 16;
+#pragma unroll
+            for (int c = 0; c < 64; c += 16) {
+                float u[16];
+                tc::tmem_ld16(my_lane + WY_COL_UT + c, u);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    dst[(c + e) / 4] = make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
+            }
+        }
+        // K'^T = (diag(fd) K)^T (thread = k): raw k^T row scaled, hi / lo
+        {
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm.kt + tc::kmajor_offset(tid, c, C)), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    x[e] *= sm.fd[c + e];
+                st_row8(rec + REC_KP_HI, tid, c, C, x, false);
+                st_row8(rec + REC_KP_LO, tid, c, C, x, true);
+            }
+        }
+        sync::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            sync::bulk_store(rec + REC_W_HI, sm.kq, 2 * 64 * 128 * 2);
+            sync::bulk_commit();
+            sync::bulk_wait_all();
+        }
+    }
+
+    pdl_trigger();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, WY_TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: the recurrence through the state of one (sequence, value head).
+// ---------------------------------------------------------------------------
+struct StSmem {
+    alignas(1024) unsigned char st[2][128 * 128 * 2];   // S~^T hi / lo [v][k]
+    alignas(1024) unsigned char rec_a[REC_A_BYTES];     // W hi, W lo, Q of the piece (record bytes 0 .. 49151)
+    alignas(1024) unsigned char rec_b[REC_B_BYTES];     // K'^T hi / lo, P hi / lo (record bytes 49152 .. 98303)
+    alignas(1024) unsigned char dt[2][128 * 64 * 2];    // Delta~^T hi / lo [v][i]
+    alignas(16) float rec_s[REC_S_BYTES / 4];           // fo, gamma of the piece (record tail)
+    float fo[C];                                        // fo of the piece being finished
+    unsigned long long bar_mma, bar_a, bar_b;
+    uint32_t tmem_base;
+    int failed;
+};
+
+constexpr uint32_t ST_TMEM_COLS = 512;
+constexpr uint32_t ST_COL_S = 0;      // S~^T          [v][k]   128 columns
+constexpr uint32_t ST_COL_D = 128;    // -S~^T W^T     [v][i]    64
+constexpr uint32_t ST_COL_O1 = 192;   // S~^T Q^T      [v][j]    64
+constexpr uint32_t ST_COL_O2 = 256;   // Delta~^T P^T  [v][j]    64
+
+// The state is kept as S = cs * S~ for a per-CTA scale cs, so a piece's
+// decay e^gamma_last multiplies cs instead of the 16 K state elements in
+// TMEM: with cs' = cs e^gamma_last the update is S~ += Delta~^T K'^T where
+// Delta~ = Delta / cs'.  When cs' leaves [2^-60, 2^60] the TMEM state is
+// rescaled once (S~ <- cs' S~) and cs returns to 1.
+__global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __grid_constant__ DecodeParams p,
+                                                                    const unsigned char *__restrict__ ws)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    StSmem &sm = *reinterpret_cast<StSmem *>(smem_raw);
+
+    pdl_prologue();
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int i = blockIdx.x / p.HV;
+    const int hv = blockIdx.x - i * p.HV;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+
+    // ---- token range and slot (uniform over the CTA) -----------------
+    int64_t bos;
+    int len;
+    if (p.cu_seqlens) {
+        const int b0 = __ldg(p.cu_seqlens + i);
+        const int e0 = __ldg(p.cu_seqlens + i + 1);
+        if (b0 < 0 || e0 < b0 || e0 > p.T_tot) {
+            if (tid == 0 && hv == 0)
+                report(p.status, GDN_DEV_BAD_SEQLENS);
+            return;
+        }
+        bos = b0;
+        len = e0 - b0;
+    } else {
+        bos = static_cast<int64_t>(i) * p.T_fixed;
+        len = p.T_fixed;
+    }
+    const int slot = __ldg(p.indices + i);
+    if (slot < -1 || slot >= p.num_slots) {
+        if (tid == 0 && hv == 0)
+            report(p.status, GDN_DEV_BAD_SLOT);
+        return;
+    }
+    if (slot < 0) {
+        for (int t = 0; t < len; ++t)
+            out[(bos + t) * p.o_tok + hv * p.o_head + tid] = __float2bfloat16_rn(0.f);
+        return;
+    }
+    if (len == 0)
+        return;
+    const int64_t eos = bos + len;
+    float *const s_gmem = p.state + static_cast<int64_t>(slot) * p.s_slot + hv * p.s_head;
+    auto rec_of = [&](int64_t b) { return ws + (b * p.HV + hv) * static_cast<int64_t>(REC_BYTES); };
+
+    // ---- set-up: barriers, TMEM, the first piece's tiles in flight, the
+    // state into TMEM and into the S~^T tiles (cs = 1) ----------------------
+    int64_t blk = bos / C;
+    if (tid == 0) {
+        sync::mbar_init(&sm.bar_mma, 1);
+        sync::mbar_init(&sm.bar_a, 1);
+        sync::mbar_init(&sm.bar_b, 1);
+        sm.failed = 0;
+        sync::fence_barrier_init();
+        const unsigned char *r = rec_of(blk);
+        sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
+        sync::bulk_load(sm.rec_a, r, REC_A_BYTES, &sm.bar_a);
+        sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES + REC_S_BYTES);
+        sync::bulk_load(sm.rec_b, r + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
+        sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_b);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.tmem_base, ST_TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t my_lane = tc::tmem_addr(tmem, warp * 32, 0);
+
+    for (int k0 = 0; k0 < K; k0 += 16) {       // thread t = v: column v of S -> lane v of S~^T
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            x[e] = __ldcs(s_gmem + (k0 + e) * V + tid);
+        tc::tmem_st16(my_lane + ST_COL_S + k0, x);
+        st_row8(sm.st[0], tid, k0, K, x, false);
+        st_row8(sm.st[0], tid, k0 + 8, K, x + 8, false);
+        st_row8(sm.st[1], tid, k0, K, x, true);
+        st_row8(sm.st[1], tid, k0 + 8, K, x + 8, true);
+    }
+    tc::tmem_wait_st();
+
+    uint32_t ph_mma = 0, ph_a = 0, ph_b = 0;
+    // copies issued and not yet waited for, with the parity their wait checks
+    bool ok = true, pend_a = true, pend_b = true;
+    uint32_t pa = 0, pb = 0;
+    // bounded wait on one of the barriers; uniform verdict over the CTA
+    auto wait_bar = [&](unsigned long long *bar, uint32_t &ph) {
+        bool w = ok && sync::mbar_wait(bar, ph, &sm.failed);
+        ph ^= 1u;
+        if (!w && ok) {
+            sm.failed = 1;
+            report(p.status, GDN_DEV_TIMEOUT);
+        }
+        ok = __syncthreads_and(w) != 0;
+        tc::fence_after_sync();
+    };
+    auto publish_smem = [&]() {
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    publish_smem();
+
+    const uint32_t ID_N64 = tc::idesc_bf16_f32(128, 64);
+    const uint32_t ID_N64_NEG = tc::idesc_bf16_f32(128, 64, true);
+    const uint32_t ID_N128 = tc::idesc_bf16_f32(128, 128);
+    const unsigned char *w_hi = sm.rec_a + REC_W_HI, *w_lo = sm.rec_a + REC_W_LO, *q_t = sm.rec_a + REC_Q;
+    const unsigned char *kp_hi = sm.rec_b + (REC_KP_HI - REC_KP_HI), *kp_lo = sm.rec_b + (REC_KP_LO - REC_KP_HI);
+    const unsigned char *p_hi = sm.rec_b + (REC_P_HI - REC_KP_HI), *p_lo = sm.rec_b + (REC_P_LO - REC_KP_HI);
+
+    float cs = 1.f;
+    for (int64_t t = bos; t < eos && ok; ++blk) {
+        const int64_t base = blk * C;
+        const int r0 = static_cast<int>(t - base);
+        const int r1 = static_cast<int>((eos < base + C ? eos : base + C) - base);
+        const bool more = base + r1 < eos;
+        const unsigned char *rec = rec_of(blk);
+
+        // this thread's row of U^T (needed after the first product)
+        float u[64];
+        {
+            const float4 *src = reinterpret_cast<const float4 *>(rec + REC_UT) + tid * 16;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float4 x = __ldg(src + m);
+                u[4 * m] = x.x;
+                u[4 * m + 1] = x.y;
+                u[4 * m + 2] = x.z;
+                u[4 * m + 3] = x.w;
+            }
+        }
+
+        // ---- product 1: -S~^T W^T (3 split products) and S~^T Q^T (2) ----
+        wait_bar(&sm.bar_a, ph_a);
+        if (!ok)
+            break;
+        pend_a = false;
+        if (tid == 0) {
+            mma_tiles(tmem + ST_COL_D, sm.st[0], K, w_hi, K, K / 16, ID_N64_NEG, false);
+            mma_tiles(tmem + ST_COL_D, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
+            mma_tiles(tmem + ST_COL_D, sm.st[1], K, w_hi, K, K / 16, ID_N64_NEG, true);
+            mma_tiles(tmem + ST_COL_O1, sm.st[0], K, q_t, K, K / 16, ID_N64, false);
+            mma_tiles(tmem + ST_COL_O1, sm.st[1], K, q_t, K, K / 16, ID_N64, true);
+            tc::mma_commit(&sm.bar_mma);
+        }
+        wait_bar(&sm.bar_mma, ph_mma);
+        if (!ok)
+            break;
+        if (more && tid == 0) {       // W and Q of the next piece, into the buffer just read
+            sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
+            sync::bulk_load(sm.rec_a, rec_of(blk + 1), REC_A_BYTES, &sm.bar_a);
+        }
+        pend_a = more;
+        pa = ph_a;
+
+        // ---- Delta~^T (thread = v) into its hi / lo tiles -----------------
+        wait_bar(&sm.bar_b, ph_b);
+        if (!ok)
+            break;
+        pend_b = false;
+        const float decay = expf(sm.rec_s[C + r1 - 1]);    // e^gamma at the piece's last row
+        const float cn = cs * decay;
+        const bool rescale = !(cn >= 0x1p-60f && cn <= 0x1p60f);
+        const float dscale = rescale ? 1.f : __fdividef(1.f, cn);
+        if (tid < C)
+            sm.fo[tid] = sm.rec_s[tid];
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+            float d[16];
+            tc::tmem_ld16(my_lane + ST_COL_D + cb, d);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int ii = cb + e;
+                d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[ii]) * dscale : 0.f;
+            }
+            st_row8(sm.dt[0], tid, cb, C, d, false);
+            st_row8(sm.dt[0], tid, cb + 8, C, d + 8, false);
+            st_row8(sm.dt[1], tid, cb, C, d, true);
+            st_row8(sm.dt[1], tid, cb + 8, C, d + 8, true);
+        }
+        if (rescale) {               // S~ <- cs' S~ in TMEM; the scale returns to 1
+#pragma unroll 1
+            for (int k0 = 0; k0 < K; k0 += 16) {
+                float x[16];
+                tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] *= cn;
+                tc::tmem_st16(my_lane + ST_COL_S + k0, x);
+            }
+            tc::tmem_wait_st();
+        }
+        const float cs_new = rescale ? 1.f : cn;
+        publish_smem();
+
+        // ---- product 2: Delta~^T P^T (3) and S~^T += Delta~^T K'^T (3) -----
+        if (tid == 0) {
+            mma_tiles(tmem + ST_COL_O2, sm.dt[0], C, p_hi, C, C / 16, ID_N64, false);
+            mma_tiles(tmem + ST_COL_O2, sm.dt[0], C, p_lo, C, C / 16, ID_N64, true);
+            mma_tiles(tmem + ST_COL_O2, sm.dt[1], C, p_hi, C, C / 16, ID_N64, true);
+            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kp_hi, C, C / 16, ID_N128, true);
+            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kp_lo, C, C / 16, ID_N128, true);
+            mma_tiles(tmem + ST_COL_S, sm.dt[1], C, kp_hi, C, C / 16, ID_N128, true);
+            tc::mma_commit(&sm.bar_mma);
+        }
+        wait_bar(&sm.bar_mma, ph_mma);
+        if (!ok)
+            break;
+        if (more && tid == 0) {       // K', P, fo, gamma of the next piece
+            const unsigned char *r = rec_of(blk + 1);
+            sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES + REC_S_BYTES);
+            sync::bulk_load(sm.rec_b, r + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
+            sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_b);
+        }
+        pend_b = more;
+        pb = ph_b;
+
+        // ---- outputs o_j = fo_j cs (S~0^T q_j) + cs' (Delta~^T P^T)_j --------
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+            float o1[16], o2[16];
+            tc::tmem_ld16(my_lane + ST_COL_O1 + cb, o1);
+            tc::tmem_ld16(my_lane + ST_COL_O2 + cb, o2);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = cb + e;
+                if (j >= r0 && j < r1)
+                    out[(base + j) * p.o_tok + hv * p.o_head + tid] =
+                        __float2bfloat16_rn(fmaf(sm.fo[j] * cs, o1[e], cs_new * o2[e]));
+            }
+        }
+
+        // ---- the next piece's S~^T tiles, or the final write-back -----------
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            float x[16];
+            tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
+            tc::tmem_wait_ld();
+            if (more) {
+                st_row8(sm.st[0], tid, k0, K, x, false);
+                st_row8(sm.st[0], tid, k0 + 8, K, x + 8, false);
+                st_row8(sm.st[1], tid, k0, K, x, true);
+                st_row8(sm.st[1], tid, k0 + 8, K, x + 8, true);
+            } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    __stcs(s_gmem + (k0 + e) * V + tid, cs_new * x[e]);
+            }
+        }
+        cs = cs_new;
+        t = base + r1;
+        publish_smem();
+    }
+
+    // a failed wait left copies in flight: let them land (bounded) before the
+    // shared memory is released
+    if (pend_a || pend_b) {
+        volatile int never = 0;
+        if (pend_a)
+            sync::mbar_wait(&sm.bar_a, pa, &never);
+        if (pend_b)
+            sync::mbar_wait(&sm.bar_b, pb, &never);
+    }
+
+    pdl_trigger();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, ST_TMEM_COLS);
+}
+
+}  // namespace split
+}  // namespace gdn

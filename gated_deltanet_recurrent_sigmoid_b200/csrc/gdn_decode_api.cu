@@ -15,6 +15,7 @@
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
 #include "gdn_chunk_kernel.cuh"
+#include "gdn_chunk_split.cuh"
 #include "gdn_decode_pipelined.cuh"
 
 namespace {
@@ -186,9 +187,9 @@ int check_indices_on_host(const int32_t *d_idx, const int32_t *d_cu, int64_t N, 
 }
 
 // Launch with or without the programmatic-stream-serialization attribute.
-template <typename Kernel>
+template <typename Kernel, typename... Args>
 cudaError_t launch_ex(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
-                      const gdn::DecodeParams &p)
+                      const Args &...args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -200,7 +201,7 @@ cudaError_t launch_ex(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, p);
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 template <int BV, int KG, typename TAct, bool GIVEN>
@@ -233,6 +234,44 @@ cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream
     }
     return launch_ex(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
                      dim3(static_cast<unsigned>(units)), dim3(gdn::chunk::THREADS), smem, stream, pdl, p);
+}
+
+// Split chunked schedule: the block kernel over ceil(T_tot / 64) x HV CTAs,
+// then the state kernel over the (sequence, value head) pairs.  The state
+// kernel always uses programmatic dependent launch behind the block kernel
+// (it waits for the block kernel's completion before reading anything).
+cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t units, cudaStream_t stream,
+                         bool pdl, bool l2norm)
+{
+    static bool ready[64];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    const size_t smem_wy = sizeof(gdn::split::WySmem), smem_st = sizeof(gdn::split::StSmem);
+    if (!ready[dev]) {
+        err = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem_wy));
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_wy));
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_st));
+        if (err != cudaSuccess)
+            return err;
+        ready[dev] = true;
+    }
+    const int64_t blocks = (static_cast<int64_t>(p.T_tot) + gdn::split::C - 1) / gdn::split::C * p.HV;
+    err = launch_ex(l2norm ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
+                    dim3(static_cast<unsigned>(blocks)), dim3(gdn::split::THREADS), smem_wy, stream, pdl, p, ws);
+    if (err != cudaSuccess)
+        return err;
+    return launch_ex(gdn::split::gdn_chunk_state_kernel, dim3(static_cast<unsigned>(units)),
+                     dim3(gdn::split::THREADS), smem_st, stream, true, p,
+                     static_cast<const unsigned char *>(ws));
 }
 
 // The tile table: (V-tile width, rows per thread) -> (BV, KG = K / rows).
@@ -312,7 +351,7 @@ int run_update(const UpdateArgs &c)
         return GDN_ERR_ARG;
     int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
     if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED &&
-        schedule != GDN_SCHEDULE_CHUNKED)
+        schedule != GDN_SCHEDULE_CHUNKED && schedule != GDN_SCHEDULE_CHUNKED_SPLIT)
         return GDN_ERR_ARG;
     if (extra && extra->reserved != 0)
         return GDN_ERR_ARG;
@@ -451,6 +490,35 @@ int run_update(const UpdateArgs &c)
         }
     }
 
+    // ---- the caller's workspace (used by the split chunked schedule only):
+    // a given workspace must be aligned and overlap no tensor of the call
+    void *const ws = extra ? extra->workspace : nullptr;
+    const uint64_t ws_bytes = extra ? extra->workspace_bytes : 0;
+    if (ws) {
+        if (!aligned(ws, 256))
+            return GDN_ERR_ALIGN;
+        Span sw;
+        sw.lo = reinterpret_cast<uintptr_t>(ws);
+        sw.hi = sw.lo + static_cast<uintptr_t>(ws_bytes);
+        const gdn_tensor *all[] = {q, k, v, ga, gb, c.given_gates ? nullptr : A_log, c.given_gates ? nullptr : dt_bias,
+                                   state_indices, cu_seqlens, out, state_pool, want_inter ? inter : nullptr};
+        for (const gdn_tensor *t : all)
+            if (t && overlap(sw, span_of(t)))
+                return GDN_ERR_ALIAS;
+        if (extra->device_status) {
+            Span st;
+            st.lo = reinterpret_cast<uintptr_t>(extra->device_status);
+            st.hi = st.lo + sizeof(uint32_t);
+            if (overlap(sw, st))
+                return GDN_ERR_ALIAS;
+        }
+    }
+    const bool ws_fits = ws && ws_bytes >= gdn::split::workspace_bytes(T_tot, HV);
+    if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT && !ws)
+        return GDN_ERR_NULL_ARG;
+    if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT && !ws_fits)
+        return GDN_ERR_ARG;
+
     // ---- supported configurations and the library's choices
     if (K != kHeadK || V != kHeadV)
         return GDN_ERR_UNSUPPORTED;
@@ -498,17 +566,18 @@ int run_update(const UpdateArgs &c)
     if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
         act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0 &&
         T_tot >= (N * HV <= kChunkedFewPairs ? kChunkedMinMeanTokensFew : kChunkedMinMeanTokensMany) * N)
-        schedule = GDN_SCHEDULE_CHUNKED;
+        schedule = ws_fits ? GDN_SCHEDULE_CHUNKED_SPLIT : GDN_SCHEDULE_CHUNKED;
     // The pipelined schedule is built for bf16 activations and fused bf16
     // gates; the chunked one for bf16 activations, fused gates and no
     // per-token states.
     if (schedule == GDN_SCHEDULE_PIPELINED &&
         (act != GDN_DTYPE_BF16 || c.given_gates || ga->dtype != GDN_DTYPE_BF16 || gb->dtype != GDN_DTYPE_BF16))
         return GDN_ERR_UNSUPPORTED;
-    if (schedule == GDN_SCHEDULE_CHUNKED && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
+    const bool chunked = schedule == GDN_SCHEDULE_CHUNKED || schedule == GDN_SCHEDULE_CHUNKED_SPLIT;
+    if (chunked && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
         return GDN_ERR_UNSUPPORTED;
-    // the chunked kernel reads v rows 16 bytes at a time, like q and k
-    if (schedule == GDN_SCHEDULE_CHUNKED && !v_rows_16b)
+    // the chunked kernels read v rows 16 bytes at a time, like q and k
+    if (chunked && !v_rows_16b)
         return GDN_ERR_ALIGN;
     const int64_t units = N * HV;
     if (units * (kHeadV / tile_v) > INT32_MAX)
@@ -574,6 +643,8 @@ int run_update(const UpdateArgs &c)
         err = launch_pipelined(p, units, stream, pdl);
     else if (schedule == GDN_SCHEDULE_CHUNKED)
         err = launch_chunked(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
+    else if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT)
+        err = launch_split(p, static_cast<unsigned char *>(ws), units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (act == GDN_DTYPE_BF16)
         err = c.given_gates ? launch_tile<__nv_bfloat16, true>(p, units, stream, pdl, tile_v, tile_rows)
                             : launch_tile<__nv_bfloat16, false>(p, units, stream, pdl, tile_v, tile_rows);
@@ -588,6 +659,13 @@ int run_update(const UpdateArgs &c)
 extern "C" {
 
 GDN_API int gdn_version(void) { return GDN_DECODE_ABI_VERSION; }
+
+GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV)
+{
+    if (T_tot <= 0 || HV <= 0)
+        return 0;
+    return gdn::split::workspace_bytes(T_tot, HV);
+}
 
 GDN_API const char *gdn_status_string(int status)
 {

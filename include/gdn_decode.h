@@ -81,7 +81,7 @@
 extern "C" {
 #endif
 
-#define GDN_DECODE_ABI_VERSION 1
+#define GDN_DECODE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -146,6 +146,17 @@ extern "C" {
                                     on the tcgen05 tensor cores (prefill-style);
                                     bf16 activations, gates from A_log/a/b/dt_bias,
                                     no GDN_WRITE_INTERMEDIATE; v aligned like q */
+#define GDN_SCHEDULE_CHUNKED_SPLIT 4 /* the same chunked algorithm as two kernels:
+                                    the products that do not depend on the state
+                                    (decay scan, A, T = (I + A)^-1, W, U, the
+                                    masked q.k matrix) for every 64-token block
+                                    of the packed token range at once, written to
+                                    the caller's workspace; then the recurrence
+                                    through the state, one CTA per (sequence,
+                                    value head).  Same restrictions as
+                                    GDN_SCHEDULE_CHUNKED, plus a workspace of
+                                    gdn_chunked_workspace_bytes(T_tot, HV) bytes
+                                    in gdn_extra */
 
 /* bits OR-ed into *device_status by the kernel */
 #define GDN_DEV_BAD_SLOT    1u
@@ -171,6 +182,12 @@ typedef struct gdn_extra {
                                               (16 or 32; 0 = library choice) */
     int32_t schedule;                      /* GDN_SCHEDULE_* (0 = library choice) */
     int32_t reserved;                      /* must be 0 */
+    void *workspace;                       /* device scratch for GDN_SCHEDULE_CHUNKED_SPLIT
+                                              (256-byte aligned, owned by the caller,
+                                              overlapping no tensor of the call; its
+                                              contents need no initialisation and are
+                                              garbage afterwards), or NULL */
+    uint64_t workspace_bytes;              /* its size in bytes */
 } gdn_extra;
 
 /*
@@ -228,6 +245,14 @@ GDN_API const char *gdn_status_string(int status);
 
 /* GDN_DECODE_ABI_VERSION of the loaded library. */
 GDN_API int gdn_version(void);
+
+/*
+ * Bytes of workspace GDN_SCHEDULE_CHUNKED_SPLIT needs for a call with T_tot
+ * tokens and HV value heads (K = V = 128): one 131,584-byte record per
+ * (64-token block of the packed token range, value head).  0 for T_tot <= 0
+ * or HV <= 0.  Host-only arithmetic, no CUDA call.
+ */
+GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV);
 
 #ifdef __cplusplus
 }

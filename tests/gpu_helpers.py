@@ -35,7 +35,7 @@ def to_device(w: Workload, device="cuda") -> dict:
 
 
 def run_gpu(w: Workload, flags=binding.L2NORM_QK, inter=False, tile_v=0, d=None, scale=None,
-            schedule=binding.SCHEDULE_AUTO, tile_rows=0):
+            schedule=binding.SCHEDULE_AUTO, tile_rows=0, workspace="auto"):
     """Run the CUDA path once; returns (device dict, status word, inter tensor)."""
     d = d or to_device(w)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -45,7 +45,7 @@ def run_gpu(w: Workload, flags=binding.L2NORM_QK, inter=False, tile_v=0, d=None,
     binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"],
                           d["state_indices"], d["cu_seqlens"], d["out"], scale=scale, flags=flags,
                           intermediate_states=inter_t, device_status=status, tile_v=tile_v, schedule=schedule,
-                          tile_rows=tile_rows)
+                          tile_rows=tile_rows, workspace=workspace)
     torch.cuda.synchronize()
     return d, int(status.item()), inter_t
 

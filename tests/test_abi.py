@@ -24,7 +24,7 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     assert set(declared_functions()) == {"gdn_decode_update", "gdn_recurrent_update", "gdn_gating",
-                                         "gdn_status_string", "gdn_version"}
+                                         "gdn_status_string", "gdn_version", "gdn_chunked_workspace_bytes"}
 
 
 def test_library_exports_every_declared_symbol(gdn_lib):
@@ -60,12 +60,14 @@ def test_header_constants_match_binding():
     assert define("GDN_NO_FINAL_WRITEBACK") == binding.NO_FINAL_WRITEBACK
     assert define("GDN_CHECK_INDICES") == binding.CHECK_INDICES
     assert define("GDN_LAUNCH_PDL") == binding.LAUNCH_PDL
+    for name in ("AUTO", "PER_TILE", "PIPELINED", "CHUNKED", "CHUNKED_SPLIT"):
+        assert define(f"GDN_SCHEDULE_{name}") == getattr(binding, f"SCHEDULE_{name}")
     for name, val in [("GDN_ERR_NULL_ARG", -1), ("GDN_ERR_DTYPE", -2), ("GDN_ERR_SHAPE", -3),
                       ("GDN_ERR_ALIGN", -4), ("GDN_ERR_ALIAS", -5), ("GDN_ERR_UNSUPPORTED", -6),
                       ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9)]:
         assert int(re.search(rf"#define {name}\s+\((-?\d+)\)", text).group(1)) == val
     assert ctypes.sizeof(binding.GdnTensor) == 8 + 4 + 4 + 8 * 4 + 8 * 4
-    assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 * 4
+    assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 * 4 + 8 + 8
 
 
 def make(N=4, T=1, H=2, HV=4, K=128, V=128, slots=8, varlen=True):
@@ -155,3 +157,34 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(build, "LIB_PATH", "/nonexistent/libgdn_decode.so")
     with pytest.raises(binding.GdnError):
         binding.load()
+
+
+def test_chunked_workspace_bytes(gdn_lib):
+    """One 131,584-byte record per (64-token block, value head); host-only."""
+    rec = 131584
+    assert binding.chunked_workspace_bytes(0, 8) == 0
+    assert binding.chunked_workspace_bytes(5, 0) == 0
+    assert binding.chunked_workspace_bytes(1, 1) == rec
+    assert binding.chunked_workspace_bytes(64, 8) == 8 * rec
+    assert binding.chunked_workspace_bytes(65, 8) == 16 * rec
+    assert binding.chunked_workspace_bytes(13488, 8) == 211 * 8 * rec
+    assert rec % 256 == 0
+
+
+def test_split_schedule_checks_its_workspace(gdn_lib):
+    """GDN_SCHEDULE_CHUNKED_SPLIT needs a workspace: missing, too small,
+    misaligned or overlapping a tensor of the call is rejected before any
+    launch; AUTO ignores one that is too small."""
+    split = binding.SCHEDULE_CHUNKED_SPLIT
+    t = make(N=2, T=3)
+    need = binding.chunked_workspace_bytes(6, 4)
+    expect(binding.ERR_NULL_ARG, t, schedule=split, workspace=None)
+    raw = torch.empty(need + 512, dtype=torch.uint8)
+    off = (-raw.data_ptr()) % 256                                       # 256-byte aligned view
+    expect(binding.ERR_ARG, t, schedule=split, workspace=raw[off:off + need - 256])
+    expect(binding.ERR_ALIGN, t, schedule=split, workspace=raw[off + 16:off + 16 + need])
+    t2 = make(N=2, T=3)
+    raw = torch.zeros(need // 4 + t2["state_pool"].numel() + 64, dtype=torch.float32)
+    big = raw[((-raw.data_ptr()) % 256) // 4:]                                         # 256-byte aligned
+    t2["state_pool"] = big[: t2["state_pool"].numel()].view(t2["state_pool"].shape)   # workspace overlaps the pool
+    expect(binding.ERR_ALIAS, t2, schedule=split, workspace=big.view(torch.uint8)[:need])

@@ -18,7 +18,15 @@ from helpers import random_problem
 pytestmark = pytest.mark.gpu
 
 CHUNKED = binding.SCHEDULE_CHUNKED
+SPLIT = binding.SCHEDULE_CHUNKED_SPLIT
 L2 = binding.L2NORM_QK
+
+
+@pytest.fixture(params=[CHUNKED, SPLIT], ids=["single", "split"])
+def sched(request):
+    """Both chunked schedules: one kernel, or the block kernel + state kernel
+    around a workspace."""
+    return request.param
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -27,8 +35,8 @@ def _lib(gdn_lib):
     return gdn_lib
 
 
-def check(w, flags=L2, scale=None):
-    d, status, _ = run_gpu(w, flags=flags, schedule=CHUNKED, scale=scale)
+def check(w, sched, flags=L2, scale=None):
+    d, status, _ = run_gpu(w, flags=flags, schedule=sched, scale=scale)
     ost, o_ref, s_ref, _ = run_oracle(w, flags=flags, scale=scale)
     assert status == ost
     assert_out_close(out_as_f32(d["out"]), o_ref)
@@ -54,39 +62,54 @@ def problem(lens, pad=(), H=4, HV=8, seed=0):
 
 @pytest.mark.parametrize("lens", [[1], [64], [65], [200, 7, 130], [3, 64, 128, 1, 300]],
                          ids=["1", "64", "65", "ragged3", "ragged5"])
-def test_chunked_matches_oracle(lens):
-    check(problem(lens, seed=len(lens)))
+def test_chunked_matches_oracle(lens, sched):
+    check(problem(lens, seed=len(lens)), sched)
 
 
-def test_chunked_padding_empty_and_gqa():
-    check(problem([70, 0, 33, 129], pad=(2,), H=2, HV=6, seed=9))
+def test_chunked_padding_empty_and_gqa(sched):
+    check(problem([70, 0, 33, 129], pad=(2,), H=2, HV=6, seed=9), sched)
 
 
-def test_chunked_l2norm_off_and_scale():
+def test_chunked_l2norm_off_and_scale(sched):
     w = problem([90, 40], seed=3)
     # L2 off: unit-length k keeps the state O(1)
     k = wl.bf16_bits_to_f32(w.k)
     w.k = wl.f32_to_bf16_bits(k / np.linalg.norm(k, axis=-1, keepdims=True))
-    check(w, flags=0)
-    check(problem([90, 40], seed=4), scale=0.2)
+    check(w, sched, flags=0)
+    check(problem([90, 40], seed=4), sched, scale=0.2)
 
 
-def test_chunked_no_final_writeback_and_fixed_layout():
-    check(problem([77, 12], seed=5), flags=L2 | binding.NO_FINAL_WRITEBACK)
-    check(wl.generate(wl.shrink(wl.SPEC_B128_T4, 16)))         # T = 4, one partial chunk each
-    check(wl.generate(wl.TINY))                                 # fixed [N, 1] layout
+def test_chunked_weak_and_mixed_decay(sched):
+    """exp(A_log) tiny: the decays stay near 1, so the state's scale never
+    leaves its range (no rescaling); mixed heads cover both cases in one
+    call."""
+    w = problem([150, 3, 70, 200], seed=12)
+    w.A_log = np.full_like(w.A_log, -9.0)
+    check(w, sched)
+    w = problem([150, 3, 70, 200], seed=13)
+    w.A_log = w.A_log.copy()
+    w.A_log[::2] = -9.0
+    check(w, sched)
+
+
+def test_chunked_no_final_writeback_and_fixed_layout(sched):
+    check(problem([77, 12], seed=5), sched, flags=L2 | binding.NO_FINAL_WRITEBACK)
+    check(wl.generate(wl.shrink(wl.SPEC_B128_T4, 16)), sched)  # T = 4, one partial chunk each
+    check(wl.generate(wl.TINY), sched)                          # fixed [N, 1] layout
+    fixed = wl.WorkloadSpec("fixed_t100", N=3, H=4, HV=8, num_slots=6, seed=14, T=100)
+    check(wl.generate(fixed), sched)                            # fixed [N, T] layout, blocks across sequences
 
 
 @pytest.mark.parametrize("spec", [wl.sweep_spec(8), wl.sweep_spec(64)], ids=lambda s: s.name)
-def test_chunked_full_size_sweeps(spec):
-    check(wl.generate(spec))
+def test_chunked_full_size_sweeps(spec, sched):
+    check(wl.generate(spec), sched)
 
 
-def test_chunked_prefill_b64_sampled():
+def test_chunked_prefill_b64_sampled(sched):
     """Full-size prefill-style batch in the benchmark's launch configuration;
     the oracle recomputes a sample of sequences."""
     w = wl.generate(wl.PREFILL_B64)
-    d, status, _ = run_gpu(w, schedule=CHUNKED)
+    d, status, _ = run_gpu(w, schedule=sched)
     assert status == 0
     rng = np.random.default_rng(0)
     seqs = np.sort(rng.choice(w.spec.N, size=6, replace=False))
@@ -99,30 +122,30 @@ def test_chunked_prefill_b64_sampled():
     assert_state_close(got, s_ref, "sampled state")
 
 
-def test_chunked_agrees_with_per_token_kernel():
+def test_chunked_agrees_with_per_token_kernel(sched):
     w = wl.generate(wl.shrink(wl.sweep_spec(64), 24))
-    a, _, _ = run_gpu(w, schedule=CHUNKED)
+    a, _, _ = run_gpu(w, schedule=sched)
     b, _, _ = run_gpu(w, schedule=binding.SCHEDULE_PER_TILE, tile_v=16, tile_rows=16)
     assert (a["state_pool"] - b["state_pool"]).abs().max().item() <= 1e-4
     assert (a["out"].float() - b["out"].float()).abs().max().item() <= 3e-2
 
 
-def test_chunked_rejects_unbuilt_modes():
+def test_chunked_rejects_unbuilt_modes(sched):
     w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 4))
     d = to_device(w)
     inter = torch.empty((w.T_tot, w.spec.HV, 128, 128), device="cuda")
     with pytest.raises(binding.GdnError) as e:
         binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"],
                               d["state_indices"], d["cu_seqlens"], d["out"], intermediate_states=inter,
-                              schedule=CHUNKED)
+                              schedule=sched)
     assert e.value.status == binding.ERR_UNSUPPORTED
 
 
-def test_chunked_device_status():
+def test_chunked_device_status(sched):
     w = problem([70, 20, 5], seed=11)
     w.state_indices = w.state_indices.copy()
     w.state_indices[1] = w.spec.num_slots           # out of range
-    d, status, _ = run_gpu(w, schedule=CHUNKED)
+    d, status, _ = run_gpu(w, schedule=sched)
     ost, o_ref, s_ref, _ = run_oracle(w)
     assert status == ost == oracle.BAD_SLOT
     assert_out_close(out_as_f32(d["out"]), o_ref)
@@ -134,13 +157,19 @@ def _bits_equal(a, b):
 
 def test_auto_schedule_picks_chunked_for_long_sequences():
     """GDN_SCHEDULE_AUTO: mean length >= 128 with few (sequence, head) pairs
-    runs the chunked kernel (bit-identical to asking for it); short
-    sequences, or a call with per-token states, run the per-tile kernel."""
+    runs the split chunked kernels when a workspace is given (the binding
+    allocates one) and the single chunked kernel without one (bit-identical
+    to asking for them); short sequences, or a call with per-token states,
+    run the per-tile kernel."""
     long_w = problem([200, 150, 300], seed=21)
     auto, _, _ = run_gpu(long_w)
+    split, _, _ = run_gpu(long_w, schedule=SPLIT)
+    assert _bits_equal(auto, split)
+    auto_nows, _, _ = run_gpu(long_w, workspace=None)
     chunked, _, _ = run_gpu(long_w, schedule=CHUNKED)
+    assert _bits_equal(auto_nows, chunked)
     per_tile, _, _ = run_gpu(long_w, schedule=binding.SCHEDULE_PER_TILE)
-    assert _bits_equal(auto, chunked) and not _bits_equal(auto, per_tile)
+    assert not _bits_equal(auto, per_tile) and not _bits_equal(auto, chunked)
 
     short_w = problem([3, 60, 10], seed=22)
     auto, _, _ = run_gpu(short_w)
