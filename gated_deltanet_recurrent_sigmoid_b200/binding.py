@@ -36,6 +36,8 @@ SCHEDULE_CHUNKED_SPLIT = 4
 OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5
 ERR_UNSUPPORTED, ERR_ARG, ERR_INDICES, ERR_CUDA = -6, -7, -8, -9
+ERR_SCRATCH = -10
+STATIC_SCRATCH_BYTES = 64 << 20     # gdn_decode_update_static_scratch's built-in array
 
 _DTYPE_CODES = {torch.bfloat16: 1, torch.float32: 2, torch.int32: 3}
 
@@ -89,6 +91,9 @@ def load() -> ctypes.CDLL:
         lib.gdn_version.argtypes = []
         lib.gdn_chunked_workspace_bytes.restype = ctypes.c_uint64
         lib.gdn_chunked_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        lib.gdn_decode_update_static_scratch.restype = ctypes.c_int
+        lib.gdn_decode_update_static_scratch.argtypes = [P] * 11 + [ctypes.c_float, ctypes.c_uint32,
+                                                                    ctypes.POINTER(GdnExtra)]
         _LIB = lib
     return _LIB
 
@@ -183,6 +188,35 @@ def decode_update(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Te
     _set_workspace(extra, ws)
     status = lib.gdn_decode_update(*[_ref(d) for d in descs], ctypes.c_float(scale), ctypes.c_uint32(flags),
                                    ctypes.byref(extra))
+    if status != OK:
+        raise GdnError(status, status_string(status))
+    return out
+
+
+def decode_update_static_scratch(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
+                                 b: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+                                 state_pool: torch.Tensor, state_indices: torch.Tensor,
+                                 cu_seqlens: Optional[torch.Tensor], out: torch.Tensor,
+                                 scale: Optional[float] = None, flags: int = L2NORM_QK,
+                                 device_status: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """``gdn_decode_update_static_scratch``: the split chunked update with the
+    library's built-in scratch array, for callers that cannot allocate device
+    memory.  Nothing is allocated here either.  Calls that may overlap on the
+    GPU share the array and must be ordered (e.g. issued on one stream).
+    Raises GdnError (ERR_SCRATCH when the call needs more than
+    STATIC_SCRATCH_BYTES of scratch)."""
+    lib = load()
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    descs = [describe(t) for t in (q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out)]
+    extra = GdnExtra()
+    extra.stream = stream.cuda_stream if stream is not None else None
+    extra.device_status = device_status.data_ptr() if device_status is not None else None
+    status = lib.gdn_decode_update_static_scratch(*[_ref(d) for d in descs], ctypes.c_float(scale),
+                                                  ctypes.c_uint32(flags), ctypes.byref(extra))
     if status != OK:
         raise GdnError(status, status_string(status))
     return out

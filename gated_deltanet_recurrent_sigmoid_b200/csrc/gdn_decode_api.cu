@@ -7,6 +7,8 @@
 // of the update's arithmetic; the kernel does all of it.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -680,6 +682,9 @@ GDN_API const char *gdn_status_string(int status)
     case GDN_ERR_ARG: return "GDN_ERR_ARG: bad scalar argument or flag";
     case GDN_ERR_INDICES: return "GDN_ERR_INDICES: bad or repeated state index, or bad cu_seqlens";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: the CUDA runtime refused the launch or copy";
+    case GDN_ERR_SCRATCH:
+        return "GDN_ERR_SCRATCH: the call needs more scratch than the library's static array holds "
+               "(gdn_decode_update_static_scratch: T_tot x HV too large)";
     default: return "unknown gdn status";
     }
 }
@@ -770,6 +775,91 @@ GDN_API int gdn_gating(const gdn_tensor *A_log, const gdn_tensor *a, const gdn_t
     cfg.stream = stream;
     const cudaError_t err = cudaLaunchKernelEx(&cfg, gdn::gdn_gating_kernel, p);
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scratch that needs no allocation: a fixed device array inside the library.
+//
+// gdn_decode_update_static_scratch serves callers that cannot allocate device
+// memory themselves (see include/gdn_decode.h).  Its scratch is this file-scope
+// array, created with the library's module on every GPU that loads the
+// library and held until the process exits.  On the host the name
+// `g_static_scratch` is only a stand-in for the device symbol, never a device
+// address: the device address is looked up once per device with
+// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_scratch[GDN_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_static_scratch on the current device, looked up on the
+// first call there.  Returns nullptr (and the CUDA error in *err) on failure.
+void *static_scratch_address(cudaError_t *err)
+{
+    static std::mutex lock;
+    static void *addr[64];
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess)
+        return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> guard(lock);
+    if (!addr[dev]) {
+        void *ptr = nullptr;
+        *err = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (*err != cudaSuccess)
+            return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                                             const gdn_tensor *a, const gdn_tensor *b, const gdn_tensor *A_log,
+                                             const gdn_tensor *dt_bias, const gdn_tensor *state_pool,
+                                             const gdn_tensor *state_indices, const gdn_tensor *cu_seqlens,
+                                             const gdn_tensor *out, float scale, uint32_t flags,
+                                             const gdn_extra *extra)
+{
+    if (!v)
+        return GDN_ERR_NULL_ARG;
+    if (extra && (extra->workspace || extra->workspace_bytes ||
+                  (extra->schedule != GDN_SCHEDULE_AUTO && extra->schedule != GDN_SCHEDULE_CHUNKED_SPLIT)))
+        return GDN_ERR_ARG;
+    // size check first: T_tot = all leading dims of v, HV = its second-to-last
+    if (v->ndim < 2 || v->ndim > 4)
+        return GDN_ERR_SHAPE;
+    int64_t T_tot = 1;
+    for (int d = 0; d < v->ndim - 2; ++d)
+        T_tot *= v->shape[d];
+    const int64_t HV = v->shape[v->ndim - 2];
+    if (T_tot < 0 || HV < 0)
+        return GDN_ERR_SHAPE;
+    if (T_tot > 0 && HV > 0 && gdn::split::workspace_bytes(T_tot, HV) > GDN_STATIC_SCRATCH_BYTES)
+        return GDN_ERR_SCRATCH;
+    cudaError_t err = cudaSuccess;
+    void *scratch = static_scratch_address(&err);
+    if (!scratch)
+        return GDN_ERR_CUDA;
+    gdn_extra x;
+    std::memset(&x, 0, sizeof x);
+    if (extra)
+        x = *extra;
+    x.schedule = GDN_SCHEDULE_CHUNKED_SPLIT;
+    x.workspace = scratch;
+    x.workspace_bytes = GDN_STATIC_SCRATCH_BYTES;
+    return gdn_decode_update(q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, cu_seqlens, out, scale, flags,
+                             &x);
 }
 
 }  // extern "C"

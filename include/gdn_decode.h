@@ -120,6 +120,8 @@ extern "C" {
 #define GDN_ERR_INDICES     (-8) /* GDN_CHECK_INDICES found a bad or repeated slot,
                                     or bad cu_seqlens */
 #define GDN_ERR_CUDA        (-9) /* the CUDA runtime refused the launch or copy */
+#define GDN_ERR_SCRATCH     (-10) /* gdn_decode_update_static_scratch: the call needs
+                                     more scratch than GDN_STATIC_SCRATCH_BYTES */
 
 /* work schedules (gdn_extra.schedule); all compute the same update */
 #define GDN_SCHEDULE_AUTO      0 /* library choice: GDN_SCHEDULE_CHUNKED when the
@@ -253,6 +255,47 @@ GDN_API int gdn_version(void);
  * or HV <= 0.  Host-only arithmetic, no CUDA call.
  */
 GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV);
+
+/* Size of the library's built-in scratch array (64 MiB; see below). */
+#define GDN_STATIC_SCRATCH_BYTES (64ull << 20)
+
+/*
+ * gdn_decode_update on the split chunked schedule, with NO device allocation
+ * by anyone: for callers that cannot allocate device memory -- code handed
+ * device buffers by a host program that owns every allocation (an inference
+ * server's memory planner, a plugin inside another framework), or code that
+ * must not call cudaMalloc because it may synchronise the device or fail
+ * under a fixed memory budget.  The pages have no counterpart of this entry
+ * point; it is an interface convenience of this library.
+ *
+ * Arguments and results are those of gdn_decode_update; the caller still
+ * passes every input and output.  The workspace is a fixed 64 MiB array
+ * inside the library (GDN_STATIC_SCRATCH_BYTES), created on every GPU that
+ * loads the library and kept until the process exits.  So:
+ *   - a call may need at most GDN_STATIC_SCRATCH_BYTES of workspace, i.e.
+ *     gdn_chunked_workspace_bytes(T_tot, HV) <= 64 MiB (510 records: about
+ *     4,000 tokens at HV = 8); larger calls return GDN_ERR_SCRATCH before
+ *     anything is launched;
+ *   - extra->workspace must be NULL (and workspace_bytes 0), extra->schedule
+ *     0 or GDN_SCHEDULE_CHUNKED_SPLIT; the call runs the split chunked
+ *     kernels, with their restrictions (bf16 activations, fused gates, no
+ *     GDN_WRITE_INTERMEDIATE);
+ *   - every call on a device shares the one array, which keeps the previous
+ *     call's contents.  Nothing in it needs to start at zero (each call writes
+ *     every workspace byte it reads before reading it), but two calls that
+ *     can overlap on the GPU (different streams, or different host threads,
+ *     on the same device) race on it: order such calls, e.g. on one stream;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on the device.
+ * The library allocates no device memory for this call.
+ */
+GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,
+                                             const gdn_tensor *a, const gdn_tensor *b,
+                                             const gdn_tensor *A_log, const gdn_tensor *dt_bias,
+                                             const gdn_tensor *state_pool, const gdn_tensor *state_indices,
+                                             const gdn_tensor *cu_seqlens, const gdn_tensor *out,
+                                             float scale, uint32_t flags, const gdn_extra *extra);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,8 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     assert set(declared_functions()) == {"gdn_decode_update", "gdn_recurrent_update", "gdn_gating",
-                                         "gdn_status_string", "gdn_version", "gdn_chunked_workspace_bytes"}
+                                         "gdn_status_string", "gdn_version", "gdn_chunked_workspace_bytes",
+                                         "gdn_decode_update_static_scratch"}
 
 
 def test_library_exports_every_declared_symbol(gdn_lib):
@@ -44,7 +45,7 @@ def test_version_matches_header(gdn_lib):
 
 
 def test_status_strings(gdn_lib):
-    for code in range(0, -10, -1):
+    for code in range(0, -11, -1):
         s = binding.status_string(code)
         assert s and "unknown" not in s
     assert "unknown" in binding.status_string(-100)
@@ -64,7 +65,8 @@ def test_header_constants_match_binding():
         assert define(f"GDN_SCHEDULE_{name}") == getattr(binding, f"SCHEDULE_{name}")
     for name, val in [("GDN_ERR_NULL_ARG", -1), ("GDN_ERR_DTYPE", -2), ("GDN_ERR_SHAPE", -3),
                       ("GDN_ERR_ALIGN", -4), ("GDN_ERR_ALIAS", -5), ("GDN_ERR_UNSUPPORTED", -6),
-                      ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9)]:
+                      ("GDN_ERR_ARG", -7), ("GDN_ERR_INDICES", -8), ("GDN_ERR_CUDA", -9),
+                      ("GDN_ERR_SCRATCH", -10)]:
         assert int(re.search(rf"#define {name}\s+\((-?\d+)\)", text).group(1)) == val
     assert ctypes.sizeof(binding.GdnTensor) == 8 + 4 + 4 + 8 * 4 + 8 * 4
     assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 * 4 + 8 + 8
