@@ -15,7 +15,7 @@
 //                           block's W, U^T, P, K'^T = (diag(fd) K)^T and raw Q
 //                           into the workspace as the byte images of the
 //                           operand tiles the second kernel feeds to tcgen05.
-//   gdn_chunk_state_kernel  one CTA per (sequence, value head): walks the
+//   gdn_chunk_state_kernel  one 512-thread CTA per (sequence, value head): walks the
 //                           blocks the sequence covers, fetching each block's
 //                           tiles with bulk copies one step ahead, and runs
 //                           only the state-dependent products.
@@ -495,6 +495,10 @@ struct StSmem {
     int failed;
 };
 
+// state kernel: ST_PARTS threads per TMEM lane, each handling 1 / ST_PARTS of
+// the columns of every per-thread phase
+constexpr int ST_PARTS = 4;
+constexpr int ST_THREADS = 128 * ST_PARTS;
 constexpr uint32_t ST_TMEM_COLS = 512;
 constexpr uint32_t ST_COL_S = 0;      // S~^T          [v][k]   128 columns
 constexpr uint32_t ST_COL_D = 128;    // -S~^T W^T     [v][i]    64
@@ -506,8 +510,8 @@ constexpr uint32_t ST_COL_O2 = 256;   // Delta~^T P^T  [v][j]    64
 // TMEM: with cs' = cs e^gamma_last the update is S~ += Delta~^T K'^T where
 // Delta~ = Delta / cs'.  When cs' leaves [2^-60, 2^60] the TMEM state is
 // rescaled once (S~ <- cs' S~) and cs returns to 1.
-__global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __grid_constant__ DecodeParams p,
-                                                                    const unsigned char *__restrict__ ws)
+__global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __grid_constant__ DecodeParams p,
+                                                                       const unsigned char *__restrict__ ws)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     StSmem &sm = *reinterpret_cast<StSmem *>(smem_raw);
@@ -516,6 +520,9 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    // thread (v, part): TMEM lane v = state column v; `part` picks which
+    // 1 / ST_PARTS of the columns of each per-thread phase it handles
+    const int v = tid & 127, part = tid >> 7;
     const int i = blockIdx.x / p.HV;
     const int hv = blockIdx.x - i * p.HV;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
@@ -544,8 +551,8 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
         return;
     }
     if (slot < 0) {
-        for (int t = 0; t < len; ++t)
-            out[(bos + t) * p.o_tok + hv * p.o_head + tid] = __float2bfloat16_rn(0.f);
+        for (int t = part; t < len; t += ST_PARTS)
+            out[(bos + t) * p.o_tok + hv * p.o_head + v] = __float2bfloat16_rn(0.f);
         return;
     }
     if (len == 0)
@@ -578,18 +585,20 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t my_lane = tc::tmem_addr(tmem, warp * 32, 0);
+    const uint32_t my_lane = tc::tmem_addr(tmem, (warp & 3) * 32, 0);
+    constexpr int KP = K / ST_PARTS, CP = C / ST_PARTS;   // columns per part: of S~^T, of the tokens
+    const int kh = KP * part;                   // this thread's k columns of S~^T
 
-    for (int k0 = 0; k0 < K; k0 += 16) {       // thread t = v: column v of S -> lane v of S~^T
+    for (int k0 = kh; k0 < kh + KP; k0 += 16) {   // column v of S (rows k) -> lane v of S~^T
         float x[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-            x[e] = __ldcs(s_gmem + (k0 + e) * V + tid);
+            x[e] = __ldcs(s_gmem + (k0 + e) * V + v);
         tc::tmem_st16(my_lane + ST_COL_S + k0, x);
-        st_row8(sm.st[0], tid, k0, K, x, false);
-        st_row8(sm.st[0], tid, k0 + 8, K, x + 8, false);
-        st_row8(sm.st[1], tid, k0, K, x, true);
-        st_row8(sm.st[1], tid, k0 + 8, K, x + 8, true);
+        st_row8(sm.st[0], v, k0, K, x, false);
+        st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
+        st_row8(sm.st[1], v, k0, K, x, true);
+        st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
     }
     tc::tmem_wait_st();
 
@@ -631,12 +640,13 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
         const bool more = base + r1 < eos;
         const unsigned char *rec = rec_of(blk);
 
-        // this thread's row of U^T (needed after the first product)
-        float u[64];
+        // this thread's part of the row of U^T (needed after the first product)
+        const int ih = CP * part;                 // this thread's token columns
+        float u[CP];
         {
-            const float4 *src = reinterpret_cast<const float4 *>(rec + REC_UT) + tid * 16;
+            const float4 *src = reinterpret_cast<const float4 *>(rec + REC_UT) + v * 16 + ih / 4;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
+            for (int m = 0; m < CP / 4; ++m) {
                 const float4 x = __ldg(src + m);
                 u[4 * m] = x.x;
                 u[4 * m + 1] = x.y;
@@ -680,23 +690,24 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
         if (tid < C)
             sm.fo[tid] = sm.rec_s[tid];
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
+        for (int cl = 0; cl < CP; cl += 16) {
+            const int cb = ih + cl;
             float d[16];
             tc::tmem_ld16(my_lane + ST_COL_D + cb, d);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int ii = cb + e;
-                d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[ii]) * dscale : 0.f;
+                d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[cl + e]) * dscale : 0.f;
             }
-            st_row8(sm.dt[0], tid, cb, C, d, false);
-            st_row8(sm.dt[0], tid, cb + 8, C, d + 8, false);
-            st_row8(sm.dt[1], tid, cb, C, d, true);
-            st_row8(sm.dt[1], tid, cb + 8, C, d + 8, true);
+            st_row8(sm.dt[0], v, cb, C, d, false);
+            st_row8(sm.dt[0], v, cb + 8, C, d + 8, false);
+            st_row8(sm.dt[1], v, cb, C, d, true);
+            st_row8(sm.dt[1], v, cb + 8, C, d + 8, true);
         }
         if (rescale) {               // S~ <- cs' S~ in TMEM; the scale returns to 1
 #pragma unroll 1
-            for (int k0 = 0; k0 < K; k0 += 16) {
+            for (int k0 = kh; k0 < kh + KP; k0 += 16) {
                 float x[16];
                 tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
                 tc::tmem_wait_ld();
@@ -734,7 +745,8 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
 
         // ---- outputs o_j = fo_j cs (S~0^T q_j) + cs' (Delta~^T P^T)_j --------
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
+        for (int cl = 0; cl < CP; cl += 16) {
+            const int cb = ih + cl;
             float o1[16], o2[16];
             tc::tmem_ld16(my_lane + ST_COL_O1 + cb, o1);
             tc::tmem_ld16(my_lane + ST_COL_O2 + cb, o2);
@@ -743,25 +755,25 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_chunk_state_kernel(const __gri
             for (int e = 0; e < 16; ++e) {
                 const int j = cb + e;
                 if (j >= r0 && j < r1)
-                    out[(base + j) * p.o_tok + hv * p.o_head + tid] =
+                    out[(base + j) * p.o_tok + hv * p.o_head + v] =
                         __float2bfloat16_rn(fmaf(sm.fo[j] * cs, o1[e], cs_new * o2[e]));
             }
         }
 
         // ---- the next piece's S~^T tiles, or the final write-back -----------
-        for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int k0 = kh; k0 < kh + KP; k0 += 16) {
             float x[16];
             tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
             tc::tmem_wait_ld();
             if (more) {
-                st_row8(sm.st[0], tid, k0, K, x, false);
-                st_row8(sm.st[0], tid, k0 + 8, K, x + 8, false);
-                st_row8(sm.st[1], tid, k0, K, x, true);
-                st_row8(sm.st[1], tid, k0 + 8, K, x + 8, true);
+                st_row8(sm.st[0], v, k0, K, x, false);
+                st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
+                st_row8(sm.st[1], v, k0, K, x, true);
+                st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
             } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    __stcs(s_gmem + (k0 + e) * V + tid, cs_new * x[e]);
+                    __stcs(s_gmem + (k0 + e) * V + v, cs_new * x[e]);
             }
         }
         cs = cs_new;

@@ -272,7 +272,7 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
     if (err != cudaSuccess)
         return err;
     return launch_ex(gdn::split::gdn_chunk_state_kernel, dim3(static_cast<unsigned>(units)),
-                     dim3(gdn::split::THREADS), smem_st, stream, true, p,
+                     dim3(gdn::split::ST_THREADS), smem_st, stream, true, p,
                      static_cast<const unsigned char *>(ws));
 }
 
