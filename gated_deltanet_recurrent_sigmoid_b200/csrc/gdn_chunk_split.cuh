@@ -53,10 +53,7 @@ namespace gdn {
 namespace split {
 
 using chunk::mma_tiles;
-using chunk::split2;
-using chunk::st_bf16;
 using chunk::st_row8;
-using chunk::sw64;
 using chunk::transpose8x8;
 
 constexpr int K = 128;
@@ -91,14 +88,14 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
 // Kernel 1: the state-independent products of one (block, value head).
 // ---------------------------------------------------------------------------
 struct WySmem {
-    // raw k rows 0..63 and q rows 64..127 [r][k]; after the K K^T / Q K^T
-    // product: A and T (fp32 64 x 64 each, swizzled); after the solve: the W
-    // hi / lo tiles staged for the bulk store
-    alignas(1024) unsigned char kq[128 * 128 * 2];
+    // 32 KB used in turn by: the raw k rows 0..63 and q rows 64..127 [r][k]
+    // (until the K K^T / Q K^T product); A and T by columns (fp32, 16 KB each,
+    // until the T diag() tiles); the T diag(fw) and T diag(beta) hi / lo
+    // tiles (8 KB each, until the W / U products); W^T staged for the record.
+    // The kernel fits three CTAs per SM (and three 128-column TMEM blocks).
+    alignas(1024) unsigned char r1[128 * 128 * 2];
     alignas(1024) unsigned char kt[128 * 64 * 2];     // raw k^T [k][i]
     alignas(1024) unsigned char vt[128 * 64 * 2];     // raw v^T [v][i]
-    alignas(1024) unsigned char tw[2][64 * 64 * 2];   // T diag(fw) hi / lo [j][i]; tw[0] first holds solve scratch
-    alignas(1024) unsigned char tu[2][64 * 64 * 2];   // T diag(beta) hi / lo [j][i]
     float kk[C], qq[C];                                // |k_j|^2, |q_j|^2
     float rk[C], rqs[C], g[C], beta[C], gam[C];
     float fa[C], fw[C], fo[C], fd[C];
@@ -108,10 +105,10 @@ struct WySmem {
     int failed;
 };
 
-constexpr uint32_t WY_TMEM_COLS = 256;
-constexpr uint32_t WY_COL_KQ = 0;     // [K;Q] K^T  [r][i]   64 columns
-constexpr uint32_t WY_COL_WT = 64;    // W^T        [k][j]   64
-constexpr uint32_t WY_COL_UT = 128;   // U^T        [v][j]   64
+constexpr uint32_t WY_TMEM_COLS = 128;
+constexpr uint32_t WY_COL_KQ = 0;     // [K;Q] K^T  [r][i]   64 columns (read before the W / U products)
+constexpr uint32_t WY_COL_WT = 0;     // W^T        [k][j]   64
+constexpr uint32_t WY_COL_UT = 64;    // U^T        [v][j]   64
 
 template <bool L2NORM>
 __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_constant__ DecodeParams p,
@@ -133,6 +130,9 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
     const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
     const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
+    unsigned char *const kq = sm.r1;
+    unsigned char *const tw_hi = sm.r1, *const tw_lo = sm.r1 + 8192;
+    unsigned char *const tu_hi = sm.r1 + 16384, *const tu_lo = sm.r1 + 24576;
 
     if (tid == 0) {
         sync::mbar_init(&sm.mbar, 1);
@@ -164,8 +164,8 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
             const int j = 8 * tg + r;
             if (j >= n)
                 kr[r] = qr[r] = vr[r] = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(j, col, K)) = kr[r];
-            *reinterpret_cast<uint4 *>(sm.kq + tc::kmajor_offset(64 + j, col, K)) = qr[r];
+            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(j, col, K)) = kr[r];
+            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(64 + j, col, K)) = qr[r];
             *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[r];
             float kf[8], qf[8];
             unpack8(kr[r], kf);
@@ -187,20 +187,31 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             *reinterpret_cast<uint4 *>(sm.vt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
-        // sum the 16 column groups of each row (lanes differing in bits 0..3)
-#pragma unroll
-        for (int off = 1; off < 16; off <<= 1)
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                kk[r] += __shfl_xor_sync(0xffffffffu, kk[r], off);
-                qq[r] += __shfl_xor_sync(0xffffffffu, qq[r], off);
-            }
-        if (kg == 0) {
+        // sum the 16 column groups of each row (lanes differing in bits
+        // 0..3) as a reduce-scatter: after halving exchanges with lanes 8, 4,
+        // 2, 1 apart, lane kg holds the total of value kg of the 16 values
+        // (|k|^2 of rows 0..7, then |q|^2 of rows 0..7 of the group)
+        {
+            float val[16];
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                sm.kk[8 * tg + r] = kk[r];
-                sm.qq[8 * tg + r] = qq[r];
+                val[r] = kk[r];
+                val[8 + r] = qq[r];
             }
+#pragma unroll
+            for (int half = 8; half >= 1; half >>= 1) {
+                const bool up = (kg & half) != 0;
+#pragma unroll
+                for (int i = 0; i < half; ++i) {
+                    const float send = up ? val[i] : val[half + i];
+                    const float keep = up ? val[half + i] : val[i];
+                    val[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+                }
+            }
+            if (kg < 8)
+                sm.kk[8 * tg + kg] = val[0];
+            else
+                sm.qq[8 * tg + kg - 8] = val[0];
         }
     }
     tc::fence_before_sync();
@@ -307,123 +318,141 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
 
     // ---- step 2: [K;Q] K^T ---------------------------------------------------
     if (tid == 0) {
-        mma_tiles(tmem + WY_COL_KQ, sm.kq, K, sm.kq, K, K / 16, ID_M128_N64, false);
+        mma_tiles(tmem + WY_COL_KQ, kq, K, kq, K, K / 16, ID_M128_N64, false);
         tc::mma_commit(&sm.mbar);
     }
     wait_mma();
 
-    float *Amat = reinterpret_cast<float *>(sm.kq);              // [64][64] fp32, swizzled
-    float *Tmat = reinterpret_cast<float *>(sm.kq + 64 * 64 * 4);
+    // A stored by columns, At[c][j] = A[j][c], and T by columns with the row
+    // index XOR-swizzled by the column (both fp32 [64][64], in r1: the raw
+    // tiles are consumed)
+    constexpr int A_LD = 64;
+    float *At = reinterpret_cast<float *>(sm.r1);
+    float *Tcol = reinterpret_cast<float *>(sm.r1 + 16384);
     if (ok) {
-        // ---- step 3: A (rows 0..63, smem) and P (rows 64..127, to the record)
-        float row[64];
+        // ---- step 3: A (rows 0..63: warps 0, 1, into At) and P (rows
+        // 64..127: warps 2, 3, straight to the record), 16 columns at a time
+        {
+            const int j = tid & 63, sj = sm.ss[j];
+            const float fj = tid < 64 ? sm.fa[j] : sm.rqs[j], gj = sm.gam[j];
+#pragma unroll 1
+            for (int cb = 0; cb < 64; cb += 16) {
+                float row[16];
+                tc::tmem_ld16(my_lane + WY_COL_KQ + cb, row);
+                tc::tmem_wait_ld();
+                if (tid < 64) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 16)
-            tc::tmem_ld16(my_lane + WY_COL_KQ + c, row + c);
-        tc::tmem_wait_ld();
-        if (tid < 64) {
-            const int j = tid, sj = sm.ss[j];
-            const float fj = sm.fa[j], gj = sm.gam[j];
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = cb + e;
+                        At[c * A_LD + j] = (c < j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[e] : 0.f;
+                    }
+                } else {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-                Amat[sw64(j, c)] = (c < j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
-        } else {
-            const int j = tid - 64, sj = sm.ss[j];
-            const float fj = sm.rqs[j], gj = sm.gam[j];
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-                row[c] = (c <= j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[c] : 0.f;
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-                st_row8(rec + REC_P_HI, j, c, C, row + c, false);
-                st_row8(rec + REC_P_LO, j, c, C, row + c, true);
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = cb + e;
+                        row[e] = (c <= j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[e] : 0.f;
+                    }
+                    st_row8(rec + REC_P_HI, j, cb, C, row, false);
+                    st_row8(rec + REC_P_HI, j, cb + 8, C, row + 8, false);
+                    st_row8(rec + REC_P_LO, j, cb, C, row, true);
+                    st_row8(rec + REC_P_LO, j, cb + 8, C, row + 8, true);
+                }
             }
         }
         __syncthreads();
 
-        // ---- step 4: T = (I + A)^-1, blocked by 16 x 16 (as in the
-        // single-kernel schedule) ------------------------------------------
-        float *X = reinterpret_cast<float *>(sm.tw[0]);   // scratch [3][16][16]
-        if (tid < 64) {
-            const int I = tid >> 4, cc = tid & 15, c = 16 * I + cc;
-            float x[16];
+        // ---- step 4: T = (I + A)^-1 by columns: warp w solves columns
+        // 16 w .. 16 w + 15, its lanes holding rows lane and lane + 32.  By
+        // elimination: x = e_c; for r = 0 .. 62, x_r' -= A[r'][r] x_r for all
+        // r' (A[r'][r] = 0 unless r' > r, so rows <= r are unchanged and x_r
+        // is final when it is broadcast from its lane).
+        {
+            const int lane = tid & 31, c0 = 16 * warp;
+            float xl[16], xh[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-                for (int m = 0; m < r; ++m)
-                    acc = fmaf(-Amat[sw64(16 * I + r, 16 * I + m)], x[m], acc);
-                x[r] = (r < cc) ? 0.f : acc;
-                Tmat[sw64(16 * I + r, c)] = x[r];
+            for (int cc = 0; cc < 16; ++cc) {
+                xl[cc] = (lane == c0 + cc) ? 1.f : 0.f;
+                xh[cc] = (lane + 32 == c0 + cc) ? 1.f : 0.f;
             }
-        } else {
-            for (int e = tid - 64; e < 6 * 256; e += 64) {
-                const int b6 = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int I = b6 < 3 ? 0 : (b6 < 5 ? 1 : 2);
-                const int J = b6 < 3 ? b6 + 1 : (b6 < 5 ? b6 - 1 : 3);
-                Tmat[sw64(16 * I + r, 16 * J + cc)] = 0.f;
+            // x_r = 0 for r < c0 in all of this warp's columns: start at c0.
+            // Rows r < 32: x_r sits in lane r's xl; rows lane and lane + 32
+            // are updated.
+#pragma unroll 1
+            for (int r = c0; r < 32; ++r) {
+                const float al = At[r * A_LD + lane], ah = At[r * A_LD + 32 + lane];   // A[lane][r], A[lane + 32][r]
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    const float xr = __shfl_sync(0xffffffffu, xl[cc], r);
+                    xl[cc] = fmaf(-al, xr, xl[cc]);
+                    xh[cc] = fmaf(-ah, xr, xh[cc]);
+                }
+            }
+            // rows r >= 32: x_r sits in lane r - 32's xh; rows < 32 are final
+#pragma unroll 1
+            for (int r = c0 > 32 ? c0 : 32; r < 63; ++r) {
+                const float ah = At[r * A_LD + 32 + lane];
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    const float xr = __shfl_sync(0xffffffffu, xh[cc], r - 32);
+                    xh[cc] = fmaf(-ah, xr, xh[cc]);
+                }
+            }
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+                const int c = c0 + cc;
+                Tcol[c * 64 + (lane ^ (c & 31))] = xl[cc];
+                Tcol[c * 64 + ((lane + 32) ^ (c & 31))] = xh[cc];
             }
         }
         __syncthreads();
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            for (int e = tid; e < nb * 256; e += THREADS) {
-                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
-                float acc = 0.f;
-                for (int M = J; M < I; ++M)
-#pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc = fmaf(Amat[sw64(16 * I + r, 16 * M + m)], Tmat[sw64(16 * M + m, 16 * J + cc)], acc);
-                X[e] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += THREADS) {
-                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = J + d;
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(Tmat[sw64(16 * I + r, 16 * I + m)], X[(J << 8) + (m << 4) + cc], acc);
-                Tmat[sw64(16 * I + r, 16 * J + cc)] = -acc;
-            }
-            __syncthreads();
-        }
-        // T diag(fw) and T diag(beta) as hi / lo operand tiles
+
+        // T diag(fw) and T diag(beta) as hi / lo operand tiles: each thread
+        // takes four 8-column chunks of rows of T (read all, then write over
+        // the area T occupied)
         {
-            const int r = tid >> 1, cbase = 32 * (tid & 1);
+            float t8[4][8];
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
+            for (int n = 0; n < 4; ++n) {
+                const int q = tid + 128 * n, r = q >> 3, c0 = (q & 7) * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    t8[n][e] = Tcol[(c0 + e) * 64 + (r ^ ((c0 + e) & 31))];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int q = tid + 128 * n, r = q >> 3, c0 = (q & 7) * 8;
                 float tw8[8], tu8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int col = cbase + c + e;
-                    const float t = Tmat[sw64(r, col)];
-                    tw8[e] = t * sm.fw[col];
-                    tu8[e] = t * sm.beta[col];
+                    tw8[e] = t8[n][e] * sm.fw[c0 + e];
+                    tu8[e] = t8[n][e] * sm.beta[c0 + e];
                 }
-                st_row8(sm.tw[0], r, cbase + c, C, tw8, false);
-                st_row8(sm.tw[1], r, cbase + c, C, tw8, true);
-                st_row8(sm.tu[0], r, cbase + c, C, tu8, false);
-                st_row8(sm.tu[1], r, cbase + c, C, tu8, true);
+                st_row8(tw_hi, r, c0, C, tw8, false);
+                st_row8(tw_lo, r, c0, C, tw8, true);
+                st_row8(tu_hi, r, c0, C, tu8, false);
+                st_row8(tu_lo, r, c0, C, tu8, true);
             }
         }
         publish_smem();
 
         // ---- step 5: W^T = K^T T_w^T and U^T = V^T T_u^T ----------------
         if (tid == 0) {
-            mma_tiles(tmem + WY_COL_WT, sm.kt, C, sm.tw[0], C, C / 16, ID_M128_N64, false);
-            mma_tiles(tmem + WY_COL_WT, sm.kt, C, sm.tw[1], C, C / 16, ID_M128_N64, true);
-            mma_tiles(tmem + WY_COL_UT, sm.vt, C, sm.tu[0], C, C / 16, ID_M128_N64, false);
-            mma_tiles(tmem + WY_COL_UT, sm.vt, C, sm.tu[1], C, C / 16, ID_M128_N64, true);
+            mma_tiles(tmem + WY_COL_WT, sm.kt, C, tw_hi, C, C / 16, ID_M128_N64, false);
+            mma_tiles(tmem + WY_COL_WT, sm.kt, C, tw_lo, C, C / 16, ID_M128_N64, true);
+            mma_tiles(tmem + WY_COL_UT, sm.vt, C, tu_hi, C, C / 16, ID_M128_N64, false);
+            mma_tiles(tmem + WY_COL_UT, sm.vt, C, tu_lo, C, C / 16, ID_M128_N64, true);
             tc::mma_commit(&sm.mbar);
         }
         wait_mma();
     }
     if (ok) {
         // ---- step 6: the record's remaining tiles -------------------------
-        // W (thread = k): hi / lo tiles [i][k] staged in the kq area (A and T
-        // are dead), then one bulk store of both
-        unsigned char *w_hi = sm.kq, *w_lo = sm.kq + 64 * 128 * 2;
+        // W (thread = k): W^T[k][.] from TMEM into a padded fp32 buffer
+        // [k][64] (column index XOR-swizzled by the row) in r1, free after the
+        // products; the hi / lo chunks of W [i][k] go to the record once it
+        // is complete
+        float *Wpad = reinterpret_cast<float *>(sm.r1);
         {
             float wcol[64];
 #pragma unroll
@@ -431,12 +460,8 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
                 tc::tmem_ld16(my_lane + WY_COL_WT + c, wcol + c);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                __nv_bfloat16 hi, lo;
-                split2(wcol[j], hi, lo);
-                st_bf16(w_hi, j, tid, K, hi);
-                st_bf16(w_lo, j, tid, K, lo);
-            }
+            for (int j = 0; j < 64; ++j)
+                Wpad[tid * 64 + (j ^ (tid & 31))] = wcol[j];
         }
         // U^T (thread = v): one fp32 row of 64
         {
@@ -464,12 +489,17 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
                 st_row8(rec + REC_KP_LO, tid, c, C, x, true);
             }
         }
-        sync::fence_proxy_async();
         __syncthreads();
-        if (tid == 0) {
-            sync::bulk_store(rec + REC_W_HI, sm.kq, 2 * 64 * 128 * 2);
-            sync::bulk_commit();
-            sync::bulk_wait_all();
+        // W hi / lo: 16-byte chunks (row i, columns k0 .. k0 + 7), eight per thread
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int q = tid + 128 * n, i = q & 63, k0 = (q >> 6) * 8;
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                w8[e] = Wpad[(k0 + e) * 64 + (i ^ ((k0 + e) & 31))];
+            st_row8(rec + REC_W_HI, i, k0, K, w8, false);
+            st_row8(rec + REC_W_LO, i, k0, K, w8, true);
         }
     }
 

@@ -262,6 +262,11 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem_st));
+        // the largest shared-memory carveout, so that three block-kernel CTAs
+        // fit on an SM
+        for (int l2 = 0; l2 < 2 && err == cudaSuccess; ++l2)
+            err = cudaFuncSetAttribute(l2 ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
+                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (err != cudaSuccess)
             return err;
         ready[dev] = true;
