@@ -64,19 +64,21 @@ constexpr int THREADS = 128;
 // One workspace record per (block, value head): byte offsets.  Tiles are in
 // the K-major core-matrix layout of tc_sm100.cuh; [r][c] names the rows and
 // the contraction dimension.
+// W hi and Q are adjacent so that [W hi; Q] is one 128-row operand, and so
+// are [K'^T hi; P hi] and [K'^T lo; P lo] (192 rows each).
 constexpr uint32_t REC_W_HI = 0;          // W hi              [i][k]   16 KB
-constexpr uint32_t REC_W_LO = 16384;      // W lo              [i][k]   16 KB
-constexpr uint32_t REC_Q = 32768;         // raw q             [j][k]   16 KB
+constexpr uint32_t REC_Q = 16384;         // raw q             [j][k]   16 KB
+constexpr uint32_t REC_W_LO = 32768;      // W lo              [i][k]   16 KB
 constexpr uint32_t REC_KP_HI = 49152;     // K'^T hi           [k][i]   16 KB
-constexpr uint32_t REC_KP_LO = 65536;     // K'^T lo           [k][i]   16 KB
-constexpr uint32_t REC_P_HI = 81920;      // P hi              [j][i]    8 KB
+constexpr uint32_t REC_P_HI = 65536;      // P hi              [j][i]    8 KB
+constexpr uint32_t REC_KP_LO = 73728;     // K'^T lo           [k][i]   16 KB
 constexpr uint32_t REC_P_LO = 90112;      // P lo              [j][i]    8 KB
 constexpr uint32_t REC_UT = 98304;        // U^T fp32, row-major [v][i]  32 KB
 constexpr uint32_t REC_FO = 131072;       // fo_j = e^gamma_j rqs_j     256 B
 constexpr uint32_t REC_GAM = 131328;      // gamma_j                    256 B
 constexpr uint32_t REC_BYTES = 131584;    // a multiple of 256
-constexpr uint32_t REC_A_BYTES = REC_KP_HI;               // W hi, W lo, Q
-constexpr uint32_t REC_B_BYTES = REC_UT - REC_KP_HI;      // K'^T hi / lo, P hi / lo
+constexpr uint32_t REC_A_BYTES = REC_KP_HI;               // W hi, Q, W lo
+constexpr uint32_t REC_B_BYTES = REC_UT - REC_KP_HI;      // K'^T hi, P hi, K'^T lo, P lo
 constexpr uint32_t REC_S_BYTES = REC_BYTES - REC_FO;      // fo, gamma
 
 __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV)
@@ -515,12 +517,15 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
 // ---------------------------------------------------------------------------
 struct StSmem {
     alignas(1024) unsigned char st[2][128 * 128 * 2];   // S~^T hi / lo [v][k]
-    alignas(1024) unsigned char rec_a[REC_A_BYTES];     // W hi, W lo, Q of the piece (record bytes 0 .. 49151)
-    alignas(1024) unsigned char rec_b[REC_B_BYTES];     // K'^T hi / lo, P hi / lo (record bytes 49152 .. 98303)
+    alignas(1024) unsigned char rec_a[REC_A_BYTES];     // W hi, Q, W lo of the piece (record bytes 0 .. 49151)
+    alignas(1024) unsigned char rec_b[REC_B_BYTES];     // K'^T hi, P hi, K'^T lo, P lo (record bytes 49152 .. 98303)
     alignas(1024) unsigned char dt[2][128 * 64 * 2];    // Delta~^T hi / lo [v][i]
     alignas(16) float rec_s[REC_S_BYTES / 4];           // fo, gamma of the piece (record tail)
-    float fo[C];                                        // fo of the piece being finished
-    unsigned long long bar_mma, bar_a, bar_b;
+    float fo[2][C];                                     // fo of the last two pieces (by piece parity)
+    // bar_d: -S~^T [W; Q]^T done; bar_s: S~^T += Delta~^T [K'; P]^T done;
+    // bar_a / bar_b / bar_r: the bulk copies of a piece's W / Q, K' / P and
+    // fo / gamma
+    unsigned long long bar_d, bar_s, bar_a, bar_b, bar_r;
     uint32_t tmem_base;
     int failed;
 };
@@ -530,10 +535,12 @@ struct StSmem {
 constexpr int ST_PARTS = 4;
 constexpr int ST_THREADS = 128 * ST_PARTS;
 constexpr uint32_t ST_TMEM_COLS = 512;
-constexpr uint32_t ST_COL_S = 0;      // S~^T          [v][k]   128 columns
-constexpr uint32_t ST_COL_D = 128;    // -S~^T W^T     [v][i]    64
-constexpr uint32_t ST_COL_O1 = 192;   // S~^T Q^T      [v][j]    64
-constexpr uint32_t ST_COL_O2 = 256;   // Delta~^T P^T  [v][j]    64
+// TMEM columns.  Product 2 writes [S~^T | O2] (192 columns) in one MMA,
+// product 1 [D | O1] (128) in one MMA; [D | O1] is double-buffered by piece
+// parity so that a piece's O1 can be read during the next piece.
+constexpr uint32_t ST_COL_S = 0;      // S~^T              [v][k]   128 columns
+constexpr uint32_t ST_COL_O2 = 128;   // Delta~^T P^T      [v][j]    64
+constexpr uint32_t ST_COL_DQ = 256;   // -S~^T W^T (64), then -S~^T Q^T (64); 2 x 128 by piece parity
 
 // The state is kept as S = cs * S~ for a per-CTA scale cs, so a piece's
 // decay e^gamma_last multiplies cs instead of the 16 K state elements in
@@ -595,17 +602,20 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     // state into TMEM and into the S~^T tiles (cs = 1) ----------------------
     int64_t blk = bos / C;
     if (tid == 0) {
-        sync::mbar_init(&sm.bar_mma, 1);
+        sync::mbar_init(&sm.bar_d, 1);
+        sync::mbar_init(&sm.bar_s, 1);
         sync::mbar_init(&sm.bar_a, 1);
         sync::mbar_init(&sm.bar_b, 1);
+        sync::mbar_init(&sm.bar_r, 1);
         sm.failed = 0;
         sync::fence_barrier_init();
         const unsigned char *r = rec_of(blk);
         sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
         sync::bulk_load(sm.rec_a, r, REC_A_BYTES, &sm.bar_a);
-        sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES + REC_S_BYTES);
+        sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES);
         sync::bulk_load(sm.rec_b, r + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
-        sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_b);
+        sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
+        sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_r);
     }
     if (warp == 0) {
         tc::tmem_alloc(&sm.tmem_base, ST_TMEM_COLS);
@@ -632,10 +642,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     }
     tc::tmem_wait_st();
 
-    uint32_t ph_mma = 0, ph_a = 0, ph_b = 0;
+    uint32_t ph_d = 0, ph_s = 0, ph_a = 0, ph_b = 0, ph_r = 0;
     // copies issued and not yet waited for, with the parity their wait checks
-    bool ok = true, pend_a = true, pend_b = true;
-    uint32_t pa = 0, pb = 0;
+    bool ok = true, pend_a = true, pend_b = true, pend_r = true;
+    uint32_t pa = 0, pb = 0, pr = 0;
     // bounded wait on one of the barriers; uniform verdict over the CTA
     auto wait_bar = [&](unsigned long long *bar, uint32_t &ph) {
         bool w = ok && sync::mbar_wait(bar, ph, &sm.failed);
@@ -655,15 +665,41 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     };
     publish_smem();
 
-    const uint32_t ID_N64 = tc::idesc_bf16_f32(128, 64);
     const uint32_t ID_N64_NEG = tc::idesc_bf16_f32(128, 64, true);
-    const uint32_t ID_N128 = tc::idesc_bf16_f32(128, 128);
-    const unsigned char *w_hi = sm.rec_a + REC_W_HI, *w_lo = sm.rec_a + REC_W_LO, *q_t = sm.rec_a + REC_Q;
-    const unsigned char *kp_hi = sm.rec_b + (REC_KP_HI - REC_KP_HI), *kp_lo = sm.rec_b + (REC_KP_LO - REC_KP_HI);
-    const unsigned char *p_hi = sm.rec_b + (REC_P_HI - REC_KP_HI), *p_lo = sm.rec_b + (REC_P_LO - REC_KP_HI);
+    const uint32_t ID_N128_NEG = tc::idesc_bf16_f32(128, 128, true);
+    const uint32_t ID_N192 = tc::idesc_bf16_f32(128, 192);
+    const unsigned char *wq_hi = sm.rec_a + REC_W_HI, *w_lo = sm.rec_a + REC_W_LO;   // [W hi; Q], W lo
+    const unsigned char *kpp_hi = sm.rec_b, *kpp_lo = sm.rec_b + (REC_KP_LO - REC_KP_HI);  // [K'^T; P] hi, lo
+
+    // Outputs of a piece are written during the next piece (while its first
+    // products run); these describe the piece whose outputs are pending.
+    int64_t out_base = 0;
+    int out_r0 = 0, out_r1 = 0, out_buf = 0;
+    float out_cs = 0.f, out_cs_new = 0.f;
+    bool out_pending = false;
+    auto write_outputs = [&]() {
+        const uint32_t o1c = ST_COL_DQ + 128u * out_buf + 64u, o2c = ST_COL_O2;
+#pragma unroll
+        for (int cl = 0; cl < CP; cl += 16) {
+            const int cb = CP * part + cl;
+            float o1[16], o2[16];
+            tc::tmem_ld16(my_lane + o1c + cb, o1);
+            tc::tmem_ld16(my_lane + o2c + cb, o2);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = cb + e;
+                if (j >= out_r0 && j < out_r1)
+                    out[(out_base + j) * p.o_tok + hv * p.o_head + v] =
+                        __float2bfloat16_rn(fmaf(-sm.fo[out_buf][j] * out_cs, o1[e], out_cs_new * o2[e]));
+            }
+        }
+        out_pending = false;
+    };
 
     float cs = 1.f;
-    for (int64_t t = bos; t < eos && ok; ++blk) {
+    int buf = 0;
+    for (int64_t t = bos; t < eos && ok; ++blk, buf ^= 1) {
         const int64_t base = blk * C;
         const int r0 = static_cast<int>(t - base);
         const int r1 = static_cast<int>((eos < base + C ? eos : base + C) - base);
@@ -685,20 +721,25 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             }
         }
 
-        // ---- product 1: -S~^T W^T (3 split products) and S~^T Q^T (2) ----
+        // ---- product 1: [D | O1] = -S~^T [W hi; Q]^T (hi and lo parts of S~)
+        // and D -= S~hi^T W lo^T (bar_d) -------------------------------------
         wait_bar(&sm.bar_a, ph_a);
         if (!ok)
             break;
         pend_a = false;
+        const uint32_t dq = ST_COL_DQ + 128u * buf;
         if (tid == 0) {
-            mma_tiles(tmem + ST_COL_D, sm.st[0], K, w_hi, K, K / 16, ID_N64_NEG, false);
-            mma_tiles(tmem + ST_COL_D, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
-            mma_tiles(tmem + ST_COL_D, sm.st[1], K, w_hi, K, K / 16, ID_N64_NEG, true);
-            mma_tiles(tmem + ST_COL_O1, sm.st[0], K, q_t, K, K / 16, ID_N64, false);
-            mma_tiles(tmem + ST_COL_O1, sm.st[1], K, q_t, K, K / 16, ID_N64, true);
-            tc::mma_commit(&sm.bar_mma);
+            mma_tiles(tmem + dq, sm.st[0], K, wq_hi, K, K / 16, ID_N128_NEG, false);
+            mma_tiles(tmem + dq, sm.st[1], K, wq_hi, K, K / 16, ID_N128_NEG, true);
+            mma_tiles(tmem + dq, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
+            tc::mma_commit(&sm.bar_d);
         }
-        wait_bar(&sm.bar_mma, ph_mma);
+        // the previous piece's outputs, while these products run
+        if (out_pending)
+            write_outputs();
+
+        // ---- Delta~^T (thread = v) into its hi / lo tiles -----------------
+        wait_bar(&sm.bar_d, ph_d);
         if (!ok)
             break;
         if (more && tid == 0) {       // W and Q of the next piece, into the buffer just read
@@ -707,9 +748,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         }
         pend_a = more;
         pa = ph_a;
-
-        // ---- Delta~^T (thread = v) into its hi / lo tiles -----------------
-        wait_bar(&sm.bar_b, ph_b);
+        wait_bar(&sm.bar_r, ph_r);
+        if (!ok)
+            break;
+        pend_r = false;
+        wait_bar(&sm.bar_b, ph_b);            // K' and P of this piece
         if (!ok)
             break;
         pend_b = false;
@@ -718,12 +761,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         const bool rescale = !(cn >= 0x1p-60f && cn <= 0x1p60f);
         const float dscale = rescale ? 1.f : __fdividef(1.f, cn);
         if (tid < C)
-            sm.fo[tid] = sm.rec_s[tid];
+            sm.fo[buf][tid] = sm.rec_s[tid];
 #pragma unroll
         for (int cl = 0; cl < CP; cl += 16) {
             const int cb = ih + cl;
             float d[16];
-            tc::tmem_ld16(my_lane + ST_COL_D + cb, d);
+            tc::tmem_ld16(my_lane + dq + cb, d);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -734,6 +777,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             st_row8(sm.dt[0], v, cb + 8, C, d + 8, false);
             st_row8(sm.dt[1], v, cb, C, d, true);
             st_row8(sm.dt[1], v, cb + 8, C, d + 8, true);
+        }
+        {                            // O2 accumulates from zero in product 2
+            float z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                z[e] = 0.f;
+#pragma unroll
+            for (int cl = 0; cl < CP; cl += 16)
+                tc::tmem_st16(my_lane + ST_COL_O2 + ih + cl, z);
         }
         if (rescale) {               // S~ <- cs' S~ in TMEM; the scale returns to 1
 #pragma unroll 1
@@ -749,46 +801,41 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             tc::tmem_wait_st();
         }
         const float cs_new = rescale ? 1.f : cn;
+        tc::tmem_wait_st();
         publish_smem();
 
-        // ---- product 2: Delta~^T P^T (3) and S~^T += Delta~^T K'^T (3) -----
+        // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T (3 split products;
+        // bar_s) ------------------------------------------------------------
         if (tid == 0) {
-            mma_tiles(tmem + ST_COL_O2, sm.dt[0], C, p_hi, C, C / 16, ID_N64, false);
-            mma_tiles(tmem + ST_COL_O2, sm.dt[0], C, p_lo, C, C / 16, ID_N64, true);
-            mma_tiles(tmem + ST_COL_O2, sm.dt[1], C, p_hi, C, C / 16, ID_N64, true);
-            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kp_hi, C, C / 16, ID_N128, true);
-            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kp_lo, C, C / 16, ID_N128, true);
-            mma_tiles(tmem + ST_COL_S, sm.dt[1], C, kp_hi, C, C / 16, ID_N128, true);
-            tc::mma_commit(&sm.bar_mma);
+            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kpp_hi, C, C / 16, ID_N192, true);
+            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kpp_lo, C, C / 16, ID_N192, true);
+            mma_tiles(tmem + ST_COL_S, sm.dt[1], C, kpp_hi, C, C / 16, ID_N192, true);
+            tc::mma_commit(&sm.bar_s);
+            if (more) {              // fo / gamma of the next piece (read above)
+                sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
+                sync::bulk_load(sm.rec_s, rec_of(blk + 1) + REC_FO, REC_S_BYTES, &sm.bar_r);
+            }
         }
-        wait_bar(&sm.bar_mma, ph_mma);
+        pend_r = more;
+        pr = ph_r;
+
+        // K' and P of the next piece once both products that read them are done
+        wait_bar(&sm.bar_s, ph_s);
         if (!ok)
             break;
-        if (more && tid == 0) {       // K', P, fo, gamma of the next piece
-            const unsigned char *r = rec_of(blk + 1);
-            sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES + REC_S_BYTES);
-            sync::bulk_load(sm.rec_b, r + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
-            sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_b);
+        if (more && tid == 0) {
+            sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES);
+            sync::bulk_load(sm.rec_b, rec_of(blk + 1) + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
         }
         pend_b = more;
         pb = ph_b;
-
-        // ---- outputs o_j = fo_j cs (S~0^T q_j) + cs' (Delta~^T P^T)_j --------
-#pragma unroll
-        for (int cl = 0; cl < CP; cl += 16) {
-            const int cb = ih + cl;
-            float o1[16], o2[16];
-            tc::tmem_ld16(my_lane + ST_COL_O1 + cb, o1);
-            tc::tmem_ld16(my_lane + ST_COL_O2 + cb, o2);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int j = cb + e;
-                if (j >= r0 && j < r1)
-                    out[(base + j) * p.o_tok + hv * p.o_head + v] =
-                        __float2bfloat16_rn(fmaf(sm.fo[j] * cs, o1[e], cs_new * o2[e]));
-            }
-        }
+        out_base = base;
+        out_r0 = r0;
+        out_r1 = r1;
+        out_buf = buf;
+        out_cs = cs;
+        out_cs_new = cs_new;
+        out_pending = true;
 
         // ---- the next piece's S~^T tiles, or the final write-back -----------
         for (int k0 = kh; k0 < kh + KP; k0 += 16) {
@@ -810,15 +857,19 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         t = base + r1;
         publish_smem();
     }
+    if (ok && out_pending)
+        write_outputs();
 
     // a failed wait left copies in flight: let them land (bounded) before the
     // shared memory is released
-    if (pend_a || pend_b) {
+    if (pend_a || pend_b || pend_r) {
         volatile int never = 0;
         if (pend_a)
             sync::mbar_wait(&sm.bar_a, pa, &never);
         if (pend_b)
             sync::mbar_wait(&sm.bar_b, pb, &never);
+        if (pend_r)
+            sync::mbar_wait(&sm.bar_r, pr, &never);
     }
 
     pdl_trigger();

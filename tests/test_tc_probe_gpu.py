@@ -21,7 +21,7 @@ def probe():
     return lib
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 64, 128), (128, 128, 64), (128, 256, 128), (128, 16, 16),
+@pytest.mark.parametrize("M,N,K", [(128, 64, 128), (128, 128, 64), (128, 256, 128), (128, 192, 64), (128, 16, 16),
                                    (64, 64, 128), (64, 128, 64)])
 @pytest.mark.parametrize("negate,twice", [(0, 0), (1, 1)], ids=["plain", "neg_acc"])
 def test_tile_product_matches_matmul(probe, M, N, K, negate, twice):
