@@ -32,6 +32,13 @@ constexpr int kHeadV = 128;
 constexpr int64_t kChunkedMinMeanTokensFew = 128;
 constexpr int64_t kChunkedMinMeanTokensMany = 256;
 constexpr int64_t kChunkedFewPairs = 1024;
+// With a workspace, AUTO takes the split chunked kernels from a lower mean
+// length (measured B200 crossovers against the per-tile kernel, lengths
+// spread over [L/2, 3L/2]): 64 tokens below 64 (sequence, value head)
+// pairs, 40 below 512, 26 from 512 on (at the threshold the split kernels
+// are 0.7-1.0 of the per-tile time; with 64-1024 sequences the ratio is
+// 1.01-1.04 at 24 tokens and 0.89-0.97 at 28).
+int64_t split_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 64 : (pairs < 512 ? 40 : 26); }
 
 int64_t elem_size(int32_t dtype)
 {
@@ -571,9 +578,12 @@ int run_update(const UpdateArgs &c)
     const bool v_rows_16b =
         aligned(v->data, 16) && stride_ok(T_tot, Lv.tok, 8) && stride_ok(HV, v->stride[v->ndim - 2], 8);
     if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
-        act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0 &&
-        T_tot >= (N * HV <= kChunkedFewPairs ? kChunkedMinMeanTokensFew : kChunkedMinMeanTokensMany) * N)
-        schedule = ws_fits ? GDN_SCHEDULE_CHUNKED_SPLIT : GDN_SCHEDULE_CHUNKED;
+        act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0) {
+        if (ws_fits && T_tot >= split_min_mean_tokens(N * HV) * N)
+            schedule = GDN_SCHEDULE_CHUNKED_SPLIT;
+        else if (T_tot >= (N * HV <= kChunkedFewPairs ? kChunkedMinMeanTokensFew : kChunkedMinMeanTokensMany) * N)
+            schedule = GDN_SCHEDULE_CHUNKED;
+    }
     // The pipelined schedule is built for bf16 activations and fused bf16
     // gates; the chunked one for bf16 activations, fused gates and no
     // per-token states.

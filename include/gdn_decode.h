@@ -124,13 +124,17 @@ extern "C" {
                                      more scratch than GDN_STATIC_SCRATCH_BYTES */
 
 /* work schedules (gdn_extra.schedule); all compute the same update */
-#define GDN_SCHEDULE_AUTO      0 /* library choice: GDN_SCHEDULE_CHUNKED when the
-                                    call qualifies for it (bf16 activations, fused
+#define GDN_SCHEDULE_AUTO      0 /* library choice.  When the call qualifies for
+                                    the chunked kernels (bf16 activations, fused
                                     gates, no per-token states, v rows 16-byte
-                                    aligned) and holds enough tokens per
-                                    sequence on average: >= 128 when N * HV <=
-                                    1024, else >= 256 (total tokens >= 128 N or
-                                    256 N); else GDN_SCHEDULE_PER_TILE */
+                                    aligned): GDN_SCHEDULE_CHUNKED_SPLIT if the
+                                    caller gives a large enough workspace and
+                                    the sequences hold, on average, >= 64 tokens
+                                    (N * HV < 64), >= 40 (N * HV < 512) or >= 26
+                                    (otherwise); without a workspace
+                                    GDN_SCHEDULE_CHUNKED from >= 128 tokens
+                                    (N * HV <= 1024) or >= 256.  Otherwise
+                                    GDN_SCHEDULE_PER_TILE */
 #define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
                                     state tile moves through registers.  Tiles
                                     (tile_v x tile_rows): 16x16, 32x16, 32x32,
