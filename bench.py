@@ -55,8 +55,8 @@ def chunked_min_mean_tokens(pairs):
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
 # dram__bytes_write.sum).  Valid only for the kernel sources it was taken on.
-NCU_TRAFFIC = {"kernel_sha256": "f6b891eb3ef14a8b7d52962a1f3d8ee3936fd0e76d342ecfa9ca84115a87cc36",
-               "workload": "decode_b512_hv8", "bytes_per_launch": 257378816 + 197948416}
+NCU_TRAFFIC = {"kernel_sha256": "56a5bd6fd0f772dbd0de9456b16af0c872fa8c6c4137184b3fa31d1fb1ea9a96",
+               "workload": "decode_b512_hv8", "bytes_per_launch": 257377792 + 202355968}
 
 
 def kernel_source_hash() -> str:
