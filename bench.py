@@ -177,6 +177,17 @@ def subset_bytes(w, seqs):
     return nbytes
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, budget_s=10.0):
     """The oracle as it stands, single-threaded, over the whole workload
     repeated until about ``budget_s`` seconds of CPU work."""
@@ -188,7 +199,7 @@ def cpu_baseline(w, budget_s=10.0):
         reps += 1
     per = total_t / reps
     return {"value": round(wl.algorithmic_bytes(w) / per / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle", "us_per_call": round(per * 1e6, 1),
+            "kind": "oracle", "us_per_call": round(per * 1e6, 1), "cpu": cpu_model(),
             "sample": f"whole {w.spec.name} workload ({w.spec.N} sequences), {reps} repetitions, "
                       f"{total_t:.1f} s single-threaded fp64 C loop nest"}
 
@@ -213,7 +224,7 @@ def cpu_baseline_all_cores(w, budget_s=10.0):
             reps += 1
     per = total_t / reps
     return {"value": round(wl.algorithmic_bytes(w) / per / 1e9, 4), "unit": "GB/s", "cores": len(groups),
-            "kind": "oracle", "us_per_call": round(per * 1e6, 1),
+            "kind": "oracle", "us_per_call": round(per * 1e6, 1), "cpu": cpu_model(),
             "sample": f"whole {w.spec.name} workload split into {len(groups)} sequence groups, one thread each, "
                       f"{reps} repetitions, {total_t:.1f} s"}
 
@@ -238,7 +249,7 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, 1),
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": round(value, 4), "unit": "GB/s",
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": round(value, 4), "unit": "GB/s", "cpu": cpu_model(),
                              "sample": f"{per_step} random sequences of {w.spec.name} per step"},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -413,40 +424,79 @@ def main():
                  "p90": round(float(np.percentile(per_launch, 90)), 3), "launches": dist_n,
                  "how": "isolated launches, CUDA events around each, inputs rotating over the copies"}
 
-    # end to end through the public API with pinned host buffers: each step
-    # copies its inputs host -> device (one packed copy), launches, copies the
-    # output back and synchronises on it
-    e2e = None
+    # end to end through the public API with pinned host buffers.  Every step
+    # copies its inputs host -> device (one packed copy), runs the update and
+    # copies its output back; the host receives every step's output.  The
+    # pipelined loop (the headline e2e) overlaps a step's copies with the
+    # neighbouring steps' kernels (the updates stay in order on one stream);
+    # the serial loop synchronises on each step before issuing the next.
+    e2e = e2e_serial = None
     if not args.skip_e2e:
         c0 = copies[0]
         s = w.spec
-        staged = binding.HostStagedDecode(c0["q"].shape[:-2], s.H, s.HV, s.K, s.V, s.N, c0["A_log"], c0["dt_bias"],
-                                          c0["state_pool"], varlen=c0["cu_seqlens"] is not None, flags=flags,
-                                          intermediate_states=c0.get("inter"), stream=stream, tile_v=args.tile_v,
-                                          tile_rows=args.tile_rows, schedule=schedule)
-        for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
-            if c0.get(name) is not None:
-                getattr(staged, name).copy_(c0[name].cpu())
+        staged_args = (c0["q"].shape[:-2], s.H, s.HV, s.K, s.V, s.N, c0["A_log"], c0["dt_bias"], c0["state_pool"])
+        staged_kw = dict(varlen=c0["cu_seqlens"] is not None, flags=flags, intermediate_states=c0.get("inter"),
+                         tile_v=args.tile_v, tile_rows=args.tile_rows, schedule=schedule)
+
+        def fill(slot):
+            for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
+                if c0.get(name) is not None:
+                    getattr(slot, name).copy_(c0[name].cpu())
+
+        def timed(run_steps):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            last_stream = run_steps()
+            e1.record(last_stream)
+            torch.cuda.synchronize(device)
+            te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            return float(te.item()) / args.e2e_steps
+
+        pipe = binding.PipelinedHostDecode(*staged_args, stream=stream, **staged_kw)
+        for slot in pipe.slots:
+            fill(slot)
+        for _ in range(4):
+            pipe.inputs()
+            pipe.step()
+        pipe.finish()
+
+        def run_pipe():
+            for _ in range(args.e2e_steps):
+                pipe.inputs()
+                pipe.step()
+            pipe.finish()
+            return pipe.copy_out
+
+        e2e_ms = timed(run_pipe)
+        e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(pipe.h2d_bytes),
+               "d2h_bytes_per_step": int(pipe.d2h_bytes), "api": "binding.PipelinedHostDecode",
+               "how": "each step: pinned host inputs -> device, update, output -> pinned host; the host "
+                      "receives every step's output; copies overlap the neighbouring steps' kernels"}
+        del pipe
+
+        staged = binding.HostStagedDecode(*staged_args, stream=stream, **staged_kw)
+        fill(staged)
         for _ in range(3):
             staged.step()
             stream.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            staged.step()
-            stream.synchronize()          # the step ends when the host holds the output
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item()) / args.e2e_steps
-        e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
-               "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(staged.h2d_bytes),
-               "d2h_bytes_per_step": int(staged.d2h_bytes), "api": "binding.HostStagedDecode"}
+
+        def run_serial():
+            for _ in range(args.e2e_steps):
+                staged.step()
+                stream.synchronize()      # the step ends when the host holds the output
+            return stream
+
+        es_ms = timed(run_serial)
+        e2e_serial = {"value": round(nbytes * world / (es_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+                      "us_per_call": round(es_ms * 1e3, 3), "api": "binding.HostStagedDecode",
+                      "how": "each step synchronised before the next"}
         del staged
 
     if rank == 0:
@@ -482,6 +532,7 @@ def main():
                          "algorithmic_flops_per_launch": nflops, "hbm_peak_source": peak_src,
                          "kernel": kname},
             "e2e": e2e,
+            "e2e_serial": e2e_serial,
             "gpu_launches": args.steps * (2 if args.unfused or "+" in kname else 1),
             "gpu_launches_note": "launches inside the timed region; the per-launch distribution and e2e run after it",
             "clocks": clocks,

@@ -399,6 +399,73 @@ class HostStagedDecode:
         return self.out_host
 
 
+class PipelinedHostDecode:
+    """Host-fed decode steps with the transfers overlapped across steps.
+
+    Two ``HostStagedDecode`` slots alternate.  Step k copies its inputs in on
+    a copy stream, runs the update on the compute stream (steps stay in
+    order there, so each step sees the previous step's state) and copies its
+    output back on a third stream; meanwhile step k+1's input copy and step
+    k-1's output copy can run beside step k's kernel.  ``inputs()`` returns
+    the host views to fill for the next step (waiting, if needed, until that
+    slot's previous input copy has read them); ``step()`` issues the step and
+    returns the host output of the step before it (waiting for it), or None
+    on the first call; ``finish()`` returns the last step's host output.
+    Constructor arguments are those of ``HostStagedDecode``.
+    """
+
+    def __init__(self, *args, stream: Optional[torch.cuda.Stream] = None, **kw):
+        dev = args[8].device if len(args) > 8 else kw["state_pool"].device
+        self.compute = stream if stream is not None else torch.cuda.Stream(dev)
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.slots = [HostStagedDecode(*args, stream=self.compute, **kw) for _ in range(2)]
+        self._h2d = [torch.cuda.Event() for _ in range(2)]
+        self._ran = [torch.cuda.Event() for _ in range(2)]
+        self._d2h = [torch.cuda.Event() for _ in range(2)]
+        self.h2d_bytes = self.slots[0].h2d_bytes
+        self.d2h_bytes = self.slots[0].d2h_bytes
+        self.k = 0
+
+    def inputs(self) -> "HostStagedDecode":
+        """The slot whose host views (``q``, ``k``, ...) the next step reads."""
+        b = self.k & 1
+        if self.k >= 2:
+            self._h2d[b].synchronize()
+        return self.slots[b]
+
+    def step(self) -> Optional[torch.Tensor]:
+        b = self.k & 1
+        s = self.slots[b]
+        if self.k >= 2:                      # slot b's device inputs were read by step k-2
+            self.copy_in.wait_event(self._ran[b])
+        with torch.cuda.stream(self.copy_in):
+            s.device_buffer.copy_(s.host_buffer, non_blocking=True)
+        self._h2d[b].record(self.copy_in)
+        self.compute.wait_event(self._h2d[b])
+        if self.k >= 2:                      # and its device output was read back by step k-2
+            self.compute.wait_event(self._d2h[b])
+        s._call()
+        self._ran[b].record(self.compute)
+        self.copy_out.wait_event(self._ran[b])
+        with torch.cuda.stream(self.copy_out):
+            s.out_host.copy_(s.out_device, non_blocking=True)
+        self._d2h[b].record(self.copy_out)
+        prev = None
+        if self.k >= 1:
+            self._d2h[b ^ 1].synchronize()
+            prev = self.slots[b ^ 1].out_host
+        self.k += 1
+        return prev
+
+    def finish(self) -> Optional[torch.Tensor]:
+        if self.k == 0:
+            return None
+        b = (self.k - 1) & 1
+        self._d2h[b].synchronize()
+        return self.slots[b].out_host
+
+
 class PreparedUnfusedCall:
     """The unfused pair as one prepared step: the gating kernel writes g and
     beta (fp32, [T_tot, HV], owned here) and the recurrence reads them --

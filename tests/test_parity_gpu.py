@@ -4,6 +4,7 @@ Tolerances, fixed for this path: the fp32 state within max abs 1e-4 of the
 fp64 oracle; the bf16 output within 1e-2 + 1e-2 |o_ref|; slot handling,
 padding, untouched memory and status bits exact.
 """
+import dataclasses
 import numpy as np
 import pytest
 import torch
@@ -384,6 +385,43 @@ def test_host_staged_decode_matches_device_call(spec):
     assert torch.equal(out, ref["out"].cpu())
     assert torch.equal(d["state_pool"], ref["state_pool"])
     assert staged.h2d_bytes >= sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v", "a", "b"))
+
+
+@pytest.mark.parametrize("spec", [wl.TINY, wl.shrink(wl.SPEC_B128_T4, 16), wl.shrink(wl.DECODE_B512, 8)],
+                         ids=lambda s: s.name)
+def test_pipelined_host_decode_matches_device_calls(spec):
+    """Five host-fed steps with different inputs, copies overlapped across
+    steps: every step's host output and the final pool are the bits of the
+    same five steps run as device-resident calls, in order."""
+    ws = [wl.generate(dataclasses.replace(spec, seed=spec.seed + 100 * n)) for n in range(5)]
+    ref = to_device(ws[0])
+    ref_outs = []
+    for w in ws:                                   # same pool and parameters, successive inputs
+        d = to_device(w)
+        binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], ref["A_log"], ref["dt_bias"],
+                              ref["state_pool"], d["state_indices"], d["cu_seqlens"], d["out"])
+        ref_outs.append(d["out"].cpu())
+    torch.cuda.synchronize()
+    d0 = to_device(ws[0])
+    varlen = ws[0].cu_seqlens is not None
+    pipe = binding.PipelinedHostDecode(d0["q"].shape[:-2], spec.H, spec.HV, spec.K, spec.V, spec.N, d0["A_log"],
+                                       d0["dt_bias"], d0["state_pool"], varlen=varlen)
+    outs = []
+    for w in ws:
+        d = to_device(w)
+        slot = pipe.inputs()
+        for name in ("q", "k", "v", "a", "b", "state_indices", "cu_seqlens"):
+            if d.get(name) is not None:
+                getattr(slot, name).copy_(d[name].cpu())
+        prev = pipe.step()
+        if prev is not None:
+            outs.append(prev.clone())
+    outs.append(pipe.finish().clone())
+    torch.cuda.synchronize()
+    assert len(outs) == len(ref_outs)
+    for got, exp in zip(outs, ref_outs):
+        assert torch.equal(got, exp)
+    assert torch.equal(d0["state_pool"], ref["state_pool"])
 
 
 @pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
