@@ -229,6 +229,38 @@ def cpu_baseline_all_cores(w, budget_s=10.0):
                       f"{reps} repetitions, {total_t:.1f} s"}
 
 
+def parity_sample(w, prepare, torch, device, nseq=8):
+    """Part of the cpu_baseline leg: one fresh call of the timed kernel on the
+    workload's original inputs, and the oracle on a sample of its sequences;
+    the largest errors and whether they meet the tolerances (state max abs
+    1e-4, output |o - o_ref| <= 1e-2 + 1e-2 |o_ref|)."""
+    import oracle
+    c = device_copy(w, torch, device)
+    prepare(c)()
+    torch.cuda.synchronize(device)
+    rng = np.random.default_rng(0)
+    seqs = np.sort(rng.choice(w.spec.N, size=min(nseq, w.spec.N), replace=False))
+    args = oracle_subset_args(w, seqs)
+    status, o_ref, s_ref, _ = oracle.update(*args)
+    lens = w.seq_lens
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    rows = np.concatenate([np.arange(starts[i], starts[i] + lens[i]) for i in seqs]).astype(np.int64)
+    s = w.spec
+    o_gpu = c["out"].reshape(w.T_tot, s.HV, s.V)[torch.from_numpy(rows).to(device)].float().cpu().numpy()
+    o_ref = o_ref.reshape(o_gpu.shape)
+    written = ~np.isnan(o_ref)
+    err_o = np.abs(o_gpu.astype(np.float64) - o_ref)[written]
+    ok_o = bool(np.all(err_o <= 1e-2 + 1e-2 * np.abs(o_ref[written])))
+    slots = w.state_indices[seqs]
+    live = slots >= 0
+    s_gpu = c["state_pool"][torch.from_numpy(slots[live].astype(np.int64)).to(device)].cpu().numpy()
+    err_s = float(np.abs(s_gpu.astype(np.float64) - s_ref).max()) if live.any() else 0.0
+    del c
+    return {"sequences": int(len(seqs)), "tokens": int(len(rows)), "oracle_status": int(status),
+            "max_abs_out_err": round(float(err_o.max()) if err_o.size else 0.0, 6),
+            "max_abs_state_err": float(f"{err_s:.3e}"), "within_tolerance": ok_o and err_s <= 1e-4}
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle on bounded per-step samples."""
     N = w.spec.N
@@ -359,20 +391,20 @@ def main():
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
     if args.pdl:
         flags |= binding.LAUNCH_PDL
-    if args.unfused:
-        # the two-kernel baseline the fused update replaces (gating, then the
-        # recurrence reading g and beta back from HBM)
-        calls = [binding.PreparedUnfusedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
-                                             c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"],
-                                             flags=flags, intermediate_states=c.get("inter"), stream=stream,
-                                             tile_v=args.tile_v, tile_rows=args.tile_rows)
-                 for c in copies]
-    else:
-        calls = [binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
-                                      c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
-                                      intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
-                                      schedule=schedule, tile_rows=args.tile_rows)
-                 for c in copies]
+    def prepare(c):
+        if args.unfused:
+            # the two-kernel baseline the fused update replaces (gating, then the
+            # recurrence reading g and beta back from HBM)
+            return binding.PreparedUnfusedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
+                                               c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"],
+                                               flags=flags, intermediate_states=c.get("inter"), stream=stream,
+                                               tile_v=args.tile_v, tile_rows=args.tile_rows)
+        return binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
+                                    c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"], flags=flags,
+                                    intermediate_states=c.get("inter"), stream=stream, tile_v=args.tile_v,
+                                    schedule=schedule, tile_rows=args.tile_rows)
+
+    calls = [prepare(c) for c in copies]
     nbytes = wl.algorithmic_bytes(w)
     torch.cuda.synchronize(device)
 
@@ -391,10 +423,12 @@ def main():
     torch.cuda.synchronize(device)
     sampler = ClockSampler(local_rank)
     time.sleep(0.2)
+    torch.cuda.nvtx.range_push(f"timed region: {args.steps} steps of {w.spec.name}")
     region0.record(stream)
     for s in range(args.steps):
         calls[s % len(calls)]()
     region1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
     if world > 1:
@@ -473,7 +507,9 @@ def main():
             pipe.finish()
             return pipe.copy_out
 
+        torch.cuda.nvtx.range_push("e2e: pipelined host-fed steps")
         e2e_ms = timed(run_pipe)
+        torch.cuda.nvtx.range_pop()
         e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(pipe.h2d_bytes),
                "d2h_bytes_per_step": int(pipe.d2h_bytes), "api": "binding.PipelinedHostDecode",
@@ -493,7 +529,9 @@ def main():
                 stream.synchronize()      # the step ends when the host holds the output
             return stream
 
+        torch.cuda.nvtx.range_push("e2e: serial host-fed steps")
         es_ms = timed(run_serial)
+        torch.cuda.nvtx.range_pop()
         e2e_serial = {"value": round(nbytes * world / (es_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                       "us_per_call": round(es_ms * 1e3, 3), "api": "binding.HostStagedDecode",
                       "how": "each step synchronised before the next"}
@@ -540,6 +578,7 @@ def main():
         if world == 1 and not args.skip_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
             line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w)
+            line["parity"] = parity_sample(w, prepare, torch, device)
         print(json.dumps(line), flush=True)
 
     del calls
