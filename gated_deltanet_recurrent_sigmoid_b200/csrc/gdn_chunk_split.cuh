@@ -15,7 +15,9 @@
 //                           block's W, U^T, P, K'^T = (diag(fd) K)^T and raw Q
 //                           into the workspace as the byte images of the
 //                           operand tiles the second kernel feeds to tcgen05.
-//   gdn_chunk_state_kernel  one 512-thread CTA per (sequence, value head): walks the
+//   gdn_chunk_state_kernel  one 512-thread CTA per (sequence, value head) (or, for
+//                           many short sequences, gdn_chunk_state_compact_kernel:
+//                           256 threads, two CTAs per SM): walks the
 //                           blocks the sequence covers, fetching each block's
 //                           tiles with bulk copies one step ahead, and runs
 //                           only the state-dependent products.
@@ -877,6 +879,324 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     __syncthreads();
     if (warp == 0)
         tc::tmem_dealloc(tmem, ST_TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2, compact form: the same recurrence in 113 KB of shared memory and
+// 256 TMEM columns, so that two CTAs share an SM -- for calls with many
+// (sequence, value head) pairs, where one CTA per SM leaves the state loads
+// and the per-piece latencies exposed.  Differences from the kernel above:
+// one 48 KB record buffer, loaded with W / Q for product 1 and then with
+// K' / P for product 2; the Delta~ tiles overlay the state tiles (dead
+// between the two products); D's TMEM columns take O2 in product 2; outputs
+// are written at the end of their own piece; 256 threads (two per TMEM lane).
+// ---------------------------------------------------------------------------
+struct StSmemCompact {
+    // S~^T hi / lo [v][k]; between product 1 and product 2 the first 32 KB
+    // hold Delta~^T hi / lo [v][i]
+    alignas(1024) unsigned char st[2][128 * 128 * 2];
+    alignas(1024) unsigned char rec[REC_A_BYTES];        // W hi, Q, W lo; then K'^T hi, P hi, K'^T lo, P lo
+    alignas(16) float rec_s[REC_S_BYTES / 4];            // fo, gamma of the piece
+    float fo[C];
+    unsigned long long bar_m, bar_a, bar_b, bar_r;       // products; copies of W / Q, K' / P, fo / gamma
+    uint32_t tmem_base;
+    int failed;
+};
+static_assert(REC_A_BYTES == REC_B_BYTES, "one buffer holds either half of a record");
+
+constexpr int SC_PARTS = 2;
+constexpr int SC_THREADS = 128 * SC_PARTS;
+constexpr uint32_t SC_TMEM_COLS = 256;
+constexpr uint32_t SC_COL_S = 0;      // S~^T                         [v][k]   128 columns
+constexpr uint32_t SC_COL_D = 128;    // -S~^T W^T; O2 in product 2   [v][i]    64
+constexpr uint32_t SC_COL_O1 = 192;   // -S~^T Q^T                    [v][j]    64
+
+__global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(const __grid_constant__ DecodeParams p,
+                                                                               const unsigned char *__restrict__ ws)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    StSmemCompact &sm = *reinterpret_cast<StSmemCompact *>(smem_raw);
+
+    pdl_prologue();
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int v = tid & 127, part = tid >> 7;
+    const int i = blockIdx.x / p.HV;
+    const int hv = blockIdx.x - i * p.HV;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+
+    int64_t bos;
+    int len;
+    if (p.cu_seqlens) {
+        const int b0 = __ldg(p.cu_seqlens + i);
+        const int e0 = __ldg(p.cu_seqlens + i + 1);
+        if (b0 < 0 || e0 < b0 || e0 > p.T_tot) {
+            if (tid == 0 && hv == 0)
+                report(p.status, GDN_DEV_BAD_SEQLENS);
+            return;
+        }
+        bos = b0;
+        len = e0 - b0;
+    } else {
+        bos = static_cast<int64_t>(i) * p.T_fixed;
+        len = p.T_fixed;
+    }
+    const int slot = __ldg(p.indices + i);
+    if (slot < -1 || slot >= p.num_slots) {
+        if (tid == 0 && hv == 0)
+            report(p.status, GDN_DEV_BAD_SLOT);
+        return;
+    }
+    if (slot < 0) {
+        for (int t = part; t < len; t += SC_PARTS)
+            out[(bos + t) * p.o_tok + hv * p.o_head + v] = __float2bfloat16_rn(0.f);
+        return;
+    }
+    if (len == 0)
+        return;
+    const int64_t eos = bos + len;
+    float *const s_gmem = p.state + static_cast<int64_t>(slot) * p.s_slot + hv * p.s_head;
+    auto rec_of = [&](int64_t b) { return ws + (b * p.HV + hv) * static_cast<int64_t>(REC_BYTES); };
+
+    int64_t blk = bos / C;
+    if (tid == 0) {
+        sync::mbar_init(&sm.bar_m, 1);
+        sync::mbar_init(&sm.bar_a, 1);
+        sync::mbar_init(&sm.bar_b, 1);
+        sync::mbar_init(&sm.bar_r, 1);
+        sm.failed = 0;
+        sync::fence_barrier_init();
+        const unsigned char *r = rec_of(blk);
+        sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
+        sync::bulk_load(sm.rec, r, REC_A_BYTES, &sm.bar_a);
+        sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
+        sync::bulk_load(sm.rec_s, r + REC_FO, REC_S_BYTES, &sm.bar_r);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.tmem_base, SC_TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t my_lane = tc::tmem_addr(tmem, (warp & 3) * 32, 0);
+    constexpr int KP = K / SC_PARTS, CP = C / SC_PARTS;
+    const int kh = KP * part, ih = CP * part;
+
+    for (int k0 = kh; k0 < kh + KP; k0 += 16) {
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            x[e] = __ldcs(s_gmem + (k0 + e) * V + v);
+        tc::tmem_st16(my_lane + SC_COL_S + k0, x);
+        st_row8(sm.st[0], v, k0, K, x, false);
+        st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
+        st_row8(sm.st[1], v, k0, K, x, true);
+        st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
+    }
+    tc::tmem_wait_st();
+
+    uint32_t ph_m = 0, ph_a = 0, ph_b = 0, ph_r = 0;
+    // copies issued and not yet waited for, with the parity their wait checks
+    bool ok = true, pend_a = true, pend_b = false, pend_r = true;
+    uint32_t pa = 0, pb = 0, pr = 0;
+    auto wait_bar = [&](unsigned long long *bar, uint32_t &ph) {
+        bool w = ok && sync::mbar_wait(bar, ph, &sm.failed);
+        ph ^= 1u;
+        if (!w && ok) {
+            sm.failed = 1;
+            report(p.status, GDN_DEV_TIMEOUT);
+        }
+        ok = __syncthreads_and(w) != 0;
+        tc::fence_after_sync();
+    };
+    auto publish_smem = [&]() {
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    publish_smem();
+
+    const uint32_t ID_N64_NEG = tc::idesc_bf16_f32(128, 64, true);
+    const uint32_t ID_N128_NEG = tc::idesc_bf16_f32(128, 128, true);
+    const uint32_t ID_N192 = tc::idesc_bf16_f32(128, 192);
+    const unsigned char *wq_hi = sm.rec + REC_W_HI, *w_lo = sm.rec + REC_W_LO;
+    const unsigned char *kpp_hi = sm.rec, *kpp_lo = sm.rec + (REC_KP_LO - REC_KP_HI);
+    unsigned char *const dt_hi = sm.st[0], *const dt_lo = sm.st[0] + 128 * 64 * 2;
+
+    float cs = 1.f;
+    for (int64_t t = bos; t < eos && ok; ++blk) {
+        const int64_t base = blk * C;
+        const int r0 = static_cast<int>(t - base);
+        const int r1 = static_cast<int>((eos < base + C ? eos : base + C) - base);
+        const bool more = base + r1 < eos;
+        const unsigned char *rec = rec_of(blk);
+
+        float u[CP];
+        {
+            const float4 *src = reinterpret_cast<const float4 *>(rec + REC_UT) + v * 16 + ih / 4;
+#pragma unroll
+            for (int m = 0; m < CP / 4; ++m) {
+                const float4 x = __ldg(src + m);
+                u[4 * m] = x.x;
+                u[4 * m + 1] = x.y;
+                u[4 * m + 2] = x.z;
+                u[4 * m + 3] = x.w;
+            }
+        }
+
+        // ---- product 1: [D | O1] = -S~^T [W hi; Q]^T, D -= S~hi^T W lo^T --
+        wait_bar(&sm.bar_a, ph_a);
+        if (!ok)
+            break;
+        pend_a = false;
+        if (tid == 0) {
+            mma_tiles(tmem + SC_COL_D, sm.st[0], K, wq_hi, K, K / 16, ID_N128_NEG, false);
+            mma_tiles(tmem + SC_COL_D, sm.st[1], K, wq_hi, K, K / 16, ID_N128_NEG, true);
+            mma_tiles(tmem + SC_COL_D, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
+            tc::mma_commit(&sm.bar_m);
+        }
+        wait_bar(&sm.bar_m, ph_m);
+        if (!ok)
+            break;
+        if (tid == 0) {               // K' and P of this piece into the buffer just read
+            sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES);
+            sync::bulk_load(sm.rec, rec + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
+        }
+        pend_b = true;
+        pb = ph_b;
+
+        // ---- Delta~^T into its tiles (over the state tiles), D -> 0 --------
+        wait_bar(&sm.bar_r, ph_r);
+        if (!ok)
+            break;
+        pend_r = false;
+        const float decay = expf(sm.rec_s[C + r1 - 1]);
+        const float cn = cs * decay;
+        const bool rescale = !(cn >= 0x1p-60f && cn <= 0x1p60f);
+        const float dscale = rescale ? 1.f : __fdividef(1.f, cn);
+        if (tid < C)
+            sm.fo[tid] = sm.rec_s[tid];
+#pragma unroll
+        for (int cl = 0; cl < CP; cl += 16) {
+            const int cb = ih + cl;
+            float d[16];
+            tc::tmem_ld16(my_lane + SC_COL_D + cb, d);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int ii = cb + e;
+                d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[cl + e]) * dscale : 0.f;
+            }
+            st_row8(dt_hi, v, cb, C, d, false);
+            st_row8(dt_hi, v, cb + 8, C, d + 8, false);
+            st_row8(dt_lo, v, cb, C, d, true);
+            st_row8(dt_lo, v, cb + 8, C, d + 8, true);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                d[e] = 0.f;
+            tc::tmem_st16(my_lane + SC_COL_D + cb, d);          // O2 accumulates from zero here
+        }
+        if (rescale) {
+#pragma unroll 1
+            for (int k0 = kh; k0 < kh + KP; k0 += 16) {
+                float x[16];
+                tc::tmem_ld16(my_lane + SC_COL_S + k0, x);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] *= cn;
+                tc::tmem_st16(my_lane + SC_COL_S + k0, x);
+            }
+        }
+        tc::tmem_wait_st();
+        const float cs_new = rescale ? 1.f : cn;
+        publish_smem();
+
+        // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T ----------------
+        wait_bar(&sm.bar_b, ph_b);
+        if (!ok)
+            break;
+        pend_b = false;
+        if (tid == 0) {
+            mma_tiles(tmem + SC_COL_S, dt_hi, C, kpp_hi, C, C / 16, ID_N192, true);
+            mma_tiles(tmem + SC_COL_S, dt_hi, C, kpp_lo, C, C / 16, ID_N192, true);
+            mma_tiles(tmem + SC_COL_S, dt_lo, C, kpp_hi, C, C / 16, ID_N192, true);
+            tc::mma_commit(&sm.bar_m);
+            if (more) {
+                sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
+                sync::bulk_load(sm.rec_s, rec_of(blk + 1) + REC_FO, REC_S_BYTES, &sm.bar_r);
+            }
+        }
+        pend_r = more;
+        pr = ph_r;
+        wait_bar(&sm.bar_m, ph_m);
+        if (!ok)
+            break;
+        if (more && tid == 0) {       // W and Q of the next piece
+            sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
+            sync::bulk_load(sm.rec, rec_of(blk + 1), REC_A_BYTES, &sm.bar_a);
+        }
+        pend_a = more;
+        pa = ph_a;
+
+        // ---- outputs o_j = fo_j cs (S~0^T q_j) + cs' (Delta~^T P^T)_j --------
+#pragma unroll
+        for (int cl = 0; cl < CP; cl += 16) {
+            const int cb = ih + cl;
+            float o1[16], o2[16];
+            tc::tmem_ld16(my_lane + SC_COL_O1 + cb, o1);
+            tc::tmem_ld16(my_lane + SC_COL_D + cb, o2);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = cb + e;
+                if (j >= r0 && j < r1)
+                    out[(base + j) * p.o_tok + hv * p.o_head + v] =
+                        __float2bfloat16_rn(fmaf(-sm.fo[j] * cs, o1[e], cs_new * o2[e]));
+            }
+        }
+
+        // ---- the next piece's S~^T tiles (over the Delta~ tiles), or the
+        // final write-back ----------------------------------------------------
+        for (int k0 = kh; k0 < kh + KP; k0 += 16) {
+            float x[16];
+            tc::tmem_ld16(my_lane + SC_COL_S + k0, x);
+            tc::tmem_wait_ld();
+            if (more) {
+                st_row8(sm.st[0], v, k0, K, x, false);
+                st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
+                st_row8(sm.st[1], v, k0, K, x, true);
+                st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
+            } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    __stcs(s_gmem + (k0 + e) * V + v, cs_new * x[e]);
+            }
+        }
+        cs = cs_new;
+        t = base + r1;
+        publish_smem();
+    }
+
+    if (pend_a || pend_b || pend_r) {
+        volatile int never = 0;
+        if (pend_a)
+            sync::mbar_wait(&sm.bar_a, pa, &never);
+        if (pend_b)
+            sync::mbar_wait(&sm.bar_b, pb, &never);
+        if (pend_r)
+            sync::mbar_wait(&sm.bar_r, pr, &never);
+    }
+
+    pdl_trigger();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0)
+        tc::tmem_dealloc(tmem, SC_TMEM_COLS);
 }
 
 }  // namespace split

@@ -39,6 +39,14 @@ constexpr int64_t kChunkedFewPairs = 1024;
 // are 0.7-1.0 of the per-tile time; with 64-1024 sequences the ratio is
 // 1.01-1.04 at 24 tokens and 0.89-0.97 at 28).
 int64_t split_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 64 : (pairs < 512 ? 40 : 26); }
+// The split schedule's state kernel in its compact form (two CTAs per SM)
+// from this many (sequence, value head) pairs per SM, for sequences of at
+// most this many tokens on average (measured on B200: 0.89-0.92x the time of
+// the full form on the varlen sweeps of 256-1024 sequences, mean ~33 tokens;
+// 1.06x on 64 sequences of ~480 tokens, where the full form's deeper
+// prefetching wins).
+constexpr int64_t kSplitCompactMinUnitsPerSm = 2;
+constexpr int64_t kSplitCompactMaxMeanTokens = 128;
 
 int64_t elem_size(int32_t dtype)
 {
@@ -253,6 +261,7 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
                          bool pdl, bool l2norm)
 {
     static bool ready[64];
+    static int sm_count[64];
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)
@@ -269,11 +278,20 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem_st));
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sizeof(gdn::split::StSmemCompact)));
         // the largest shared-memory carveout, so that three block-kernel CTAs
-        // fit on an SM
+        // (two compact state-kernel CTAs) fit on an SM
         for (int l2 = 0; l2 < 2 && err == cudaSuccess; ++l2)
             err = cudaFuncSetAttribute(l2 ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
                                        cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
+                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (err == cudaSuccess)
+            err = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess)
             return err;
         ready[dev] = true;
@@ -283,6 +301,13 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
                     dim3(static_cast<unsigned>(blocks)), dim3(gdn::split::THREADS), smem_wy, stream, pdl, p, ws);
     if (err != cudaSuccess)
         return err;
+    // Many (sequence, head) pairs: the compact state kernel (two CTAs per SM);
+    // otherwise the one with more threads and deeper prefetching.
+    if (units >= kSplitCompactMinUnitsPerSm * sm_count[dev] &&
+        static_cast<int64_t>(p.T_tot) <= kSplitCompactMaxMeanTokens * p.N)
+        return launch_ex(gdn::split::gdn_chunk_state_compact_kernel, dim3(static_cast<unsigned>(units)),
+                         dim3(gdn::split::SC_THREADS), sizeof(gdn::split::StSmemCompact), stream, true, p,
+                         static_cast<const unsigned char *>(ws));
     return launch_ex(gdn::split::gdn_chunk_state_kernel, dim3(static_cast<unsigned>(units)),
                      dim3(gdn::split::ST_THREADS), smem_st, stream, true, p,
                      static_cast<const unsigned char *>(ws));

@@ -179,3 +179,18 @@ def test_auto_schedule_picks_chunked_for_long_sequences():
     auto_d, _, auto_i = run_gpu(long_w, inter=True)
     pt_d, _, pt_i = run_gpu(long_w, inter=True, schedule=binding.SCHEDULE_PER_TILE)
     assert _bits_equal(auto_d, pt_d) and torch.equal(auto_i, pt_i)
+
+
+def test_split_compact_many_short_sequences():
+    """Enough short sequences (320 x 8 heads) that the split schedule runs its
+    compact state kernel: empty sequences, padded slots, weak and strong
+    decays, all compared whole with the oracle."""
+    rng = np.random.default_rng(41)
+    lens = [int(x) for x in rng.integers(0, 41, size=320)]
+    lens[5] = 0
+    lens[17] = 64
+    lens[18] = 65
+    w = problem(lens, pad=(3, 77, 200), seed=41)
+    w.A_log = w.A_log.copy()
+    w.A_log[::2] = -9.0
+    check(w, SPLIT)
