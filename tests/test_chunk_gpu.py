@@ -194,3 +194,63 @@ def test_split_compact_many_short_sequences():
     w.A_log = w.A_log.copy()
     w.A_log[::2] = -9.0
     check(w, SPLIT)
+
+
+def _args(d):
+    return (d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"], d["state_pool"], d["state_indices"],
+            d["cu_seqlens"], d["out"])
+
+
+def test_split_graph_capture_and_pdl_chain():
+    """The split schedule (two kernels) captures in a CUDA graph and chains
+    with programmatic dependent launch: two chained calls replayed from a
+    graph, and two chained PDL calls, give the bits of two eager calls."""
+    w = problem([150, 40, 90], seed=51)
+    eager = to_device(w)
+    for _ in range(2):
+        binding.decode_update(*_args(eager), schedule=SPLIT)
+    torch.cuda.synchronize()
+
+    d = to_device(w)
+    pool0 = d["state_pool"].clone()
+    ws = torch.empty(binding.chunked_workspace_bytes(w.T_tot, w.spec.HV), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    call = binding.PreparedCall(*_args(d), stream=stream, schedule=SPLIT, workspace=ws)
+    call()                                   # one-time per-device set-up outside the capture
+    torch.cuda.synchronize()
+    d["state_pool"].copy_(pool0)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        call()
+        call()
+    d["state_pool"].copy_(pool0)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(d["out"], eager["out"]) and torch.equal(d["state_pool"], eager["state_pool"])
+
+    p = to_device(w)
+    for _ in range(2):
+        binding.decode_update(*_args(p), schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
+    torch.cuda.synchronize()
+    assert torch.equal(p["out"], eager["out"]) and torch.equal(p["state_pool"], eager["state_pool"])
+
+
+def test_split_writes_nothing_outside_its_workspace():
+    """Guard bands around the workspace keep their sentinel bytes; the
+    minimal workspace (gdn_chunked_workspace_bytes exactly) is enough."""
+    w = problem([70, 3, 130, 64], seed=52)
+    d = to_device(w)
+    need = binding.chunked_workspace_bytes(w.T_tot, w.spec.HV)
+    guard = 4096
+    buf = torch.full((need + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = buf[guard:guard + need]
+    assert ws.data_ptr() % 256 == 0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.decode_update(*_args(d), schedule=SPLIT, workspace=ws, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert bool((buf[:guard] == 0xA5).all()) and bool((buf[guard + need:] == 0xA5).all())
+    ost, o_ref, s_ref, _ = run_oracle(w)
+    assert_out_close(out_as_f32(d["out"]), o_ref)
