@@ -56,7 +56,6 @@ namespace split {
 
 using chunk::mma_tiles;
 using chunk::st_row8;
-using chunk::transpose8x8;
 
 constexpr int K = 128;
 constexpr int V = 128;
@@ -92,15 +91,15 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
 // Kernel 1: the state-independent products of one (block, value head).
 // ---------------------------------------------------------------------------
 struct WySmem {
-    // 32 KB used in turn by: the raw k rows 0..63 and q rows 64..127 [r][k]
-    // (until the K K^T / Q K^T product); A and T by columns (fp32, 16 KB each,
-    // until the T diag() tiles); the T diag(fw) and T diag(beta) hi / lo
-    // tiles (8 KB each, until the W / U products); W^T staged for the record.
-    // The kernel fits three CTAs per SM (and three 128-column TMEM blocks).
-    alignas(1024) unsigned char r1[128 * 128 * 2];
-    alignas(1024) unsigned char kt[128 * 64 * 2];     // raw k^T [k][i]
-    alignas(1024) unsigned char vt[128 * 64 * 2];     // raw v^T [v][i]
-    float kk[C], qq[C];                                // |k_j|^2, |q_j|^2
+    // raw k rows 0..63 [i][k] (kept until the record's K' is written; also
+    // the MN-major A operand K^T of the W product) and raw q rows 64..127
+    // (until the K K^T / Q K^T product; then A, fp32)
+    alignas(1024) unsigned char kq[128 * 128 * 2];
+    // T by columns (fp32); the q half of kq and r2 (32 KB together) then hold
+    // the T diag(fw) / T diag(beta) hi / lo tiles, then W^T staged for the record
+    alignas(1024) unsigned char r2[64 * 64 * 4];
+    alignas(1024) unsigned char vtile[64 * 128 * 2];  // raw v rows [i][v] (MN-major A operand V^T of the U product)
+    float kk[2][C], qq[2][C];                          // |k_j|^2, |q_j|^2 over each half of the row
     float rk[C], rqs[C], g[C], beta[C], gam[C];
     float fa[C], fw[C], fo[C], fd[C];
     int ss[C], se[C];                                  // segment [ss, se) of row j within the block
@@ -134,9 +133,9 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
     const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
     const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
-    unsigned char *const kq = sm.r1;
-    unsigned char *const tw_hi = sm.r1, *const tw_lo = sm.r1 + 8192;
-    unsigned char *const tu_hi = sm.r1 + 16384, *const tu_lo = sm.r1 + 24576;
+    unsigned char *const kq = sm.kq, *const ktile = sm.kq, *const qhalf = sm.kq + 16384;
+    unsigned char *const tw_hi = qhalf, *const tw_lo = qhalf + 8192;      // over the q half of kq ...
+    unsigned char *const tu_hi = sm.r2, *const tu_lo = sm.r2 + 8192;      // ... and r2 (contiguous)
 
     if (tid == 0) {
         sync::mbar_init(&sm.mbar, 1);
@@ -148,75 +147,46 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         tc::tmem_relinquish();
     }
 
-    // ---- step 1: raw q, k, v of the block into the operand tiles; raw q
-    // also straight into the record; squared norms of k and q -------------
-    // thread (tg, kg): rows 8 tg .. 8 tg + 7, columns 8 kg .. 8 kg + 7
+    // ---- step 1: raw k, q, v rows of the block into the operand tiles
+    // (k and q rows: K-major for the K K^T / Q K^T product; k and v rows also
+    // serve the W and U products as MN-major operands K^T, V^T); raw q also
+    // straight into the record; squared norms of k and q.  Thread (j, half)
+    // handles row j, columns 64 half .. 64 half + 63, so a warp's 16-byte
+    // stores cover 32 consecutive rows (no bank conflicts).
     {
-        const int tg = tid >> 4, kg = tid & 15, col = 8 * kg;
+        const int j = tid & 63, half = tid >> 6;
+        const int64_t tok = t0 + (j < n ? j : 0);
+        const __nv_bfloat16 *kp = k + tok * p.k_tok + h * p.k_head + 64 * half;
+        const __nv_bfloat16 *qp = q + tok * p.q_tok + h * p.q_head + 64 * half;
+        const __nv_bfloat16 *vp = v + tok * p.v_tok + hv * p.v_head + 64 * half;
         uint4 kr[8], qr[8], vr[8];
-        float kk[8], qq[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int j = 8 * tg + r;
-            const int64_t tok = t0 + (j < n ? j : 0);
-            kr[r] = __ldg(reinterpret_cast<const uint4 *>(k + tok * p.k_tok + h * p.k_head + col));
-            qr[r] = __ldg(reinterpret_cast<const uint4 *>(q + tok * p.q_tok + h * p.q_head + col));
-            vr[r] = __ldg(reinterpret_cast<const uint4 *>(v + tok * p.v_tok + hv * p.v_head + col));
+        for (int c = 0; c < 8; ++c) {
+            kr[c] = __ldg(reinterpret_cast<const uint4 *>(kp) + c);
+            qr[c] = __ldg(reinterpret_cast<const uint4 *>(qp) + c);
+            vr[c] = __ldg(reinterpret_cast<const uint4 *>(vp) + c);
         }
+        float kk = 0.f, qq = 0.f;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int j = 8 * tg + r;
+        for (int c = 0; c < 8; ++c) {
             if (j >= n)
-                kr[r] = qr[r] = vr[r] = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(j, col, K)) = kr[r];
-            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(64 + j, col, K)) = qr[r];
-            *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[r];
+                kr[c] = qr[c] = vr[c] = make_uint4(0u, 0u, 0u, 0u);
+            const int col = 64 * half + 8 * c;
+            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(j, col, K)) = kr[c];
+            *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(64 + j, col, K)) = qr[c];
+            *reinterpret_cast<uint4 *>(sm.vtile + tc::kmajor_offset(j, col, K)) = vr[c];
+            *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[c];
             float kf[8], qf[8];
-            unpack8(kr[r], kf);
-            unpack8(qr[r], qf);
-            kk[r] = 0.f;
-            qq[r] = 0.f;
+            unpack8(kr[c], kf);
+            unpack8(qr[c], qf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                kk[r] = fmaf(kf[e], kf[e], kk[r]);
-                qq[r] = fmaf(qf[e], qf[e], qq[r]);
+                kk = fmaf(kf[e], kf[e], kk);
+                qq = fmaf(qf[e], qf[e], qq);
             }
         }
-        uint4 tr[8];
-        transpose8x8(kr, tr);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<uint4 *>(sm.kt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
-        transpose8x8(vr, tr);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<uint4 *>(sm.vt + tc::kmajor_offset(col + e, 8 * tg, C)) = tr[e];
-        // sum the 16 column groups of each row (lanes differing in bits
-        // 0..3) as a reduce-scatter: after halving exchanges with lanes 8, 4,
-        // 2, 1 apart, lane kg holds the total of value kg of the 16 values
-        // (|k|^2 of rows 0..7, then |q|^2 of rows 0..7 of the group)
-        {
-            float val[16];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                val[r] = kk[r];
-                val[8 + r] = qq[r];
-            }
-#pragma unroll
-            for (int half = 8; half >= 1; half >>= 1) {
-                const bool up = (kg & half) != 0;
-#pragma unroll
-                for (int i = 0; i < half; ++i) {
-                    const float send = up ? val[i] : val[half + i];
-                    const float keep = up ? val[half + i] : val[i];
-                    val[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-                }
-            }
-            if (kg < 8)
-                sm.kk[8 * tg + kg] = val[0];
-            else
-                sm.qq[8 * tg + kg - 8] = val[0];
-        }
+        sm.kk[half][j] = kk;
+        sm.qq[half][j] = qq;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -231,8 +201,8 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         float rk = 0.f, rq = 0.f, g = 0.f, be = 0.f;
         if (j < n) {
             const int64_t tok = t0 + j;
-            rk = L2NORM ? rsqrtf(sm.kk[j] + 1e-6f) : 1.f;
-            rq = (L2NORM ? rsqrtf(sm.qq[j] + 1e-6f) : 1.f) * p.scale;
+            rk = L2NORM ? rsqrtf(sm.kk[0][j] + sm.kk[1][j] + 1e-6f) : 1.f;
+            rq = (L2NORM ? rsqrtf(sm.qq[0][j] + sm.qq[1][j] + 1e-6f) : 1.f) * p.scale;
             const float a_t = gate_value(gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32), p.a_f32);
             const float b_t = gate_value(gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32), p.b_f32);
             const float x = a_t + __ldg(p.dt_bias + hv * p.dt_stride);
@@ -327,12 +297,12 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     }
     wait_mma();
 
-    // A stored by columns, At[c][j] = A[j][c], and T by columns with the row
-    // index XOR-swizzled by the column (both fp32 [64][64], in r1: the raw
-    // tiles are consumed)
+    // A stored by columns, At[c][j] = A[j][c] (fp32 [64][64], over the q half
+    // of kq, consumed by the product above), and T by columns with the row
+    // index XOR-swizzled by the column (fp32 [64][64], in r2)
     constexpr int A_LD = 64;
-    float *At = reinterpret_cast<float *>(sm.r1);
-    float *Tcol = reinterpret_cast<float *>(sm.r1 + 16384);
+    float *At = reinterpret_cast<float *>(qhalf);
+    float *Tcol = reinterpret_cast<float *>(sm.r2);
     if (ok) {
         // ---- step 3: A (rows 0..63: warps 0, 1, into At) and P (rows
         // 64..127: warps 2, 3, straight to the record), 16 columns at a time
@@ -440,23 +410,31 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         }
         publish_smem();
 
-        // ---- step 5: W^T = K^T T_w^T and U^T = V^T T_u^T ----------------
+        // ---- step 5: W^T = K^T T_w^T and U^T = V^T T_u^T, with K^T and V^T
+        // read MN-major straight from the raw row tiles (8-row groups of
+        // tokens 2048 bytes apart, 8-column chunks 128 bytes apart) -----------
         if (tid == 0) {
-            mma_tiles(tmem + WY_COL_WT, sm.kt, C, tw_hi, C, C / 16, ID_M128_N64, false);
-            mma_tiles(tmem + WY_COL_WT, sm.kt, C, tw_lo, C, C / 16, ID_M128_N64, true);
-            mma_tiles(tmem + WY_COL_UT, sm.vt, C, tu_hi, C, C / 16, ID_M128_N64, false);
-            mma_tiles(tmem + WY_COL_UT, sm.vt, C, tu_lo, C, C / 16, ID_M128_N64, true);
+            const uint32_t ID_AMN = tc::idesc_bf16_f32(128, 64, false, true);
+            auto mma_amn = [&](uint32_t d, const unsigned char *a, const unsigned char *b, bool acc) {
+                for (uint32_t sl = 0; sl < C / 16; ++sl)
+                    tc::mma_bf16(d, tc::mn_desc(tc::smem_u32(a) + sl * 2u * 2048u, 2048u, 128u),
+                                 tc::kslice_desc(b, C, sl), ID_AMN, (acc || sl > 0) ? 1u : 0u);
+            };
+            mma_amn(tmem + WY_COL_WT, ktile, tw_hi, false);
+            mma_amn(tmem + WY_COL_WT, ktile, tw_lo, true);
+            mma_amn(tmem + WY_COL_UT, sm.vtile, tu_hi, false);
+            mma_amn(tmem + WY_COL_UT, sm.vtile, tu_lo, true);
             tc::mma_commit(&sm.mbar);
         }
         wait_mma();
     }
     if (ok) {
         // ---- step 6: the record's remaining tiles -------------------------
-        // W (thread = k): W^T[k][.] from TMEM into a padded fp32 buffer
-        // [k][64] (column index XOR-swizzled by the row) in r1, free after the
-        // products; the hi / lo chunks of W [i][k] go to the record once it
-        // is complete
-        float *Wpad = reinterpret_cast<float *>(sm.r1);
+        // W (thread = k): W^T[k][.] from TMEM into an fp32 buffer [k][64]
+        // (column index XOR-swizzled by the row) over the q half of kq and r2,
+        // free after the products; the hi / lo chunks of W [i][k] go to the
+        // record once it is complete
+        float *Wpad = reinterpret_cast<float *>(qhalf);
         {
             float wcol[64];
 #pragma unroll
@@ -480,15 +458,17 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
                     dst[(c + e) / 4] = make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
             }
         }
-        // K'^T = (diag(fd) K)^T (thread = k): raw k^T row scaled, hi / lo
+        // K'^T = (diag(fd) K)^T (thread = k): column k of the raw k rows,
+        // scaled, hi / lo
         {
 #pragma unroll
             for (int c = 0; c < 64; c += 8) {
                 float x[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm.kt + tc::kmajor_offset(tid, c, C)), x);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    x[e] *= sm.fd[c + e];
+                    x[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                               ktile + tc::kmajor_offset(c + e, tid, K))) *
+                           sm.fd[c + e];
                 st_row8(rec + REC_KP_HI, tid, c, C, x, false);
                 st_row8(rec + REC_KP_LO, tid, c, C, x, true);
             }

@@ -54,14 +54,28 @@ __device__ __forceinline__ uint64_t kslice_desc(const void *tile, uint32_t cols,
     return smem_desc(smem_u32(tile) + s * 256u, 128u, (cols >> 3) * 128u);
 }
 
+// Descriptor of an operand stored MN-major (16-byte rows of 8 consecutive
+// M / N elements at one K index, 8 such rows per core matrix): `k_stride` is
+// the byte distance between core matrices along K, `mn_stride` along M / N.
+// As for K-major operands, the leading byte offset carries the K-direction
+// stride and the stride byte offset the M / N-direction one (checked by the
+// one-tile probe).
+__device__ __forceinline__ uint64_t mn_desc(uint32_t saddr, uint32_t k_stride, uint32_t mn_stride)
+{
+    return smem_desc(saddr, k_stride, mn_stride);
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, A and B K-major, optional
 // negation of A.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bool negate_a = false)
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bool negate_a = false,
+                                                      bool a_mn_major = false, bool b_mn_major = false)
 {
     return (1u << 4)                           // D format: fp32
            | (1u << 7)                         // A format: bf16
            | (1u << 10)                        // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)      // negate A
+           | ((a_mn_major ? 1u : 0u) << 15)    // A major-ness: 1 = MN-major
+           | ((b_mn_major ? 1u : 0u) << 16)    // B major-ness: 1 = MN-major
            | ((N >> 3) << 17)                  // N / 8
            | ((M >> 4) << 24);                 // M / 16
 }
