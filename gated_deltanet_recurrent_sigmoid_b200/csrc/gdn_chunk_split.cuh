@@ -335,48 +335,135 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         }
         __syncthreads();
 
-        // ---- step 4: T = (I + A)^-1 by columns: warp w solves columns
-        // 16 w .. 16 w + 15, its lanes holding rows lane and lane + 32.  By
-        // elimination: x = e_c; for r = 0 .. 62, x_r' -= A[r'][r] x_r for all
-        // r' (A[r'][r] = 0 unless r' > r, so rows <= r are unchanged and x_r
-        // is final when it is broadcast from its lane).
+        // ---- step 4: T = (I + A)^-1, A strictly lower triangular, by
+        // recursive doubling over 16 x 16 blocks:
+        //   level 1: each warp inverts one diagonal block by substitution;
+        //   level 2: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
+        //   level 3: T_[23][01] = -T_[23][23] (A_[23][01] T_[01][01]) (32 x 32).
+        // The intermediate products sit in the upper triangle of At, whose
+        // entries (A[r][c] = 0 for r < c) are never read: level 2's at column
+        // block 2p + 1, rows of block 2p; level 3's at columns 32.., rows ..31.
+        // Every element of T is written: the diagonal blocks in full (their
+        // upper triangles zero), the upper off-diagonal blocks as zeros.
+        auto T_at = [&](int r, int c) -> float & { return Tcol[c * 64 + (r ^ (c & 31))]; };
         {
-            const int lane = tid & 31, c0 = 16 * warp;
-            float xl[16], xh[16];
+            // level 1: warp w, block b = 16 w; lane (rho, hf) holds row rho of
+            // columns 8 hf .. 8 hf + 7.  For r = 0 .. 14: x_rho -= A[rho][r] x_r
+            // (x_r is final by then; A[rho][r] = 0 unless rho > r)
+            const int lane = tid & 31, rho = lane & 15, hf = lane >> 4, b = 16 * warp;
+            float x[8];
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-                xl[cc] = (lane == c0 + cc) ? 1.f : 0.f;
-                xh[cc] = (lane + 32 == c0 + cc) ? 1.f : 0.f;
-            }
-            // x_r = 0 for r < c0 in all of this warp's columns: start at c0.
-            // Rows r < 32: x_r sits in lane r's xl; rows lane and lane + 32
-            // are updated.
-#pragma unroll 1
-            for (int r = c0; r < 32; ++r) {
-                const float al = At[r * A_LD + lane], ah = At[r * A_LD + 32 + lane];   // A[lane][r], A[lane + 32][r]
+            for (int cc = 0; cc < 8; ++cc)
+                x[cc] = (rho == 8 * hf + cc) ? 1.f : 0.f;
 #pragma unroll
-                for (int cc = 0; cc < 16; ++cc) {
-                    const float xr = __shfl_sync(0xffffffffu, xl[cc], r);
-                    xl[cc] = fmaf(-al, xr, xl[cc]);
-                    xh[cc] = fmaf(-ah, xr, xh[cc]);
-                }
-            }
-            // rows r >= 32: x_r sits in lane r - 32's xh; rows < 32 are final
-#pragma unroll 1
-            for (int r = c0 > 32 ? c0 : 32; r < 63; ++r) {
-                const float ah = At[r * A_LD + 32 + lane];
+            for (int r = 0; r < 15; ++r) {
+                const float a = At[(b + r) * A_LD + b + rho];
 #pragma unroll
-                for (int cc = 0; cc < 16; ++cc) {
-                    const float xr = __shfl_sync(0xffffffffu, xh[cc], r - 32);
-                    xh[cc] = fmaf(-ah, xr, xh[cc]);
-                }
+                for (int cc = 0; cc < 8; ++cc)
+                    x[cc] = fmaf(-a, __shfl_sync(0xffffffffu, x[cc], r + 16 * hf), x[cc]);
             }
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-                const int c = c0 + cc;
-                Tcol[c * 64 + (lane ^ (c & 31))] = xl[cc];
-                Tcol[c * 64 + ((lane + 32) ^ (c & 31))] = xh[cc];
+            for (int cc = 0; cc < 8; ++cc)
+                T_at(b + rho, b + 8 * hf + cc) = x[cc];
+            // zeros: the six 16 x 16 blocks above the diagonal
+            for (int e = tid; e < 6 * 256; e += THREADS) {
+                const int blkid = e >> 8, rb = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
+                const int cb = rb + 1 + blkid - (rb == 0 ? 0 : (rb == 1 ? 3 : 5));
+                T_at(16 * rb + ((e >> 4) & 15), 16 * cb + (e & 15)) = 0.f;
             }
+        }
+        __syncthreads();
+        const int t64 = tid & 63, pr = warp >> 1, C0 = 32 * pr, R1 = C0 + 16;
+        {
+            // level 2, product 1: M1 = A_[R1][C0] T_[C0][C0] (16 x 16) of pair
+            // pr; thread: column j, rows 4 rg .. 4 rg + 3
+            const int j = t64 & 15, rg = t64 >> 4;
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+                const float t = T_at(C0 + kk, C0 + j);
+                const float4 a4 = *reinterpret_cast<const float4 *>(At + (C0 + kk) * A_LD + R1 + 4 * rg);
+                m[0] = fmaf(a4.x, t, m[0]);
+                m[1] = fmaf(a4.y, t, m[1]);
+                m[2] = fmaf(a4.z, t, m[2]);
+                m[3] = fmaf(a4.w, t, m[3]);
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+                At[(R1 + 4 * rg + ii) * A_LD + C0 + j] = m[ii];      // M1[i][j]
+        }
+        __syncthreads();
+        {
+            // level 2, product 2: T_[R1][C0] = -T_[R1][R1] M1; thread: row i,
+            // columns 4 cg .. 4 cg + 3
+            const int i = t64 & 15, cg = t64 >> 4;
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+                const float t = T_at(R1 + i, R1 + kk);
+                const float4 m4 = *reinterpret_cast<const float4 *>(At + (R1 + kk) * A_LD + C0 + 4 * cg);
+                o[0] = fmaf(-t, m4.x, o[0]);
+                o[1] = fmaf(-t, m4.y, o[1]);
+                o[2] = fmaf(-t, m4.z, o[2]);
+                o[3] = fmaf(-t, m4.w, o[3]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                T_at(R1 + i, C0 + 4 * cg + jj) = o[jj];
+        }
+        __syncthreads();
+        {
+            // level 3, product 1: M = A_[23][01] T_[01][01] (32 x 32); thread:
+            // column j = lane, rows 8 w .. 8 w + 7
+            const int j = tid & 31;
+            float m[8];
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii)
+                m[ii] = 0.f;
+#pragma unroll 8
+            for (int kk = 0; kk < 32; ++kk) {
+                const float t = T_at(kk, j);
+                const float4 a0 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 32 + 8 * warp);
+                const float4 a1 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 36 + 8 * warp);
+                m[0] = fmaf(a0.x, t, m[0]);
+                m[1] = fmaf(a0.y, t, m[1]);
+                m[2] = fmaf(a0.z, t, m[2]);
+                m[3] = fmaf(a0.w, t, m[3]);
+                m[4] = fmaf(a1.x, t, m[4]);
+                m[5] = fmaf(a1.y, t, m[5]);
+                m[6] = fmaf(a1.z, t, m[6]);
+                m[7] = fmaf(a1.w, t, m[7]);
+            }
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii)
+                At[(32 + 8 * warp + ii) * A_LD + j] = m[ii];       // M[i][j]
+        }
+        __syncthreads();
+        {
+            // level 3, product 2: T_[23][01] = -T_[23][23] M; thread: row
+            // 32 + i (i = lane), columns 8 w .. 8 w + 7
+            const int i = tid & 31;
+            float o[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                o[jj] = 0.f;
+#pragma unroll 8
+            for (int kk = 0; kk < 32; ++kk) {
+                const float t = T_at(32 + i, 32 + kk);
+                const float4 m0 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 8 * warp);
+                const float4 m1 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 4 + 8 * warp);
+                o[0] = fmaf(-t, m0.x, o[0]);
+                o[1] = fmaf(-t, m0.y, o[1]);
+                o[2] = fmaf(-t, m0.z, o[2]);
+                o[3] = fmaf(-t, m0.w, o[3]);
+                o[4] = fmaf(-t, m1.x, o[4]);
+                o[5] = fmaf(-t, m1.y, o[5]);
+                o[6] = fmaf(-t, m1.z, o[6]);
+                o[7] = fmaf(-t, m1.w, o[7]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                T_at(32 + i, 8 * warp + jj) = o[jj];
         }
         __syncthreads();
 
