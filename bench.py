@@ -229,11 +229,13 @@ def cpu_baseline_all_cores(w, budget_s=10.0):
                       f"{reps} repetitions, {total_t:.1f} s"}
 
 
-def parity_sample(w, prepare, torch, device, nseq=8):
+def parity_sample(w, prepare, torch, device, nseq=8, final_writeback=True):
     """Part of the cpu_baseline leg: one fresh call of the timed kernel on the
     workload's original inputs, and the oracle on a sample of its sequences;
     the largest errors and whether they meet the tolerances (state max abs
-    1e-4, output |o - o_ref| <= 1e-2 + 1e-2 |o_ref|)."""
+    1e-4, output |o - o_ref| <= 1e-2 + 1e-2 |o_ref|).  Without the final
+    write-back the pool slots must be bit-identical to the inputs and the
+    state after each sequence's last token is read from the per-token states."""
     import oracle
     c = device_copy(w, torch, device)
     prepare(c)()
@@ -253,12 +255,24 @@ def parity_sample(w, prepare, torch, device, nseq=8):
     ok_o = bool(np.all(err_o <= 1e-2 + 1e-2 * np.abs(o_ref[written])))
     slots = w.state_indices[seqs]
     live = slots >= 0
-    s_gpu = c["state_pool"][torch.from_numpy(slots[live].astype(np.int64)).to(device)].cpu().numpy()
+    pool_slots = torch.from_numpy(slots[live].astype(np.int64)).to(device)
+    pool_untouched = None
+    if final_writeback:
+        s_gpu = c["state_pool"][pool_slots].cpu().numpy()
+    else:
+        pool_untouched = bool(np.array_equal(c["state_pool"][pool_slots].cpu().numpy(),
+                                             w.state_pool[slots[live]]))
+        last = [starts[i] + lens[i] - 1 for i in seqs[live]]
+        s_gpu = c["inter"][torch.tensor(last, dtype=torch.int64, device=device)].cpu().numpy()
     err_s = float(np.abs(s_gpu.astype(np.float64) - s_ref).max()) if live.any() else 0.0
     del c
-    return {"sequences": int(len(seqs)), "tokens": int(len(rows)), "oracle_status": int(status),
-            "max_abs_out_err": round(float(err_o.max()) if err_o.size else 0.0, 6),
-            "max_abs_state_err": float(f"{err_s:.3e}"), "within_tolerance": ok_o and err_s <= 1e-4}
+    res = {"sequences": int(len(seqs)), "tokens": int(len(rows)), "oracle_status": int(status),
+           "max_abs_out_err": round(float(err_o.max()) if err_o.size else 0.0, 6),
+           "max_abs_state_err": float(f"{err_s:.3e}"),
+           "within_tolerance": ok_o and err_s <= 1e-4 and pool_untouched is not False}
+    if pool_untouched is not None:
+        res["pool_untouched"] = pool_untouched
+    return res
 
 
 def run_reference(args, w):
@@ -353,6 +367,9 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time the two-kernel pair (gating, then the recurrence) instead of the fused update")
+    ap.add_argument("--no-final-writeback", dest="final_writeback", action="store_false",
+                    help="leave the pool untouched (GDN_NO_FINAL_WRITEBACK): the per-token states are the "
+                         "result; requires a workload that writes them")
     ap.add_argument("--no-pdl", dest="pdl", action="store_false",
                     help="launch in plain stream order instead of with programmatic dependent launch")
     args = ap.parse_args()
@@ -361,6 +378,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = wl.generate(wl.BY_NAME[args.workload])
+    if not args.final_writeback and not w.spec.intermediate:
+        ap.error("--no-final-writeback needs a workload that writes the per-token states")
 
     if args.impl == "reference":
         if rank == 0:
@@ -389,6 +408,8 @@ def main():
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
+    if not args.final_writeback:
+        flags |= binding.NO_FINAL_WRITEBACK
     if args.pdl:
         flags |= binding.LAUNCH_PDL
     def prepare(c):
@@ -405,7 +426,7 @@ def main():
                                     schedule=schedule, tile_rows=args.tile_rows)
 
     calls = [prepare(c) for c in copies]
-    nbytes = wl.algorithmic_bytes(w)
+    nbytes = wl.algorithmic_bytes(w, final_writeback=args.final_writeback)
     torch.cuda.synchronize(device)
 
     # warm-up
@@ -554,7 +575,8 @@ def main():
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(w, world, args.pdl),
+            "config": workload_config(w, world, args.pdl) | ({} if args.final_writeback else
+                                                             {"final_writeback": False}),
             "us_per_call": round(avg_kernel_ms * 1e3, 3),
             "launch_us": launch_us,
             "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
@@ -578,7 +600,7 @@ def main():
         if world == 1 and not args.skip_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
             line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w)
-            line["parity"] = parity_sample(w, prepare, torch, device)
+            line["parity"] = parity_sample(w, prepare, torch, device, final_writeback=args.final_writeback)
         print(json.dumps(line), flush=True)
 
     del calls

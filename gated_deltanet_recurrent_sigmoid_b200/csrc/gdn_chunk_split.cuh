@@ -93,12 +93,14 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
 struct WySmem {
     // raw k rows 0..63 [i][k] (kept until the record's K' is written; also
     // the MN-major A operand K^T of the W product) and raw q rows 64..127
-    // (until the K K^T / Q K^T product; then A, fp32)
+    // (until the K K^T / Q K^T product; then A by columns (fp32), then the
+    // T diag(fw) hi / lo tiles and, once the W product is done, the
+    // T diag(beta) ones)
     alignas(1024) unsigned char kq[128 * 128 * 2];
-    // T by columns (fp32); the q half of kq and r2 (32 KB together) then hold
-    // the T diag(fw) / T diag(beta) hi / lo tiles, then W^T staged for the record
-    alignas(1024) unsigned char r2[64 * 64 * 4];
-    alignas(1024) unsigned char vtile[64 * 128 * 2];  // raw v rows [i][v] (MN-major A operand V^T of the U product)
+    // T by columns (fp32), then the raw v rows [i][v] (the MN-major A operand
+    // V^T of the U product); the q half of kq and r2 (32 KB together) then
+    // stage W^T for the record
+    alignas(1024) unsigned char r2[64 * 128 * 2];
     float kk[2][C], qq[2][C];                          // |k_j|^2, |q_j|^2 over each half of the row
     float rk[C], rqs[C], g[C], beta[C], gam[C];
     float fa[C], fw[C], fo[C], fd[C];
@@ -114,7 +116,7 @@ constexpr uint32_t WY_COL_WT = 0;     // W^T        [k][j]   64
 constexpr uint32_t WY_COL_UT = 64;    // U^T        [v][j]   64
 
 template <bool L2NORM>
-__global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_constant__ DecodeParams p,
+__global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_constant__ DecodeParams p,
                                                                 unsigned char *__restrict__ ws)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -133,9 +135,9 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
     const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
     const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
-    unsigned char *const kq = sm.kq, *const ktile = sm.kq, *const qhalf = sm.kq + 16384;
-    unsigned char *const tw_hi = qhalf, *const tw_lo = qhalf + 8192;      // over the q half of kq ...
-    unsigned char *const tu_hi = sm.r2, *const tu_lo = sm.r2 + 8192;      // ... and r2 (contiguous)
+    unsigned char *const kq = sm.kq, *const ktile = sm.kq, *const qhalf = sm.kq + 16384, *const vtile = sm.r2;
+    // the T diag() operand tiles, in turn over the q half of kq
+    unsigned char *const tw_hi = qhalf, *const tw_lo = qhalf + 8192, *const tu_hi = qhalf, *const tu_lo = qhalf + 8192;
 
     if (tid == 0) {
         sync::mbar_init(&sm.mbar, 1);
@@ -147,34 +149,34 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         tc::tmem_relinquish();
     }
 
-    // ---- step 1: raw k, q, v rows of the block into the operand tiles
-    // (k and q rows: K-major for the K K^T / Q K^T product; k and v rows also
-    // serve the W and U products as MN-major operands K^T, V^T); raw q also
-    // straight into the record; squared norms of k and q.  Thread (j, half)
-    // handles row j, columns 64 half .. 64 half + 63, so a warp's 16-byte
-    // stores cover 32 consecutive rows (no bank conflicts).
+    // ---- step 1: raw k and q rows of the block into the operand tile
+    // (K-major for the K K^T / Q K^T product; the k rows also serve the W
+    // product as the MN-major operand K^T); raw q also straight into the
+    // record; squared norms of k and q; the v rows (needed from the U
+    // product on) are only fetched into L2.  Thread (j, half) handles row
+    // j, columns 64 half .. 64 half + 63, so a warp's 16-byte stores cover
+    // 32 consecutive rows (no bank conflicts).
     {
         const int j = tid & 63, half = tid >> 6;
         const int64_t tok = t0 + (j < n ? j : 0);
         const __nv_bfloat16 *kp = k + tok * p.k_tok + h * p.k_head + 64 * half;
         const __nv_bfloat16 *qp = q + tok * p.q_tok + h * p.q_head + 64 * half;
-        const __nv_bfloat16 *vp = v + tok * p.v_tok + hv * p.v_head + 64 * half;
-        uint4 kr[8], qr[8], vr[8];
+        uint4 kr[8], qr[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             kr[c] = __ldg(reinterpret_cast<const uint4 *>(kp) + c);
             qr[c] = __ldg(reinterpret_cast<const uint4 *>(qp) + c);
-            vr[c] = __ldg(reinterpret_cast<const uint4 *>(vp) + c);
         }
+        if (half == 0 && j < n)
+            sync::prefetch_l2(v + tok * p.v_tok + hv * p.v_head, V * 2);
         float kk = 0.f, qq = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             if (j >= n)
-                kr[c] = qr[c] = vr[c] = make_uint4(0u, 0u, 0u, 0u);
+                kr[c] = qr[c] = make_uint4(0u, 0u, 0u, 0u);
             const int col = 64 * half + 8 * c;
             *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(j, col, K)) = kr[c];
             *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(64 + j, col, K)) = qr[c];
-            *reinterpret_cast<uint4 *>(sm.vtile + tc::kmajor_offset(j, col, K)) = vr[c];
             *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[c];
             float kf[8], qf[8];
             unpack8(kr[c], kf);
@@ -289,6 +291,14 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         tc::fence_after_sync();
     };
     const uint32_t ID_M128_N64 = tc::idesc_bf16_f32(128, 64);
+    // D[128 x 64] (+)= A B^T, A read MN-major from a raw [64][128] row tile
+    // (its transpose), B a K-major [64][64] tile
+    auto mma_amn = [&](uint32_t d, const unsigned char *a, const unsigned char *b, bool acc) {
+        const uint32_t ID_AMN = tc::idesc_bf16_f32(128, 64, false, true);
+        for (uint32_t sl = 0; sl < C / 16; ++sl)
+            tc::mma_bf16(d, tc::mn_desc(tc::smem_u32(a) + sl * 2u * 2048u, 2048u, 128u), tc::kslice_desc(b, C, sl),
+                         ID_AMN, (acc || sl > 0) ? 1u : 0u);
+    };
 
     // ---- step 2: [K;Q] K^T ---------------------------------------------------
     if (tid == 0) {
@@ -303,6 +313,7 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     constexpr int A_LD = 64;
     float *At = reinterpret_cast<float *>(qhalf);
     float *Tcol = reinterpret_cast<float *>(sm.r2);
+    float t8[4][8];     // rows of T, kept for the two T diag() tile pairs
     if (ok) {
         // ---- step 3: A (rows 0..63: warps 0, 1, into At) and P (rows
         // 64..127: warps 2, 3, straight to the record), 16 columns at a time
@@ -467,50 +478,66 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         }
         __syncthreads();
 
-        // T diag(fw) and T diag(beta) as hi / lo operand tiles: each thread
-        // takes four 8-column chunks of rows of T (read all, then write over
-        // the area T occupied)
+        // T diag(fw) and T diag(beta) as hi / lo operand tiles, in turn over
+        // the q half of kq: each thread keeps four 8-column chunks of rows of
+        // T in registers (thread: row r = qi & 63, so a warp's reads of T and
+        // its 16-byte tile stores cover 32 consecutive rows)
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            const int qi = tid + 128 * ch, r = qi & 63, c0 = (qi >> 6) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                t8[ch][e] = Tcol[(c0 + e) * 64 + (r ^ ((c0 + e) & 31))];
+        }
+        __syncthreads();
+        // the raw v rows into r2, asynchronously (rows past the end: zeros)
         {
-            float t8[4][8];
+            const int j = tid & 63, half = tid >> 6;
+            const __nv_bfloat16 *vp = v + (t0 + (j < n ? j : 0)) * p.v_tok + hv * p.v_head + 64 * half;
 #pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int q = tid + 128 * n, r = q >> 3, c0 = (q & 7) * 8;
+            for (int c = 0; c < 8; ++c)
+                sync::cp_async16(vtile + tc::kmajor_offset(j, 64 * half + 8 * c, V), vp + 8 * c, j < n ? 16u : 0u);
+            sync::cp_async_commit();
+        }
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    t8[n][e] = Tcol[(c0 + e) * 64 + (r ^ ((c0 + e) & 31))];
-            }
-            __syncthreads();
+        for (int ch = 0; ch < 4; ++ch) {
+            const int qi = tid + 128 * ch, r = qi & 63, c0 = (qi >> 6) * 8;
+            float x8[8];
 #pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int q = tid + 128 * n, r = q >> 3, c0 = (q & 7) * 8;
-                float tw8[8], tu8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    tw8[e] = t8[n][e] * sm.fw[c0 + e];
-                    tu8[e] = t8[n][e] * sm.beta[c0 + e];
-                }
-                st_row8(tw_hi, r, c0, C, tw8, false);
-                st_row8(tw_lo, r, c0, C, tw8, true);
-                st_row8(tu_hi, r, c0, C, tu8, false);
-                st_row8(tu_lo, r, c0, C, tu8, true);
-            }
+            for (int e = 0; e < 8; ++e)
+                x8[e] = t8[ch][e] * sm.fw[c0 + e];
+            st_row8(tw_hi, r, c0, C, x8, false);
+            st_row8(tw_lo, r, c0, C, x8, true);
         }
         publish_smem();
 
-        // ---- step 5: W^T = K^T T_w^T and U^T = V^T T_u^T, with K^T and V^T
+        // ---- step 5: W^T = K^T T_w^T, then U^T = V^T T_u^T, with K^T and V^T
         // read MN-major straight from the raw row tiles (8-row groups of
         // tokens 2048 bytes apart, 8-column chunks 128 bytes apart) -----------
         if (tid == 0) {
-            const uint32_t ID_AMN = tc::idesc_bf16_f32(128, 64, false, true);
-            auto mma_amn = [&](uint32_t d, const unsigned char *a, const unsigned char *b, bool acc) {
-                for (uint32_t sl = 0; sl < C / 16; ++sl)
-                    tc::mma_bf16(d, tc::mn_desc(tc::smem_u32(a) + sl * 2u * 2048u, 2048u, 128u),
-                                 tc::kslice_desc(b, C, sl), ID_AMN, (acc || sl > 0) ? 1u : 0u);
-            };
             mma_amn(tmem + WY_COL_WT, ktile, tw_hi, false);
             mma_amn(tmem + WY_COL_WT, ktile, tw_lo, true);
-            mma_amn(tmem + WY_COL_UT, sm.vtile, tu_hi, false);
-            mma_amn(tmem + WY_COL_UT, sm.vtile, tu_lo, true);
+            tc::mma_commit(&sm.mbar);
+        }
+        wait_mma();
+    }
+    if (ok) {
+        // T diag(beta) over the T diag(fw) tiles, whose product is done
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            const int qi = tid + 128 * ch, r = qi & 63, c0 = (qi >> 6) * 8;
+            float x8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                x8[e] = t8[ch][e] * sm.beta[c0 + e];
+            st_row8(tu_hi, r, c0, C, x8, false);
+            st_row8(tu_lo, r, c0, C, x8, true);
+        }
+        sync::cp_async_wait_all();
+        publish_smem();
+        if (tid == 0) {
+            mma_amn(tmem + WY_COL_UT, vtile, tu_hi, false);
+            mma_amn(tmem + WY_COL_UT, vtile, tu_lo, true);
             tc::mma_commit(&sm.mbar);
         }
         wait_mma();
@@ -518,9 +545,9 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
     if (ok) {
         // ---- step 6: the record's remaining tiles -------------------------
         // W (thread = k): W^T[k][.] from TMEM into an fp32 buffer [k][64]
-        // (column index XOR-swizzled by the row) over the q half of kq and r2,
-        // free after the products; the hi / lo chunks of W [i][k] go to the
-        // record once it is complete
+        // (column index XOR-swizzled by the row) over the q half of kq and r2
+        // (the v rows), free after the products; the hi / lo chunks of W
+        // [i][k] go to the record once it is complete
         float *Wpad = reinterpret_cast<float *>(qhalf);
         {
             float wcol[64];
@@ -574,6 +601,7 @@ __global__ void __launch_bounds__(THREADS) gdn_chunk_wy_kernel(const __grid_cons
         }
     }
 
+    sync::cp_async_wait_all();      // the v rows' copies, on a path that skipped their use
     pdl_trigger();
     tc::fence_before_sync();
     __syncthreads();

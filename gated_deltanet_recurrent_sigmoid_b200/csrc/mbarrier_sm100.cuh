@@ -96,5 +96,23 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // generic-proxy shared-memory writes -> visible to the async proxy (bulk copies)
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Per-thread 16-byte asynchronous copy global -> shared.  Both addresses 16-byte
+// aligned; `src_bytes` (0 or 16) bytes are read and the rest of the 16 zero-filled.
+// Complete with cp_async_wait_all() in the issuing thread (before the CTA exits).
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Hint: bring `bytes` of global memory (16-byte aligned, a multiple of 16) into L2.
+__device__ __forceinline__ void prefetch_l2(const void *gmem_src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
+}
+
 }  // namespace sync
 }  // namespace gdn
