@@ -43,6 +43,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "gdn_chunk_kernel.cuh"
@@ -103,12 +104,17 @@ struct WySmem {
     alignas(1024) unsigned char r2[64 * 128 * 2];
     float kk[2][C], qq[2][C];                          // |k_j|^2, |q_j|^2 over each half of the row
     float rk[C], rqs[C], g[C], beta[C], gam[C];
-    float fa[C], fw[C], fo[C], fd[C];
+    float fw[C], fo[C], fd[C];
+    // base-2 exponents of the A and P factors (see step 3)
+    float ua[C], uq[C], wc[C];
     int ss[C], se[C];                                  // segment [ss, se) of row j within the block
     unsigned long long mbar;
     uint32_t tmem_base;
     int failed;
 };
+
+static_assert(offsetof(WySmem, g) % 16 == 0 && offsetof(WySmem, ua) % 16 == 0 && offsetof(WySmem, wc) % 16 == 0,
+              "g, ua and wc are read as 16-byte vectors");
 
 constexpr uint32_t WY_TMEM_COLS = 128;
 constexpr uint32_t WY_COL_KQ = 0;     // [K;Q] K^T  [r][i]   64 columns (read before the W / U products)
@@ -149,6 +155,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
         tc::tmem_relinquish();
     }
 
+    uint32_t a_raw = 0, b_raw = 0;      // raw gates of row tid (threads 0..63)
     // ---- step 1: raw k and q rows of the block into the operand tile
     // (K-major for the K K^T / Q K^T product; the k rows also serve the W
     // product as the MN-major operand K^T); raw q also straight into the
@@ -167,8 +174,45 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
             kr[c] = __ldg(reinterpret_cast<const uint4 *>(kp) + c);
             qr[c] = __ldg(reinterpret_cast<const uint4 *>(qp) + c);
         }
-        if (half == 0 && j < n)
-            sync::prefetch_l2(v + tok * p.v_tok + hv * p.v_head, V * 2);
+        if (half == 0) {
+            // row j's gates (used after the barrier) and its v row into L2
+            if (j < n) {
+                sync::prefetch_l2(v + tok * p.v_tok + hv * p.v_head, V * 2);
+                a_raw = gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32);
+                b_raw = gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32);
+            }
+        } else {
+            // segment [ss, se) of row j within the block (rows past the end:
+            // a segment of their own), while the loads above are in flight
+            int ss = j, se = j + 1;
+            if (j < n) {
+                int64_t s_beg, s_end;
+                if (p.cu_seqlens) {
+                    // the last sequence starting at or before tok (binary search
+                    // over cu_seqlens[0..N]; kept in bounds even if it is invalid)
+                    int lo = 0, hi = p.N;            // cu[lo] <= tok < cu[hi] when valid
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (__ldg(p.cu_seqlens + mid) <= tok)
+                            lo = mid;
+                        else
+                            hi = mid;
+                    }
+                    s_beg = __ldg(p.cu_seqlens + lo);
+                    s_end = __ldg(p.cu_seqlens + lo + 1);
+                } else {
+                    const int64_t s = tok / p.T_fixed;
+                    s_beg = s * p.T_fixed;
+                    s_end = s_beg + p.T_fixed;
+                }
+                if (s_beg <= tok && tok < s_end) {
+                    ss = static_cast<int>((s_beg > t0 ? s_beg : t0) - t0);
+                    se = static_cast<int>((s_end < t0 + n ? s_end : t0 + n) - t0);
+                }
+            }
+            sm.ss[j] = ss;
+            sm.se[j] = se;
+        }
         float kk = 0.f, qq = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -196,17 +240,14 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     const uint32_t tmem = sm.tmem_base;
     const uint32_t my_lane = tc::tmem_addr(tmem, warp * 32, 0);
 
-    // ---- per-row scalars: gates and norms (threads 0..63), segment of the
-    // row (threads 64..127) -------------------------------------------------
+    // ---- per-row scalars: gates and norms (threads 0..63) ----------------
     if (tid < C) {
         const int j = tid;
         float rk = 0.f, rq = 0.f, g = 0.f, be = 0.f;
         if (j < n) {
-            const int64_t tok = t0 + j;
             rk = L2NORM ? rsqrtf(sm.kk[0][j] + sm.kk[1][j] + 1e-6f) : 1.f;
             rq = (L2NORM ? rsqrtf(sm.qq[0][j] + sm.qq[1][j] + 1e-6f) : 1.f) * p.scale;
-            const float a_t = gate_value(gate_raw(p.a, tok * p.a_tok + hv * p.a_head, p.a_f32), p.a_f32);
-            const float b_t = gate_value(gate_raw(p.b, tok * p.b_tok + hv * p.b_head, p.b_f32), p.b_f32);
+            const float a_t = gate_value(a_raw, p.a_f32), b_t = gate_value(b_raw, p.b_f32);
             const float x = a_t + __ldg(p.dt_bias + hv * p.dt_stride);
             g = -expf(__ldg(p.A_log + hv * p.A_stride)) * (x > 20.f ? x : log1pf(expf(x)));
             be = 1.f / (1.f + expf(-b_t));
@@ -215,55 +256,40 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
         sm.rqs[j] = rq;
         sm.g[j] = g;
         sm.beta[j] = be;
-    } else {
-        const int j = tid - C;
-        int ss = j, se = j + 1;      // rows past the end: a segment of their own
-        if (j < n) {
-            const int64_t tok = t0 + j;
-            int64_t s_beg, s_end;
-            if (p.cu_seqlens) {
-                // the last sequence starting at or before tok (binary search
-                // over cu_seqlens[0..N]; kept in bounds even if it is invalid)
-                int lo = 0, hi = p.N;            // cu[lo] <= tok < cu[hi] when valid
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (__ldg(p.cu_seqlens + mid) <= tok)
-                        lo = mid;
-                    else
-                        hi = mid;
-                }
-                s_beg = __ldg(p.cu_seqlens + lo);
-                s_end = __ldg(p.cu_seqlens + lo + 1);
-            } else {
-                const int64_t s = tok / p.T_fixed;
-                s_beg = s * p.T_fixed;
-                s_end = s_beg + p.T_fixed;
-            }
-            if (s_beg <= tok && tok < s_end) {
-                ss = static_cast<int>((s_beg > t0 ? s_beg : t0) - t0);
-                se = static_cast<int>((s_end < t0 + n ? s_end : t0 + n) - t0);
-            }
-        }
-        sm.ss[j] = ss;
-        sm.se[j] = se;
     }
     __syncthreads();
     if (tid < C) {
-        // gamma_j: running sum of g over the row's segment
-        const int j = tid;
+        // gamma_j: running sum of g over the row's segment, in index order
+        // (the masked-out terms add exact zeros); the 16-byte reads of g are
+        // the same for every thread
+        const int j = tid, s0 = sm.ss[j];
         float acc = 0.f;
-        for (int i = sm.ss[j]; i <= j; ++i)
-            acc += sm.g[i];
+#pragma unroll
+        for (int q4 = 0; q4 < C / 4; ++q4) {
+            const float4 g4 = reinterpret_cast<const float4 *>(sm.g)[q4];
+            const int i = 4 * q4;
+            acc += (i >= s0 && i <= j) ? g4.x : 0.f;
+            acc += (i + 1 >= s0 && i + 1 <= j) ? g4.y : 0.f;
+            acc += (i + 2 >= s0 && i + 2 <= j) ? g4.z : 0.f;
+            acc += (i + 3 >= s0 && i + 3 <= j) ? g4.w : 0.f;
+        }
         sm.gam[j] = acc;
     }
     __syncthreads();
     if (tid < C) {
         const int j = tid;
         const float gj = sm.gam[j], gl = sm.gam[sm.se[j] - 1];
-        sm.fa[j] = sm.beta[j] * sm.rk[j];
         sm.fw[j] = sm.beta[j] * expf(gj) * sm.rk[j];
         sm.fo[j] = expf(gj) * sm.rqs[j];
         sm.fd[j] = expf(gl - gj) * sm.rk[j];
+        // A[j][c] = beta_j rk_j rk_c e^(gamma_j - gamma_c) (K K^T)[j][c] and
+        // P[j][i] = rqs_j rk_i e^(gamma_j - gamma_i) (Q K^T)[j][i] as one power
+        // of two each: 2^(ua_j - wc_c), 2^(uq_j - wc_i).  A zero factor (beta = 0,
+        // or a row past the end) gives an exponent of -inf, hence an exact 0.
+        const float g2 = gj * 1.4426950408889634f;
+        sm.ua[j] = g2 + log2f(sm.beta[j] * sm.rk[j]);
+        sm.uq[j] = g2 + log2f(sm.rqs[j]);
+        sm.wc[j] = g2 - log2f(sm.rk[j]);
         reinterpret_cast<float *>(rec + REC_FO)[j] = sm.fo[j];
         reinterpret_cast<float *>(rec + REC_GAM)[j] = gj;
     }
@@ -315,73 +341,96 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     float *Tcol = reinterpret_cast<float *>(sm.r2);
     float t8[4][8];     // rows of T, kept for the two T diag() tile pairs
     if (ok) {
-        // ---- step 3: A (rows 0..63: warps 0, 1, into At) and P (rows
-        // 64..127: warps 2, 3, straight to the record), 16 columns at a time
-        {
-            const int j = tid & 63, sj = sm.ss[j];
-            const float fj = tid < 64 ? sm.fa[j] : sm.rqs[j], gj = sm.gam[j];
+        // ---- step 3: A by columns (warps 0, 1, into At) and P by rows (warps
+        // 2, 3, straight to the record), 16 TMEM columns at a time.  K K^T is
+        // symmetric, so TMEM lane c (row c) holds column c of it: thread c
+        // writes column c of A as contiguous 16-byte vectors.  A[j][c] is
+        // nonzero for c < j in the same segment, i.e. c < j < se_c; P[j][i] for
+        // ss_j <= i <= j.
+        if (tid < 64) {
+            const int c = tid, ce = sm.se[c];
+            const float w = sm.wc[c];
+#pragma unroll 1
+            for (int jb = 0; jb < 64; jb += 16) {
+                float kk16[16];
+                tc::tmem_ld16(my_lane + WY_COL_KQ + jb, kk16);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int j0 = jb + 4 * e4;
+                    const float4 u4 = *reinterpret_cast<const float4 *>(sm.ua + j0);
+                    float4 a4;
+                    a4.x = (j0 > c && j0 < ce) ? kk16[4 * e4] * exp2f(u4.x - w) : 0.f;
+                    a4.y = (j0 + 1 > c && j0 + 1 < ce) ? kk16[4 * e4 + 1] * exp2f(u4.y - w) : 0.f;
+                    a4.z = (j0 + 2 > c && j0 + 2 < ce) ? kk16[4 * e4 + 2] * exp2f(u4.z - w) : 0.f;
+                    a4.w = (j0 + 3 > c && j0 + 3 < ce) ? kk16[4 * e4 + 3] * exp2f(u4.w - w) : 0.f;
+                    *reinterpret_cast<float4 *>(At + c * A_LD + j0) = a4;
+                }
+            }
+        } else {
+            const int j = tid - 64, sj = sm.ss[j];
+            const float u = sm.uq[j];
 #pragma unroll 1
             for (int cb = 0; cb < 64; cb += 16) {
                 float row[16];
                 tc::tmem_ld16(my_lane + WY_COL_KQ + cb, row);
                 tc::tmem_wait_ld();
-                if (tid < 64) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c = cb + e;
-                        At[c * A_LD + j] = (c < j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[e] : 0.f;
-                    }
-                } else {
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 w4 = *reinterpret_cast<const float4 *>(sm.wc + cb + 4 * e4);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c = cb + e;
-                        row[e] = (c <= j && c >= sj) ? fj * sm.rk[c] * expf(gj - sm.gam[c]) * row[e] : 0.f;
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = cb + 4 * e4 + e;
+                        row[4 * e4 + e] = (i <= j && i >= sj) ? row[4 * e4 + e] * exp2f(u - wv[e]) : 0.f;
                     }
-                    st_row8(rec + REC_P_HI, j, cb, C, row, false);
-                    st_row8(rec + REC_P_HI, j, cb + 8, C, row + 8, false);
-                    st_row8(rec + REC_P_LO, j, cb, C, row, true);
-                    st_row8(rec + REC_P_LO, j, cb + 8, C, row + 8, true);
                 }
+                st_row8(rec + REC_P_HI, j, cb, C, row, false);
+                st_row8(rec + REC_P_HI, j, cb + 8, C, row + 8, false);
+                st_row8(rec + REC_P_LO, j, cb, C, row, true);
+                st_row8(rec + REC_P_LO, j, cb + 8, C, row + 8, true);
             }
         }
         __syncthreads();
 
         // ---- step 4: T = (I + A)^-1, A strictly lower triangular, by
         // recursive doubling over 16 x 16 blocks:
-        //   level 1: each warp inverts one diagonal block by substitution;
+        //   level 1: the diagonal blocks by substitution, a thread per column;
         //   level 2: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
         //   level 3: T_[23][01] = -T_[23][23] (A_[23][01] T_[01][01]) (32 x 32).
         // The intermediate products sit in the upper triangle of At, whose
         // entries (A[r][c] = 0 for r < c) are never read: level 2's at column
         // block 2p + 1, rows of block 2p; level 3's at columns 32.., rows ..31.
-        // Every element of T is written: the diagonal blocks in full (their
-        // upper triangles zero), the upper off-diagonal blocks as zeros.
+        // The diagonal blocks are written in full (their upper triangles
+        // zero); the blocks above them are never written, and every read that
+        // can reach one selects zero instead.
         auto T_at = [&](int r, int c) -> float & { return Tcol[c * 64 + (r ^ (c & 31))]; };
-        {
-            // level 1: warp w, block b = 16 w; lane (rho, hf) holds row rho of
-            // columns 8 hf .. 8 hf + 7.  For r = 0 .. 14: x_rho -= A[rho][r] x_r
-            // (x_r is final by then; A[rho][r] = 0 unless rho > r)
-            const int lane = tid & 31, rho = lane & 15, hf = lane >> 4, b = 16 * warp;
-            float x[8];
+        if (tid < 64) {
+            // level 1: thread (bw, cl) takes column cl of diagonal block bw
+            // (rows b .. b + 15, b = 16 bw), all 16 rows in registers: x = e_cl;
+            // for r = 0 .. 14, x_rho -= A[rho][r] x_r for every rho (A[rho][r] = 0
+            // unless rho > r; x_r is final once the steps before r are done).
+            // Column r of the block is read as the 16-byte groups holding rows
+            // > r; no lane exchanges, so the only dependent chain is the FMAs.
+            const int b = 16 * (tid >> 4), cl = tid & 15;
+            float x[16];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                x[cc] = (rho == 8 * hf + cc) ? 1.f : 0.f;
+            for (int rho = 0; rho < 16; ++rho)
+                x[rho] = (rho == cl) ? 1.f : 0.f;
 #pragma unroll
             for (int r = 0; r < 15; ++r) {
-                const float a = At[(b + r) * A_LD + b + rho];
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    x[cc] = fmaf(-a, __shfl_sync(0xffffffffu, x[cc], r + 16 * hf), x[cc]);
+                for (int g = (r + 1) >> 2; g < 4; ++g) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(At + (b + r) * A_LD + b + 4 * g);
+                    x[4 * g] = fmaf(-a4.x, x[r], x[4 * g]);
+                    x[4 * g + 1] = fmaf(-a4.y, x[r], x[4 * g + 1]);
+                    x[4 * g + 2] = fmaf(-a4.z, x[r], x[4 * g + 2]);
+                    x[4 * g + 3] = fmaf(-a4.w, x[r], x[4 * g + 3]);
+                }
             }
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                T_at(b + rho, b + 8 * hf + cc) = x[cc];
-            // zeros: the six 16 x 16 blocks above the diagonal
-            for (int e = tid; e < 6 * 256; e += THREADS) {
-                const int blkid = e >> 8, rb = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
-                const int cb = rb + 1 + blkid - (rb == 0 ? 0 : (rb == 1 ? 3 : 5));
-                T_at(16 * rb + ((e >> 4) & 15), 16 * cb + (e & 15)) = 0.f;
-            }
+            for (int rho = 0; rho < 16; ++rho)
+                T_at(b + rho, b + cl) = x[rho];
         }
         __syncthreads();
         const int t64 = tid & 63, pr = warp >> 1, C0 = 32 * pr, R1 = C0 + 16;
@@ -433,7 +482,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                 m[ii] = 0.f;
 #pragma unroll 8
             for (int kk = 0; kk < 32; ++kk) {
-                const float t = T_at(kk, j);
+                const float t = kk >= j ? T_at(kk, j) : 0.f;
                 const float4 a0 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 32 + 8 * warp);
                 const float4 a1 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 36 + 8 * warp);
                 m[0] = fmaf(a0.x, t, m[0]);
@@ -460,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                 o[jj] = 0.f;
 #pragma unroll 8
             for (int kk = 0; kk < 32; ++kk) {
-                const float t = T_at(32 + i, 32 + kk);
+                const float t = kk <= i ? T_at(32 + i, 32 + kk) : 0.f;
                 const float4 m0 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 8 * warp);
                 const float4 m1 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 4 + 8 * warp);
                 o[0] = fmaf(-t, m0.x, o[0]);
@@ -487,7 +536,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
             const int qi = tid + 128 * ch, r = qi & 63, c0 = (qi >> 6) * 8;
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                t8[ch][e] = Tcol[(c0 + e) * 64 + (r ^ ((c0 + e) & 31))];
+                t8[ch][e] = c0 + e <= r ? Tcol[(c0 + e) * 64 + (r ^ ((c0 + e) & 31))] : 0.f;
         }
         __syncthreads();
         // the raw v rows into r2, asynchronously (rows past the end: zeros)

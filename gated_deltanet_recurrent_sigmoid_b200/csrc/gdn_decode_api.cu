@@ -282,7 +282,7 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
             err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sizeof(gdn::split::StSmemCompact)));
-        // the largest shared-memory carveout, so that three block-kernel CTAs
+        // the largest shared-memory carveout, so that four block-kernel CTAs
         // (two compact state-kernel CTAs) fit on an SM
         for (int l2 = 0; l2 < 2 && err == cudaSuccess; ++l2)
             err = cudaFuncSetAttribute(l2 ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
