@@ -58,29 +58,42 @@ namespace split {
 using chunk::mma_tiles;
 using chunk::st_row8;
 
+// D (+)= A B^T with A a K-major [128][a_cols] tile (k-slices of 16 columns)
+// and B stored as the [kdim][b_cols] row tile of B^T, read MN-major: core
+// matrices 128 bytes apart along N (= b_cols), (b_cols / 8) * 128 bytes apart
+// along the contraction.
+__device__ __forceinline__ void mma_tiles_bmn(uint32_t d, const unsigned char *a, uint32_t a_cols,
+                                              const unsigned char *b, uint32_t b_cols, uint32_t slices,
+                                              uint32_t idesc, bool accumulate)
+{
+    const uint32_t kstride = (b_cols >> 3) * 128u;
+    for (uint32_t s = 0; s < slices; ++s)
+        tc::mma_bf16(d, tc::kslice_desc(a, a_cols, s), tc::mn_desc(tc::smem_u32(b) + s * 2u * kstride, kstride, 128u),
+                     idesc, (accumulate || s > 0) ? 1u : 0u);
+}
+
 constexpr int K = 128;
 constexpr int V = 128;
 constexpr int C = 64;            // tokens per block
 constexpr int THREADS = 128;
 
 // One workspace record per (block, value head): byte offsets.  Tiles are in
-// the K-major core-matrix layout of tc_sm100.cuh; [r][c] names the rows and
-// the contraction dimension.
-// W hi and Q are adjacent so that [W hi; Q] is one 128-row operand, and so
-// are [K'^T hi; P hi] and [K'^T lo; P lo] (192 rows each).
-constexpr uint32_t REC_W_HI = 0;          // W hi              [i][k]   16 KB
-constexpr uint32_t REC_Q = 16384;         // raw q             [j][k]   16 KB
-constexpr uint32_t REC_W_LO = 32768;      // W lo              [i][k]   16 KB
-constexpr uint32_t REC_KP_HI = 49152;     // K'^T hi           [k][i]   16 KB
-constexpr uint32_t REC_P_HI = 65536;      // P hi              [j][i]    8 KB
-constexpr uint32_t REC_KP_LO = 73728;     // K'^T lo           [k][i]   16 KB
-constexpr uint32_t REC_P_LO = 90112;      // P lo              [j][i]    8 KB
+// the core-matrix layout of tc_sm100.cuh (tc::kmajor_offset) for [r][c]: 16-byte
+// rows of 8 consecutive c, r being the contraction index of the product that
+// reads them; they are read as MN-major operands, [W^T hi | Q^T] as one
+// 128-wide operand and [K' | P^T] as one 192-wide operand.
+constexpr uint32_t REC_WQ_HI = 0;         // [W^T hi | Q^T]    [k][i | j]    32 KB
+constexpr uint32_t REC_W_LO = 32768;      // W^T lo            [k][i]        16 KB
+constexpr uint32_t WQ_COLS = C + C;       // 128
+constexpr uint32_t REC_KP_HI = 49152;     // [K' | P^T] hi     [i][k | j]    24 KB
+constexpr uint32_t REC_KP_LO = 73728;     // [K' | P^T] lo     [i][k | j]    24 KB
+constexpr uint32_t KP_COLS = K + C;       // 192
 constexpr uint32_t REC_UT = 98304;        // U^T fp32, row-major [v][i]  32 KB
 constexpr uint32_t REC_FO = 131072;       // fo_j = e^gamma_j rqs_j     256 B
 constexpr uint32_t REC_GAM = 131328;      // gamma_j                    256 B
 constexpr uint32_t REC_BYTES = 131584;    // a multiple of 256
-constexpr uint32_t REC_A_BYTES = REC_KP_HI;               // W hi, Q, W lo
-constexpr uint32_t REC_B_BYTES = REC_UT - REC_KP_HI;      // K'^T hi, P hi, K'^T lo, P lo
+constexpr uint32_t REC_A_BYTES = REC_KP_HI;               // [W^T hi | Q^T], W^T lo
+constexpr uint32_t REC_B_BYTES = REC_UT - REC_KP_HI;      // [K' | P^T] hi, lo
 constexpr uint32_t REC_S_BYTES = REC_BYTES - REC_FO;      // fo, gamma
 
 __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV)
@@ -99,8 +112,7 @@ struct WySmem {
     // T diag(beta) ones)
     alignas(1024) unsigned char kq[128 * 128 * 2];
     // T by columns (fp32), then the raw v rows [i][v] (the MN-major A operand
-    // V^T of the U product); the q half of kq and r2 (32 KB together) then
-    // stage W^T for the record
+    // V^T of the U product)
     alignas(1024) unsigned char r2[64 * 128 * 2];
     float kk[2][C], qq[2][C];                          // |k_j|^2, |q_j|^2 over each half of the row
     float rk[C], rqs[C], g[C], beta[C], gam[C];
@@ -117,7 +129,7 @@ static_assert(offsetof(WySmem, g) % 16 == 0 && offsetof(WySmem, ua) % 16 == 0 &&
               "g, ua and wc are read as 16-byte vectors");
 
 constexpr uint32_t WY_TMEM_COLS = 128;
-constexpr uint32_t WY_COL_KQ = 0;     // [K;Q] K^T  [r][i]   64 columns (read before the W / U products)
+constexpr uint32_t WY_COL_KQ = 0;     // K [K;Q]^T  [i][c | j] 128 columns (read before the W / U products)
 constexpr uint32_t WY_COL_WT = 0;     // W^T        [k][j]   64
 constexpr uint32_t WY_COL_UT = 64;    // U^T        [v][j]   64
 
@@ -221,7 +233,6 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
             const int col = 64 * half + 8 * c;
             *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(j, col, K)) = kr[c];
             *reinterpret_cast<uint4 *>(kq + tc::kmajor_offset(64 + j, col, K)) = qr[c];
-            *reinterpret_cast<uint4 *>(rec + REC_Q + tc::kmajor_offset(j, col, K)) = qr[c];
             float kf[8], qf[8];
             unpack8(kr[c], kf);
             unpack8(qr[c], qf);
@@ -240,7 +251,34 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     const uint32_t tmem = sm.tmem_base;
     const uint32_t my_lane = tc::tmem_addr(tmem, warp * 32, 0);
 
+    // Q^T into the record (columns 64.. of [W^T hi | Q^T]) by warps 2 and 3
+    // while warps 0 and 1 compute the per-row scalars: each 8 x 8 block (rows
+    // 8 jg.., columns 8 kg..) of the q rows is one core matrix of the row tile,
+    // loaded transposed with ldmatrix; lane t then holds Q^T[8 kg + t/4][8 jg +
+    // 2 (t%4) + {0, 1}], and a warp's 4-byte stores fill the block's 128 bytes.
+    auto q_transposed = [&](int it0, int it1) {
+        const int lane = tid & 31;
+        for (int it = it0; it < it1; ++it) {
+            const int mb = ((warp - 2) * 16 + it) * 4;          // 4 blocks per load
+            const int mr = mb + (lane >> 3);
+            const uint32_t src = tc::smem_u32(qhalf + tc::kmajor_offset(8 * (mr & 7) + (lane & 7), 8 * (mr >> 3), K));
+            uint32_t d[4];
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                         : "r"(src));
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int m = mb + x;
+                *reinterpret_cast<uint32_t *>(rec + REC_WQ_HI +
+                                              tc::kmajor_offset(8 * (m >> 3) + (lane >> 2), C + 8 * (m & 7) + 2 * (lane & 3),
+                                                                WQ_COLS)) = d[x];
+            }
+        }
+    };
+
     // ---- per-row scalars: gates and norms (threads 0..63) ----------------
+    if (tid >= C)
+        q_transposed(0, 8);
     if (tid < C) {
         const int j = tid;
         float rk = 0.f, rq = 0.f, g = 0.f, be = 0.f;
@@ -258,6 +296,8 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
         sm.beta[j] = be;
     }
     __syncthreads();
+    if (tid >= C)
+        q_transposed(8, 16);
     if (tid < C) {
         // gamma_j: running sum of g over the row's segment, in index order
         // (the masked-out terms add exact zeros); the 16-byte reads of g are
@@ -316,7 +356,6 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
         __syncthreads();
         tc::fence_after_sync();
     };
-    const uint32_t ID_M128_N64 = tc::idesc_bf16_f32(128, 64);
     // D[128 x 64] (+)= A B^T, A read MN-major from a raw [64][128] row tile
     // (its transpose), B a K-major [64][64] tile
     auto mma_amn = [&](uint32_t d, const unsigned char *a, const unsigned char *b, bool acc) {
@@ -326,9 +365,10 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                          ID_AMN, (acc || sl > 0) ? 1u : 0u);
     };
 
-    // ---- step 2: [K;Q] K^T ---------------------------------------------------
+    // ---- step 2: [K;Q] [K;Q]^T, of which lanes 0..63 (the k rows) are used:
+    // K K^T in columns 0..63, K Q^T in 64..127 -------------------------------
     if (tid == 0) {
-        mma_tiles(tmem + WY_COL_KQ, kq, K, kq, K, K / 16, ID_M128_N64, false);
+        mma_tiles(tmem + WY_COL_KQ, kq, K, kq, K, K / 16, tc::idesc_bf16_f32(128, 128), false);
         tc::mma_commit(&sm.mbar);
     }
     wait_mma();
@@ -341,12 +381,12 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     float *Tcol = reinterpret_cast<float *>(sm.r2);
     float t8[4][8];     // rows of T, kept for the two T diag() tile pairs
     if (ok) {
-        // ---- step 3: A by columns (warps 0, 1, into At) and P by rows (warps
-        // 2, 3, straight to the record), 16 TMEM columns at a time.  K K^T is
-        // symmetric, so TMEM lane c (row c) holds column c of it: thread c
-        // writes column c of A as contiguous 16-byte vectors.  A[j][c] is
-        // nonzero for c < j in the same segment, i.e. c < j < se_c; P[j][i] for
-        // ss_j <= i <= j.
+        // ---- step 3: A and P^T by columns of K [K;Q]^T (warps 0, 1) and the
+        // K' rows (warps 2, 3).  K K^T is symmetric, so TMEM lane c (row c)
+        // holds column c of it: thread c writes column c of A into At as
+        // contiguous 16-byte vectors, and row c of P^T (K Q^T row c) to the
+        // record.  A[j][c] is nonzero for c < j in the same segment, i.e.
+        // c < j < se_c; P[j][c] for c <= j < se_c.
         if (tid < 64) {
             const int c = tid, ce = sm.se[c];
             const float w = sm.wc[c];
@@ -367,28 +407,39 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                     *reinterpret_cast<float4 *>(At + c * A_LD + j0) = a4;
                 }
             }
-        } else {
-            const int j = tid - 64, sj = sm.ss[j];
-            const float u = sm.uq[j];
 #pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 16) {
-                float row[16];
-                tc::tmem_ld16(my_lane + WY_COL_KQ + cb, row);
+            for (int jb = 0; jb < 64; jb += 16) {
+                float pt[16];
+                tc::tmem_ld16(my_lane + WY_COL_KQ + 64 + jb, pt);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 w4 = *reinterpret_cast<const float4 *>(sm.wc + cb + 4 * e4);
-                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                    const float4 u4 = *reinterpret_cast<const float4 *>(sm.uq + jb + 4 * e4);
+                    const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int i = cb + 4 * e4 + e;
-                        row[4 * e4 + e] = (i <= j && i >= sj) ? row[4 * e4 + e] * exp2f(u - wv[e]) : 0.f;
+                        const int j = jb + 4 * e4 + e;
+                        pt[4 * e4 + e] = (j >= c && j < ce) ? pt[4 * e4 + e] * exp2f(uv[e] - w) : 0.f;
                     }
                 }
-                st_row8(rec + REC_P_HI, j, cb, C, row, false);
-                st_row8(rec + REC_P_HI, j, cb + 8, C, row + 8, false);
-                st_row8(rec + REC_P_LO, j, cb, C, row, true);
-                st_row8(rec + REC_P_LO, j, cb + 8, C, row + 8, true);
+                st_row8(rec + REC_KP_HI, c, K + jb, KP_COLS, pt, false);
+                st_row8(rec + REC_KP_HI, c, K + jb + 8, KP_COLS, pt + 8, false);
+                st_row8(rec + REC_KP_LO, c, K + jb, KP_COLS, pt, true);
+                st_row8(rec + REC_KP_LO, c, K + jb + 8, KP_COLS, pt + 8, true);
+            }
+        } else {
+            // K' = diag(fd) K: row j of the raw k rows, scaled, hi / lo
+            const int j = tid - 64;
+            const float f = sm.fd[j];
+#pragma unroll 4
+            for (int col = 0; col < K; col += 8) {
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(ktile + tc::kmajor_offset(j, col, K)), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    x[e] *= f;
+                st_row8(rec + REC_KP_HI, j, col, KP_COLS, x, false);
+                st_row8(rec + REC_KP_LO, j, col, KP_COLS, x, true);
             }
         }
         __syncthreads();
@@ -593,20 +644,17 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     }
     if (ok) {
         // ---- step 6: the record's remaining tiles -------------------------
-        // W (thread = k): W^T[k][.] from TMEM into an fp32 buffer [k][64]
-        // (column index XOR-swizzled by the row) over the q half of kq and r2
-        // (the v rows), free after the products; the hi / lo chunks of W
-        // [i][k] go to the record once it is complete
-        float *Wpad = reinterpret_cast<float *>(qhalf);
-        {
-            float wcol[64];
-#pragma unroll
-            for (int c = 0; c < 64; c += 16)
-                tc::tmem_ld16(my_lane + WY_COL_WT + c, wcol + c);
+        // W^T (thread = k): row k of W^T from TMEM, hi / lo, straight to the
+        // record
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 16) {
+            float w[16];
+            tc::tmem_ld16(my_lane + WY_COL_WT + c, w);
             tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-                Wpad[tid * 64 + (j ^ (tid & 31))] = wcol[j];
+            st_row8(rec + REC_WQ_HI, tid, c, WQ_COLS, w, false);
+            st_row8(rec + REC_WQ_HI, tid, c + 8, WQ_COLS, w + 8, false);
+            st_row8(rec + REC_W_LO, tid, c, C, w, true);
+            st_row8(rec + REC_W_LO, tid, c + 8, C, w + 8, true);
         }
         // U^T (thread = v): one fp32 row of 64
         {
@@ -621,33 +669,6 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                     dst[(c + e) / 4] = make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
             }
         }
-        // K'^T = (diag(fd) K)^T (thread = k): column k of the raw k rows,
-        // scaled, hi / lo
-        {
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    x[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                               ktile + tc::kmajor_offset(c + e, tid, K))) *
-                           sm.fd[c + e];
-                st_row8(rec + REC_KP_HI, tid, c, C, x, false);
-                st_row8(rec + REC_KP_LO, tid, c, C, x, true);
-            }
-        }
-        __syncthreads();
-        // W hi / lo: 16-byte chunks (row i, columns k0 .. k0 + 7), eight per thread
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int q = tid + 128 * n, i = q & 63, k0 = (q >> 6) * 8;
-            float w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                w8[e] = Wpad[(k0 + e) * 64 + (i ^ ((k0 + e) & 31))];
-            st_row8(rec + REC_W_HI, i, k0, K, w8, false);
-            st_row8(rec + REC_W_LO, i, k0, K, w8, true);
-        }
     }
 
     sync::cp_async_wait_all();      // the v rows' copies, on a path that skipped their use
@@ -661,6 +682,37 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // Kernel 2: the recurrence through the state of one (sequence, value head).
 // ---------------------------------------------------------------------------
+
+// Product 1 of a piece, issued by one thread and committed to `bar`:
+// [D | O1] = -S~^T [W hi; Q]^T (N = 128, from column dq_col) from the hi and
+// lo state tiles (K-major [v][k]), then D -= S~hi^T W lo^T; the record tiles
+// [W^T hi | Q^T] and W^T lo are read MN-major.
+__device__ __forceinline__ void state_product1(uint32_t tmem, uint32_t dq_col, const unsigned char *st_hi,
+                                               const unsigned char *st_lo, const unsigned char *wq_hi,
+                                               const unsigned char *w_lo, unsigned long long *bar)
+{
+    const uint32_t ID_WQ = tc::idesc_bf16_f32(128, WQ_COLS, true, false, true);  // negated; B MN-major
+    const uint32_t ID_W = tc::idesc_bf16_f32(128, C, true, false, true);
+    mma_tiles_bmn(tmem + dq_col, st_hi, K, wq_hi, WQ_COLS, K / 16, ID_WQ, false);
+    mma_tiles_bmn(tmem + dq_col, st_lo, K, wq_hi, WQ_COLS, K / 16, ID_WQ, true);
+    mma_tiles_bmn(tmem + dq_col, st_hi, K, w_lo, C, K / 16, ID_W, true);
+    tc::mma_commit(bar);
+}
+
+// Product 2 of a piece, issued by one thread and committed to `bar`:
+// [S~^T | O2] += Delta~^T [K' | P^T] (N = 192, from column s_col) for the split
+// pairs (hi, hi), (hi, lo), (lo, hi); the [K' | P^T] tiles ([i][k | j]) are
+// read MN-major.
+__device__ __forceinline__ void state_product2(uint32_t tmem, uint32_t s_col, const unsigned char *dt_hi,
+                                               const unsigned char *dt_lo, const unsigned char *kp_hi,
+                                               const unsigned char *kp_lo, unsigned long long *bar)
+{
+    const uint32_t ID = tc::idesc_bf16_f32(128, KP_COLS, false, false, true);  // B MN-major
+    mma_tiles_bmn(tmem + s_col, dt_hi, C, kp_hi, KP_COLS, C / 16, ID, true);
+    mma_tiles_bmn(tmem + s_col, dt_hi, C, kp_lo, KP_COLS, C / 16, ID, true);
+    mma_tiles_bmn(tmem + s_col, dt_lo, C, kp_hi, KP_COLS, C / 16, ID, true);
+    tc::mma_commit(bar);
+}
 struct StSmem {
     alignas(1024) unsigned char st[2][128 * 128 * 2];   // S~^T hi / lo [v][k]
     alignas(1024) unsigned char rec_a[REC_A_BYTES];     // W hi, Q, W lo of the piece (record bytes 0 .. 49151)
@@ -811,11 +863,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     };
     publish_smem();
 
-    const uint32_t ID_N64_NEG = tc::idesc_bf16_f32(128, 64, true);
-    const uint32_t ID_N128_NEG = tc::idesc_bf16_f32(128, 128, true);
-    const uint32_t ID_N192 = tc::idesc_bf16_f32(128, 192);
-    const unsigned char *wq_hi = sm.rec_a + REC_W_HI, *w_lo = sm.rec_a + REC_W_LO;   // [W hi; Q], W lo
-    const unsigned char *kpp_hi = sm.rec_b, *kpp_lo = sm.rec_b + (REC_KP_LO - REC_KP_HI);  // [K'^T; P] hi, lo
+    const unsigned char *wq_hi = sm.rec_a + REC_WQ_HI, *w_lo = sm.rec_a + REC_W_LO;
+    const unsigned char *kp_hi = sm.rec_b, *kp_lo = sm.rec_b + (REC_KP_LO - REC_KP_HI);
 
     // Outputs of a piece are written during the next piece (while its first
     // products run); these describe the piece whose outputs are pending.
@@ -874,12 +923,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             break;
         pend_a = false;
         const uint32_t dq = ST_COL_DQ + 128u * buf;
-        if (tid == 0) {
-            mma_tiles(tmem + dq, sm.st[0], K, wq_hi, K, K / 16, ID_N128_NEG, false);
-            mma_tiles(tmem + dq, sm.st[1], K, wq_hi, K, K / 16, ID_N128_NEG, true);
-            mma_tiles(tmem + dq, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
-            tc::mma_commit(&sm.bar_d);
-        }
+        if (tid == 0)
+            state_product1(tmem, dq, sm.st[0], sm.st[1], wq_hi, w_lo, &sm.bar_d);
         // the previous piece's outputs, while these products run
         if (out_pending)
             write_outputs();
@@ -953,10 +998,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T (3 split products;
         // bar_s) ------------------------------------------------------------
         if (tid == 0) {
-            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kpp_hi, C, C / 16, ID_N192, true);
-            mma_tiles(tmem + ST_COL_S, sm.dt[0], C, kpp_lo, C, C / 16, ID_N192, true);
-            mma_tiles(tmem + ST_COL_S, sm.dt[1], C, kpp_hi, C, C / 16, ID_N192, true);
-            tc::mma_commit(&sm.bar_s);
+            state_product2(tmem, ST_COL_S, sm.dt[0], sm.dt[1], kp_hi, kp_lo, &sm.bar_s);
             if (more) {              // fo / gamma of the next piece (read above)
                 sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
                 sync::bulk_load(sm.rec_s, rec_of(blk + 1) + REC_FO, REC_S_BYTES, &sm.bar_r);
@@ -1164,11 +1206,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
     };
     publish_smem();
 
-    const uint32_t ID_N64_NEG = tc::idesc_bf16_f32(128, 64, true);
-    const uint32_t ID_N128_NEG = tc::idesc_bf16_f32(128, 128, true);
-    const uint32_t ID_N192 = tc::idesc_bf16_f32(128, 192);
-    const unsigned char *wq_hi = sm.rec + REC_W_HI, *w_lo = sm.rec + REC_W_LO;
-    const unsigned char *kpp_hi = sm.rec, *kpp_lo = sm.rec + (REC_KP_LO - REC_KP_HI);
+    const unsigned char *wq_hi = sm.rec + REC_WQ_HI, *w_lo = sm.rec + REC_W_LO;
+    const unsigned char *kp_hi = sm.rec, *kp_lo = sm.rec + (REC_KP_LO - REC_KP_HI);
     unsigned char *const dt_hi = sm.st[0], *const dt_lo = sm.st[0] + 128 * 64 * 2;
 
     float cs = 1.f;
@@ -1197,12 +1236,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
         if (!ok)
             break;
         pend_a = false;
-        if (tid == 0) {
-            mma_tiles(tmem + SC_COL_D, sm.st[0], K, wq_hi, K, K / 16, ID_N128_NEG, false);
-            mma_tiles(tmem + SC_COL_D, sm.st[1], K, wq_hi, K, K / 16, ID_N128_NEG, true);
-            mma_tiles(tmem + SC_COL_D, sm.st[0], K, w_lo, K, K / 16, ID_N64_NEG, true);
-            tc::mma_commit(&sm.bar_m);
-        }
+        if (tid == 0)
+            state_product1(tmem, SC_COL_D, sm.st[0], sm.st[1], wq_hi, w_lo, &sm.bar_m);
         wait_bar(&sm.bar_m, ph_m);
         if (!ok)
             break;
@@ -1266,10 +1301,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
             break;
         pend_b = false;
         if (tid == 0) {
-            mma_tiles(tmem + SC_COL_S, dt_hi, C, kpp_hi, C, C / 16, ID_N192, true);
-            mma_tiles(tmem + SC_COL_S, dt_hi, C, kpp_lo, C, C / 16, ID_N192, true);
-            mma_tiles(tmem + SC_COL_S, dt_lo, C, kpp_hi, C, C / 16, ID_N192, true);
-            tc::mma_commit(&sm.bar_m);
+            state_product2(tmem, SC_COL_S, dt_hi, dt_lo, kp_hi, kp_lo, &sm.bar_m);
             if (more) {
                 sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
                 sync::bulk_load(sm.rec_s, rec_of(blk + 1) + REC_FO, REC_S_BYTES, &sm.bar_r);
