@@ -50,7 +50,7 @@ ROTATING_COPIES = 4
 def chunked_min_mean_tokens(pairs):
     """The split chunked kernels' threshold (the binding always passes a
     workspace)."""
-    return 64 if pairs < 64 else (40 if pairs < 512 else 26)
+    return 40 if pairs < 64 else (30 if pairs < 512 else 18)
 
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +

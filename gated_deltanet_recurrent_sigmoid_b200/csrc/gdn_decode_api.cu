@@ -34,11 +34,11 @@ constexpr int64_t kChunkedMinMeanTokensMany = 256;
 constexpr int64_t kChunkedFewPairs = 1024;
 // With a workspace, AUTO takes the split chunked kernels from a lower mean
 // length (measured B200 crossovers against the per-tile kernel, lengths
-// spread over [L/2, 3L/2]): 64 tokens below 64 (sequence, value head)
-// pairs, 40 below 512, 26 from 512 on (at the threshold the split kernels
-// are 0.7-1.0 of the per-tile time; with 64-1024 sequences the ratio is
-// 1.01-1.04 at 24 tokens and 0.89-0.97 at 28).
-int64_t split_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 64 : (pairs < 512 ? 40 : 26); }
+// spread over [L/2, 3L/2]): 40 tokens below 64 (sequence, value head)
+// pairs, 30 below 512, 18 from 512 on (split / per-tile time: 1 sequence
+// 1.04 at 36 tokens, 0.81 at 48; 8 sequences 1.23 at 23, 0.90 at 33; 64-1024
+// sequences 0.98-1.06 at 16, 0.88-0.92 at 20).
+int64_t split_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 40 : (pairs < 512 ? 30 : 18); }
 // The split schedule's state kernel in its compact form (two CTAs per SM)
 // from this many (sequence, value head) pairs per SM, for sequences of at
 // most this many tokens on average (measured on B200: 0.89-0.92x the time of

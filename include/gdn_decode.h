@@ -129,8 +129,8 @@ extern "C" {
                                     gates, no per-token states, v rows 16-byte
                                     aligned): GDN_SCHEDULE_CHUNKED_SPLIT if the
                                     caller gives a large enough workspace and
-                                    the sequences hold, on average, >= 64 tokens
-                                    (N * HV < 64), >= 40 (N * HV < 512) or >= 26
+                                    the sequences hold, on average, >= 40 tokens
+                                    (N * HV < 64), >= 30 (N * HV < 512) or >= 18
                                     (otherwise); without a workspace
                                     GDN_SCHEDULE_CHUNKED from >= 128 tokens
                                     (N * HV <= 1024) or >= 256.  Otherwise
