@@ -534,6 +534,7 @@ def main():
         e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(pipe.h2d_bytes),
                "d2h_bytes_per_step": int(pipe.d2h_bytes), "api": "binding.PipelinedHostDecode",
+               "pipeline_depth": pipe.depth,
                "how": "each step: pinned host inputs -> device, update, output -> pinned host; the host "
                       "receives every step's output; copies overlap the neighbouring steps' kernels"}
         del pipe

@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
-from typing import Optional
+from typing import List, Optional
 
 import torch
 
@@ -62,6 +62,17 @@ class GdnExtra(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64)]
 
 
+class GdnHostStep(ctypes.Structure):
+    _fields_ = ([(n, ctypes.POINTER(GdnTensor)) for n in
+                 ("q", "k", "v", "a", "b", "A_log", "dt_bias", "state_pool", "state_indices", "cu_seqlens", "out")] +
+                [("scale", ctypes.c_float), ("flags", ctypes.c_uint32), ("extra", ctypes.POINTER(GdnExtra)),
+                 ("host_in", ctypes.c_void_p), ("dev_in", ctypes.c_void_p), ("in_bytes", ctypes.c_uint64),
+                 ("dev_out", ctypes.c_void_p), ("host_out", ctypes.c_void_p), ("out_bytes", ctypes.c_uint64),
+                 ("copy_in_stream", ctypes.c_void_p), ("copy_out_stream", ctypes.c_void_p),
+                 ("ev_h2d", ctypes.c_void_p), ("ev_ran", ctypes.c_void_p), ("ev_d2h", ctypes.c_void_p),
+                 ("reused", ctypes.c_int32)])
+
+
 _LIB = None
 
 
@@ -91,6 +102,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_version.argtypes = []
         lib.gdn_chunked_workspace_bytes.restype = ctypes.c_uint64
         lib.gdn_chunked_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        lib.gdn_host_step_issue.restype = ctypes.c_int
+        lib.gdn_host_step_issue.argtypes = [ctypes.POINTER(GdnHostStep)]
         lib.gdn_decode_update_static_scratch.restype = ctypes.c_int
         lib.gdn_decode_update_static_scratch.argtypes = [P] * 11 + [ctypes.c_float, ctypes.c_uint32,
                                                                     ctypes.POINTER(GdnExtra)]
@@ -331,12 +344,23 @@ class PreparedCall:
         _set_workspace(self._extra, self.workspace)
         self._args = [_ref(d) for d in self._descs] + [ctypes.c_float(scale), ctypes.c_uint32(flags),
                                                        ctypes.byref(self._extra)]
+        self._scale, self._flags = float(scale), int(flags)
         self._fn = self._lib.gdn_decode_update
 
     def __call__(self) -> None:
         status = self._fn(*self._args)
         if status != OK:
             raise GdnError(status, status_string(status))
+
+    def fill_host_step(self, st: "GdnHostStep") -> None:
+        """Copy this call's arguments into a gdn_host_step (the transfer
+        fields are the caller's)."""
+        names = ("q", "k", "v", "a", "b", "A_log", "dt_bias", "state_pool", "state_indices", "cu_seqlens", "out")
+        for name, d in zip(names, self._descs):
+            setattr(st, name, ctypes.pointer(d) if d is not None else None)
+        st.scale = self._scale
+        st.flags = self._flags
+        st.extra = ctypes.pointer(self._extra)
 
 
 class HostStagedDecode:
@@ -402,68 +426,81 @@ class HostStagedDecode:
 class PipelinedHostDecode:
     """Host-fed decode steps with the transfers overlapped across steps.
 
-    Two ``HostStagedDecode`` slots alternate.  Step k copies its inputs in on
-    a copy stream, runs the update on the compute stream (steps stay in
-    order there, so each step sees the previous step's state) and copies its
-    output back on a third stream; meanwhile step k+1's input copy and step
-    k-1's output copy can run beside step k's kernel.  ``inputs()`` returns
-    the host views to fill for the next step (waiting, if needed, until that
-    slot's previous input copy has read them); ``step()`` issues the step and
-    returns the host output of the step before it (waiting for it), or None
-    on the first call; ``finish()`` returns the last step's host output.
-    Constructor arguments are those of ``HostStagedDecode``.
+    ``depth`` ``HostStagedDecode`` slots are used in turn.  Step k copies its
+    inputs in on a copy stream, runs the update on the compute stream (steps
+    stay in order there, so each step sees the previous step's state) and
+    copies its output back on a third stream; meanwhile later steps' input
+    copies and earlier steps' output copies run beside step k's kernel.
+    ``inputs()`` returns the host views to fill for the next step (waiting, if
+    needed, until that slot's previous input copy has read them); ``step()``
+    issues the step and returns the host output of the step issued
+    ``depth - 1`` calls before it (waiting for it), or None while the pipeline
+    fills; ``finish()`` returns the host outputs of the steps still pending,
+    in order.  A returned output stays valid until the next ``step()`` call.
+    With depth 3 the host waits for an output one step after its kernel has
+    ended, so it keeps issuing ahead of the GPU.  Other arguments are those of
+    ``HostStagedDecode``.
     """
 
-    def __init__(self, *args, stream: Optional[torch.cuda.Stream] = None, **kw):
+    def __init__(self, *args, stream: Optional[torch.cuda.Stream] = None, depth: int = 3, **kw):
+        if depth < 2:
+            raise ValueError("depth must be at least 2")
         dev = args[8].device if len(args) > 8 else kw["state_pool"].device
+        self.depth = int(depth)
         self.compute = stream if stream is not None else torch.cuda.Stream(dev)
         self.copy_in = torch.cuda.Stream(dev)
         self.copy_out = torch.cuda.Stream(dev)
-        self.slots = [HostStagedDecode(*args, stream=self.compute, **kw) for _ in range(2)]
-        self._h2d = [torch.cuda.Event() for _ in range(2)]
-        self._ran = [torch.cuda.Event() for _ in range(2)]
-        self._d2h = [torch.cuda.Event() for _ in range(2)]
+        self.slots = [HostStagedDecode(*args, stream=self.compute, **kw) for _ in range(self.depth)]
+        self._h2d = [torch.cuda.Event() for _ in range(self.depth)]
+        self._ran = [torch.cuda.Event() for _ in range(self.depth)]
+        self._d2h = [torch.cuda.Event() for _ in range(self.depth)]
         self.h2d_bytes = self.slots[0].h2d_bytes
         self.d2h_bytes = self.slots[0].d2h_bytes
-        self.k = 0
+        self.k = 0          # steps issued
+        self.done = 0       # steps whose output has been returned
+        # one gdn_host_step per slot: the whole step is one C call.  torch
+        # creates an event's CUDA handle at its first record; record each once.
+        for e in self._h2d + self._ran + self._d2h:
+            e.record(self.compute)
+        self._issue = load().gdn_host_step_issue
+        self._steps = []
+        for b, sl in enumerate(self.slots):
+            st = GdnHostStep()
+            sl._call.fill_host_step(st)
+            st.host_in, st.dev_in, st.in_bytes = sl.host_buffer.data_ptr(), sl.device_buffer.data_ptr(), sl.h2d_bytes
+            st.dev_out, st.host_out, st.out_bytes = sl.out_device.data_ptr(), sl.out_host.data_ptr(), sl.d2h_bytes
+            st.copy_in_stream, st.copy_out_stream = self.copy_in.cuda_stream, self.copy_out.cuda_stream
+            st.ev_h2d, st.ev_ran, st.ev_d2h = (self._h2d[b].cuda_event, self._ran[b].cuda_event,
+                                                self._d2h[b].cuda_event)
+            self._steps.append((st, ctypes.byref(st)))
 
     def inputs(self) -> "HostStagedDecode":
         """The slot whose host views (``q``, ``k``, ...) the next step reads."""
-        b = self.k & 1
-        if self.k >= 2:
+        b = self.k % self.depth
+        if self.k >= self.depth:
             self._h2d[b].synchronize()
         return self.slots[b]
 
-    def step(self) -> Optional[torch.Tensor]:
-        b = self.k & 1
-        s = self.slots[b]
-        if self.k >= 2:                      # slot b's device inputs were read by step k-2
-            self.copy_in.wait_event(self._ran[b])
-        with torch.cuda.stream(self.copy_in):
-            s.device_buffer.copy_(s.host_buffer, non_blocking=True)
-        self._h2d[b].record(self.copy_in)
-        self.compute.wait_event(self._h2d[b])
-        if self.k >= 2:                      # and its device output was read back by step k-2
-            self.compute.wait_event(self._d2h[b])
-        s._call()
-        self._ran[b].record(self.compute)
-        self.copy_out.wait_event(self._ran[b])
-        with torch.cuda.stream(self.copy_out):
-            s.out_host.copy_(s.out_device, non_blocking=True)
-        self._d2h[b].record(self.copy_out)
-        prev = None
-        if self.k >= 1:
-            self._d2h[b ^ 1].synchronize()
-            prev = self.slots[b ^ 1].out_host
-        self.k += 1
-        return prev
-
-    def finish(self) -> Optional[torch.Tensor]:
-        if self.k == 0:
-            return None
-        b = (self.k - 1) & 1
+    def _output(self) -> torch.Tensor:
+        b = self.done % self.depth
         self._d2h[b].synchronize()
+        self.done += 1
         return self.slots[b].out_host
+
+    def step(self) -> Optional[torch.Tensor]:
+        # gdn_host_step_issue: copy in (after step k - depth's update has read
+        # slot b), update (after step k - depth's output has left slot b),
+        # copy out, each ordered by the slot's events
+        st, ref = self._steps[self.k % self.depth]
+        st.reused = 1 if self.k >= self.depth else 0
+        status = self._issue(ref)
+        if status != OK:
+            raise GdnError(status, status_string(status))
+        self.k += 1
+        return self._output() if self.k - self.done >= self.depth else None
+
+    def finish(self) -> List[torch.Tensor]:
+        return [self._output() for _ in range(self.k - self.done)]
 
 
 class PreparedUnfusedCall:

@@ -902,4 +902,41 @@ GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tens
                              &x);
 }
 
+GDN_API int gdn_host_step_issue(const gdn_host_step *s)
+{
+    if (!s || !s->extra || !s->host_in || !s->dev_in || !s->dev_out || !s->host_out || !s->ev_h2d ||
+        !s->ev_ran || !s->ev_d2h)
+        return GDN_ERR_NULL_ARG;
+    cudaStream_t compute = static_cast<cudaStream_t>(s->extra->stream);
+    cudaStream_t cin = static_cast<cudaStream_t>(s->copy_in_stream);
+    cudaStream_t cout = static_cast<cudaStream_t>(s->copy_out_stream);
+    cudaEvent_t h2d = static_cast<cudaEvent_t>(s->ev_h2d), ran = static_cast<cudaEvent_t>(s->ev_ran),
+                d2h = static_cast<cudaEvent_t>(s->ev_d2h);
+    cudaError_t err = cudaSuccess;
+    if (s->reused)
+        err = cudaStreamWaitEvent(cin, ran, 0);
+    if (err == cudaSuccess && s->in_bytes)
+        err = cudaMemcpyAsync(s->dev_in, s->host_in, s->in_bytes, cudaMemcpyHostToDevice, cin);
+    if (err == cudaSuccess)
+        err = cudaEventRecord(h2d, cin);
+    if (err == cudaSuccess)
+        err = cudaStreamWaitEvent(compute, h2d, 0);
+    if (err == cudaSuccess && s->reused)
+        err = cudaStreamWaitEvent(compute, d2h, 0);
+    if (err != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int status = gdn_decode_update(s->q, s->k, s->v, s->a, s->b, s->A_log, s->dt_bias, s->state_pool,
+                                         s->state_indices, s->cu_seqlens, s->out, s->scale, s->flags, s->extra);
+    if (status != GDN_OK)
+        return status;
+    err = cudaEventRecord(ran, compute);
+    if (err == cudaSuccess)
+        err = cudaStreamWaitEvent(cout, ran, 0);
+    if (err == cudaSuccess && s->out_bytes)
+        err = cudaMemcpyAsync(s->host_out, s->dev_out, s->out_bytes, cudaMemcpyDeviceToHost, cout);
+    if (err == cudaSuccess)
+        err = cudaEventRecord(d2h, cout);
+    return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -301,6 +301,55 @@ GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tens
                                              const gdn_tensor *cu_seqlens, const gdn_tensor *out,
                                              float scale, uint32_t flags, const gdn_extra *extra);
 
+/*
+ * One step of a host-fed update loop, issued in a single call: the pinned
+ * host -> device copy of the step's packed inputs, the update, and the
+ * device -> host copy of its output, each on its own stream and ordered by
+ * events, so that a loop keeping several such steps in flight overlaps the
+ * transfers of neighbouring steps with the update (the step's cost on the
+ * host is one call instead of a dozen runtime calls).  Host plumbing: the
+ * pages have no counterpart of it.
+ *
+ * Per slot (a set of buffers reused every `depth` steps) the caller keeps one
+ * gdn_host_step; per call the library enqueues, in order:
+ *   copy_in:  [wait ev_ran, if `reused`] copy in_bytes host_in -> dev_in;
+ *             record ev_h2d
+ *   compute:  wait ev_h2d; [wait ev_d2h, if `reused`]; gdn_decode_update with
+ *             the descriptors below (they describe views of dev_in and
+ *             dev_out; extra->stream is the compute stream); record ev_ran
+ *   copy_out: wait ev_ran; copy out_bytes dev_out -> host_out; record ev_d2h
+ * `reused` (nonzero when the slot served an earlier step) makes the copy in
+ * wait until that step's update has read dev_in, and the update wait until
+ * that step's output has left dev_out.  Nothing waits on the host: the
+ * caller synchronises on ev_h2d before rewriting host_in and on ev_d2h
+ * before reading host_out.  host_in / host_out should be pinned (page-locked)
+ * for the copies to be asynchronous.  Streams and events are the caller's
+ * (cudaStream_t / cudaEvent_t, events preferably without timing).
+ *
+ * Returns the update's status (nothing after a failed update is enqueued),
+ * GDN_ERR_NULL_ARG for a missing pointer, or GDN_ERR_CUDA when the runtime
+ * refuses a copy or an event operation (steps enqueued before it stay
+ * enqueued).
+ */
+typedef struct {
+    const gdn_tensor *q, *k, *v, *a, *b, *A_log, *dt_bias, *state_pool, *state_indices, *cu_seqlens, *out;
+    float scale;
+    uint32_t flags;
+    const gdn_extra *extra;       /* required: its stream is the compute stream */
+    const void *host_in;
+    void *dev_in;
+    uint64_t in_bytes;
+    const void *dev_out;
+    void *host_out;
+    uint64_t out_bytes;
+    void *copy_in_stream;         /* cudaStream_t */
+    void *copy_out_stream;        /* cudaStream_t */
+    void *ev_h2d, *ev_ran, *ev_d2h; /* cudaEvent_t */
+    int32_t reused;
+} gdn_host_step;
+
+GDN_API int gdn_host_step_issue(const gdn_host_step *step);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,7 +25,7 @@ def declared_functions():
 def test_header_declares_the_abi():
     assert set(declared_functions()) == {"gdn_decode_update", "gdn_recurrent_update", "gdn_gating",
                                          "gdn_status_string", "gdn_version", "gdn_chunked_workspace_bytes",
-                                         "gdn_decode_update_static_scratch"}
+                                         "gdn_decode_update_static_scratch", "gdn_host_step_issue"}
 
 
 def test_library_exports_every_declared_symbol(gdn_lib):
@@ -70,6 +70,8 @@ def test_header_constants_match_binding():
         assert int(re.search(rf"#define {name}\s+\((-?\d+)\)", text).group(1)) == val
     assert ctypes.sizeof(binding.GdnTensor) == 8 + 4 + 4 + 8 * 4 + 8 * 4
     assert ctypes.sizeof(binding.GdnExtra) == 8 + 8 + 8 + 4 * 4 + 8 + 8
+    # 11 descriptors, scale + flags, extra, 2 x (2 pointers + size), 2 streams, 3 events, reused (+ padding)
+    assert ctypes.sizeof(binding.GdnHostStep) == 11 * 8 + 8 + 8 + 2 * 24 + 16 + 24 + 8
 
 
 def make(N=4, T=1, H=2, HV=4, K=128, V=128, slots=8, varlen=True):
@@ -190,3 +192,16 @@ def test_split_schedule_checks_its_workspace(gdn_lib):
     big = raw[((-raw.data_ptr()) % 256) // 4:]                                         # 256-byte aligned
     t2["state_pool"] = big[: t2["state_pool"].numel()].view(t2["state_pool"].shape)   # workspace overlaps the pool
     expect(binding.ERR_ALIAS, t2, schedule=split, workspace=big.view(torch.uint8)[:need])
+
+
+def test_host_step_rejects_missing_pointers(gdn_lib):
+    """gdn_host_step_issue checks its pointers before any CUDA call."""
+    assert gdn_lib.gdn_host_step_issue(None) == binding.ERR_NULL_ARG
+    st = binding.GdnHostStep()
+    assert gdn_lib.gdn_host_step_issue(ctypes.byref(st)) == binding.ERR_NULL_ARG
+    extra = binding.GdnExtra()
+    st.extra = ctypes.pointer(extra)
+    buf = (ctypes.c_char * 64)()
+    st.host_in = st.dev_in = st.dev_out = st.host_out = ctypes.addressof(buf)
+    st.ev_h2d = st.ev_ran = None
+    assert gdn_lib.gdn_host_step_issue(ctypes.byref(st)) == binding.ERR_NULL_ARG

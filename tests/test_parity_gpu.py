@@ -389,10 +389,12 @@ def test_host_staged_decode_matches_device_call(spec):
 
 @pytest.mark.parametrize("spec", [wl.TINY, wl.shrink(wl.SPEC_B128_T4, 16), wl.shrink(wl.DECODE_B512, 8)],
                          ids=lambda s: s.name)
-def test_pipelined_host_decode_matches_device_calls(spec):
+@pytest.mark.parametrize("depth", [2, 3, 4])
+def test_pipelined_host_decode_matches_device_calls(spec, depth):
     """Five host-fed steps with different inputs, copies overlapped across
-    steps: every step's host output and the final pool are the bits of the
-    same five steps run as device-resident calls, in order."""
+    steps (2, 3 or 4 slots in flight): every step's host output and the final
+    pool are the bits of the same five steps run as device-resident calls, in
+    order."""
     ws = [wl.generate(dataclasses.replace(spec, seed=spec.seed + 100 * n)) for n in range(5)]
     ref = to_device(ws[0])
     ref_outs = []
@@ -405,7 +407,7 @@ def test_pipelined_host_decode_matches_device_calls(spec):
     d0 = to_device(ws[0])
     varlen = ws[0].cu_seqlens is not None
     pipe = binding.PipelinedHostDecode(d0["q"].shape[:-2], spec.H, spec.HV, spec.K, spec.V, spec.N, d0["A_log"],
-                                       d0["dt_bias"], d0["state_pool"], varlen=varlen)
+                                       d0["dt_bias"], d0["state_pool"], varlen=varlen, depth=depth)
     outs = []
     for w in ws:
         d = to_device(w)
@@ -416,7 +418,7 @@ def test_pipelined_host_decode_matches_device_calls(spec):
         prev = pipe.step()
         if prev is not None:
             outs.append(prev.clone())
-    outs.append(pipe.finish().clone())
+    outs.extend(o.clone() for o in pipe.finish())
     torch.cuda.synchronize()
     assert len(outs) == len(ref_outs)
     for got, exp in zip(outs, ref_outs):
