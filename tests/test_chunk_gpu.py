@@ -181,6 +181,30 @@ def test_auto_schedule_picks_chunked_for_long_sequences():
     assert _bits_equal(auto_d, pt_d) and torch.equal(auto_i, pt_i)
 
 
+def test_chunked_strided_views_of_packed_projections(sched):
+    """q, k, v as column slices of one packed projection row (token stride
+    wider than a head's row) and a, b interleaved per value head: the same
+    bits as contiguous inputs, on both chunked schedules."""
+    w = problem([200, 37, 130, 64, 5], seed=61)
+    ref, _, _ = run_gpu(w, schedule=sched)
+    d = to_device(w)
+    T, H, HV, K, V = w.T_tot, w.spec.H, w.spec.HV, w.spec.K, w.spec.V
+    width = 2 * H * K + HV * V + 64
+    packed = torch.zeros(T, width, dtype=torch.bfloat16, device="cuda")
+    packed[:, :H * K] = d["q"].reshape(T, -1)
+    packed[:, H * K:2 * H * K] = d["k"].reshape(T, -1)
+    packed[:, 2 * H * K:2 * H * K + HV * V] = d["v"].reshape(T, -1)
+    q = packed[:, :H * K].view(T, H, K)
+    k = packed[:, H * K:2 * H * K].view(T, H, K)
+    v = packed[:, 2 * H * K:2 * H * K + HV * V].view(T, HV, V)
+    ba = torch.stack([d["b"], d["a"]], dim=-1).contiguous()          # [T, HV, 2]
+    b, a = ba[..., 0], ba[..., 1]
+    binding.decode_update(q, k, v, a, b, d["A_log"], d["dt_bias"], d["state_pool"], d["state_indices"],
+                          d["cu_seqlens"], d["out"], schedule=sched)
+    torch.cuda.synchronize()
+    assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
+
+
 def test_split_compact_many_short_sequences():
     """Enough short sequences (320 x 8 heads) that the split schedule runs its
     compact state kernel: empty sequences, padded slots, weak and strong
