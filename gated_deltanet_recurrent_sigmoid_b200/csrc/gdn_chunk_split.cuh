@@ -722,8 +722,8 @@ struct StSmem {
     float fo[2][C];                                     // fo of the last two pieces (by piece parity)
     // bar_d: -S~^T [W; Q]^T done; bar_s: S~^T += Delta~^T [K'; P]^T done;
     // bar_a / bar_b / bar_r: the bulk copies of a piece's W / Q, K' / P and
-    // fo / gamma
-    unsigned long long bar_d, bar_s, bar_a, bar_b, bar_r;
+    // fo / gamma; bar_x: the copy of the state at the start
+    unsigned long long bar_d, bar_s, bar_a, bar_b, bar_r, bar_x;
     uint32_t tmem_base;
     int failed;
 };
@@ -805,8 +805,13 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         sync::mbar_init(&sm.bar_a, 1);
         sync::mbar_init(&sm.bar_b, 1);
         sync::mbar_init(&sm.bar_r, 1);
+        sync::mbar_init(&sm.bar_x, 1);
         sm.failed = 0;
         sync::fence_barrier_init();
+        // the state S [k][v] (64 KB, contiguous) into the state-tile region in
+        // one bulk copy, beside the first piece's records
+        sync::mbar_arrive_expect_tx(&sm.bar_x, K * V * 4);
+        sync::bulk_load(sm.st, s_gmem, K * V * 4, &sm.bar_x);
         const unsigned char *r = rec_of(blk);
         sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
         sync::bulk_load(sm.rec_a, r, REC_A_BYTES, &sm.bar_a);
@@ -827,22 +832,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     constexpr int KP = K / ST_PARTS, CP = C / ST_PARTS;   // columns per part: of S~^T, of the tokens
     const int kh = KP * part;                   // this thread's k columns of S~^T
 
-    for (int k0 = kh; k0 < kh + KP; k0 += 16) {   // column v of S (rows k) -> lane v of S~^T
-        float x[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            x[e] = __ldcs(s_gmem + (k0 + e) * V + v);
-        tc::tmem_st16(my_lane + ST_COL_S + k0, x);
-        st_row8(sm.st[0], v, k0, K, x, false);
-        st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
-        st_row8(sm.st[1], v, k0, K, x, true);
-        st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
-    }
-    tc::tmem_wait_st();
-
-    uint32_t ph_d = 0, ph_s = 0, ph_a = 0, ph_b = 0, ph_r = 0;
+    uint32_t ph_d = 0, ph_s = 0, ph_a = 0, ph_b = 0, ph_r = 0, ph_x = 0;
     // copies issued and not yet waited for, with the parity their wait checks
-    bool ok = true, pend_a = true, pend_b = true, pend_r = true;
+    bool ok = true, pend_a = true, pend_b = true, pend_r = true, pend_x = true;
     uint32_t pa = 0, pb = 0, pr = 0;
     // bounded wait on one of the barriers; uniform verdict over the CTA
     auto wait_bar = [&](unsigned long long *bar, uint32_t &ph) {
@@ -855,6 +847,29 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         ok = __syncthreads_and(w) != 0;
         tc::fence_after_sync();
     };
+
+    // column v of S (this thread's rows k) from the copied state into
+    // registers; once every thread holds its part, into TMEM (lane v of
+    // S~^T) and the S~^T hi / lo tiles over the same region
+    wait_bar(&sm.bar_x, ph_x);
+    if (ok) {
+        pend_x = false;
+        const float *raw = reinterpret_cast<const float *>(sm.st);
+        float x[KP];
+#pragma unroll
+        for (int kk = 0; kk < KP; ++kk)
+            x[kk] = raw[(kh + kk) * V + v];
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < KP; c += 16) {
+            tc::tmem_st16(my_lane + ST_COL_S + kh + c, x + c);
+            st_row8(sm.st[0], v, kh + c, K, x + c, false);
+            st_row8(sm.st[0], v, kh + c + 8, K, x + c + 8, false);
+            st_row8(sm.st[1], v, kh + c, K, x + c, true);
+            st_row8(sm.st[1], v, kh + c + 8, K, x + c + 8, true);
+        }
+        tc::tmem_wait_st();
+    }
     auto publish_smem = [&]() {
         tc::fence_proxy_async_smem();
         tc::fence_before_sync();
@@ -1050,7 +1065,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
 
     // a failed wait left copies in flight: let them land (bounded) before the
     // shared memory is released
-    if (pend_a || pend_b || pend_r) {
+    if (pend_a || pend_b || pend_r || pend_x) {
         volatile int never = 0;
         if (pend_a)
             sync::mbar_wait(&sm.bar_a, pa, &never);
@@ -1058,6 +1073,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             sync::mbar_wait(&sm.bar_b, pb, &never);
         if (pend_r)
             sync::mbar_wait(&sm.bar_r, pr, &never);
+        if (pend_x)
+            sync::mbar_wait(&sm.bar_x, 0, &never);
     }
 
     pdl_trigger();
