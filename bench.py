@@ -306,15 +306,19 @@ def run_reference(args, w):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, chunk_ok=False):
+def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, chunk_ok=False, sms=148):
     """Name of the kernel the library launches for these settings (mirrors
-    the library's documented choice)."""
+    the library's documented choice, including the split schedule's compact
+    state kernel from 2 (sequence, head) pairs per SM at <= 128 tokens per
+    sequence on average)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if (schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok
             and mean_tokens >= chunked_min_mean_tokens(pairs)):
         schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
     if schedule == binding.SCHEDULE_CHUNKED_SPLIT:
-        return "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"
+        state = ("gdn_chunk_state_compact_kernel" if pairs >= 2 * sms and mean_tokens <= 128
+                 else "gdn_chunk_state_kernel")
+        return f"gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::{state}"
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
     if schedule == binding.SCHEDULE_CHUNKED:
@@ -571,7 +575,8 @@ def main():
             traffic = NCU_TRAFFIC["bytes_per_launch"]
         kname = ("gdn::gdn_gating_kernel + " if args.unfused else "") + kernel_name(
             schedule, args.tile_v, args.tile_rows, w.T_tot == w.spec.N and not w.spec.intermediate,
-            w.spec.N * w.spec.HV, w.T_tot / max(1, w.spec.N), not args.unfused and not w.spec.intermediate)
+            w.spec.N * w.spec.HV, w.T_tot / max(1, w.spec.N), not args.unfused and not w.spec.intermediate,
+            torch.cuda.get_device_properties(device).multi_processor_count)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
