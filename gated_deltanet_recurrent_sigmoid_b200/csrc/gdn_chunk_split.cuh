@@ -1177,6 +1177,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
         sync::mbar_arrive_expect_tx(&sm.bar_x, K * V * 4);
         sync::bulk_load(sm.st, s_gmem, K * V * 4, &sm.bar_x);
         const unsigned char *r = rec_of(blk);
+        sync::prefetch_l2(r + REC_UT, REC_FO - REC_UT);     // U^T of the first piece (read per thread)
         sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
         sync::bulk_load(sm.rec, r, REC_A_BYTES, &sm.bar_a);
         sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
@@ -1250,6 +1251,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
         const int r1 = static_cast<int>((eos < base + C ? eos : base + C) - base);
         const bool more = base + r1 < eos;
         const unsigned char *rec = rec_of(blk);
+        if (more && tid == 0)           // the next piece's U^T, into L2 ahead of its per-thread reads
+            sync::prefetch_l2(rec_of(blk + 1) + REC_UT, REC_FO - REC_UT);
 
         float u[CP];
         {
