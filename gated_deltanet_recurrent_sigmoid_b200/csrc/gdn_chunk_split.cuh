@@ -15,7 +15,7 @@
 //                           block's W, U^T, P, K'^T = (diag(fd) K)^T and raw Q
 //                           into the workspace as the byte images of the
 //                           operand tiles the second kernel feeds to tcgen05.
-//   gdn_chunk_state_kernel  one 512-thread CTA per (sequence, value head) (or, for
+//   gdn_chunk_state_kernel  one 544-thread CTA per (sequence, value head) (or, for
 //                           many short sequences, gdn_chunk_state_compact_kernel:
 //                           256 threads, two CTAs per SM): walks the
 //                           blocks the sequence covers, fetching each block's
@@ -729,9 +729,13 @@ struct StSmem {
 };
 
 // state kernel: ST_PARTS threads per TMEM lane, each handling 1 / ST_PARTS of
-// the columns of every per-thread phase
+// the columns of every per-thread phase (the workers), plus one warp whose
+// first thread issues the products and the bulk copies, so that issuing the
+// first product does not hold back a worker warp's output stores
 constexpr int ST_PARTS = 4;
-constexpr int ST_THREADS = 128 * ST_PARTS;
+constexpr int ST_WORKERS = 128 * ST_PARTS;
+constexpr int ST_THREADS = ST_WORKERS + 32;
+constexpr int ST_ISSUER = ST_WORKERS;
 constexpr uint32_t ST_TMEM_COLS = 512;
 // TMEM columns.  Product 2 writes [S~^T | O2] (192 columns) in one MMA,
 // product 1 [D | O1] (128) in one MMA; [D | O1] is double-buffered by piece
@@ -755,9 +759,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    // thread (v, part): TMEM lane v = state column v; `part` picks which
-    // 1 / ST_PARTS of the columns of each per-thread phase it handles
+    // worker thread (v, part): TMEM lane v = state column v; `part` picks
+    // which 1 / ST_PARTS of the columns of each per-thread phase it handles
     const int v = tid & 127, part = tid >> 7;
+    const bool worker = tid < ST_WORKERS;
     const int i = blockIdx.x / p.HV;
     const int hv = blockIdx.x - i * p.HV;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
@@ -786,8 +791,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         return;
     }
     if (slot < 0) {
-        for (int t = part; t < len; t += ST_PARTS)
-            out[(bos + t) * p.o_tok + hv * p.o_head + v] = __float2bfloat16_rn(0.f);
+        if (worker)
+            for (int t = part; t < len; t += ST_PARTS)
+                out[(bos + t) * p.o_tok + hv * p.o_head + v] = __float2bfloat16_rn(0.f);
         return;
     }
     if (len == 0)
@@ -799,7 +805,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     // ---- set-up: barriers, TMEM, the first piece's tiles in flight, the
     // state into TMEM and into the S~^T tiles (cs = 1) ----------------------
     int64_t blk = bos / C;
-    if (tid == 0) {
+    if (tid == ST_ISSUER) {
         sync::mbar_init(&sm.bar_d, 1);
         sync::mbar_init(&sm.bar_s, 1);
         sync::mbar_init(&sm.bar_a, 1);
@@ -856,19 +862,23 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         pend_x = false;
         const float *raw = reinterpret_cast<const float *>(sm.st);
         float x[KP];
+        if (worker) {
 #pragma unroll
-        for (int kk = 0; kk < KP; ++kk)
-            x[kk] = raw[(kh + kk) * V + v];
-        __syncthreads();
-#pragma unroll
-        for (int c = 0; c < KP; c += 16) {
-            tc::tmem_st16(my_lane + ST_COL_S + kh + c, x + c);
-            st_row8(sm.st[0], v, kh + c, K, x + c, false);
-            st_row8(sm.st[0], v, kh + c + 8, K, x + c + 8, false);
-            st_row8(sm.st[1], v, kh + c, K, x + c, true);
-            st_row8(sm.st[1], v, kh + c + 8, K, x + c + 8, true);
+            for (int kk = 0; kk < KP; ++kk)
+                x[kk] = raw[(kh + kk) * V + v];
         }
-        tc::tmem_wait_st();
+        __syncthreads();
+        if (worker) {
+#pragma unroll
+            for (int c = 0; c < KP; c += 16) {
+                tc::tmem_st16(my_lane + ST_COL_S + kh + c, x + c);
+                st_row8(sm.st[0], v, kh + c, K, x + c, false);
+                st_row8(sm.st[0], v, kh + c + 8, K, x + c + 8, false);
+                st_row8(sm.st[1], v, kh + c, K, x + c, true);
+                st_row8(sm.st[1], v, kh + c + 8, K, x + c + 8, true);
+            }
+            tc::tmem_wait_st();
+        }
     }
     auto publish_smem = [&]() {
         tc::fence_proxy_async_smem();
@@ -890,7 +900,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
     auto write_outputs = [&]() {
         const uint32_t o1c = ST_COL_DQ + 128u * out_buf + 64u, o2c = ST_COL_O2;
 #pragma unroll
-        for (int cl = 0; cl < CP; cl += 16) {
+        for (int cl = 0; cl < CP && worker; cl += 16) {
             const int cb = CP * part + cl;
             float o1[16], o2[16];
             tc::tmem_ld16(my_lane + o1c + cb, o1);
@@ -919,7 +929,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         // this thread's part of the row of U^T (needed after the first product)
         const int ih = CP * part;                 // this thread's token columns
         float u[CP];
-        {
+        if (worker) {
             const float4 *src = reinterpret_cast<const float4 *>(rec + REC_UT) + v * 16 + ih / 4;
 #pragma unroll
             for (int m = 0; m < CP / 4; ++m) {
@@ -938,7 +948,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             break;
         pend_a = false;
         const uint32_t dq = ST_COL_DQ + 128u * buf;
-        if (tid == 0)
+        if (tid == ST_ISSUER)
             state_product1(tmem, dq, sm.st[0], sm.st[1], wq_hi, w_lo, &sm.bar_d);
         // the previous piece's outputs, while these products run
         if (out_pending)
@@ -948,7 +958,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         wait_bar(&sm.bar_d, ph_d);
         if (!ok)
             break;
-        if (more && tid == 0) {       // W and Q of the next piece, into the buffer just read
+        if (more && tid == ST_ISSUER) {     // W and Q of the next piece, into the buffer just read
             sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
             sync::bulk_load(sm.rec_a, rec_of(blk + 1), REC_A_BYTES, &sm.bar_a);
         }
@@ -969,7 +979,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         if (tid < C)
             sm.fo[buf][tid] = sm.rec_s[tid];
 #pragma unroll
-        for (int cl = 0; cl < CP; cl += 16) {
+        for (int cl = 0; cl < CP && worker; cl += 16) {
             const int cb = ih + cl;
             float d[16];
             tc::tmem_ld16(my_lane + dq + cb, d);
@@ -990,10 +1000,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             for (int e = 0; e < 16; ++e)
                 z[e] = 0.f;
 #pragma unroll
-            for (int cl = 0; cl < CP; cl += 16)
+            for (int cl = 0; cl < CP && worker; cl += 16)
                 tc::tmem_st16(my_lane + ST_COL_O2 + ih + cl, z);
         }
-        if (rescale) {               // S~ <- cs' S~ in TMEM; the scale returns to 1
+        if (rescale && worker) {     // S~ <- cs' S~ in TMEM; the scale returns to 1
 #pragma unroll 1
             for (int k0 = kh; k0 < kh + KP; k0 += 16) {
                 float x[16];
@@ -1012,7 +1022,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
 
         // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T (3 split products;
         // bar_s) ------------------------------------------------------------
-        if (tid == 0) {
+        if (tid == ST_ISSUER) {
             state_product2(tmem, ST_COL_S, sm.dt[0], sm.dt[1], kp_hi, kp_lo, &sm.bar_s);
             if (more) {              // fo / gamma of the next piece (read above)
                 sync::mbar_arrive_expect_tx(&sm.bar_r, REC_S_BYTES);
@@ -1026,7 +1036,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         wait_bar(&sm.bar_s, ph_s);
         if (!ok)
             break;
-        if (more && tid == 0) {
+        if (more && tid == ST_ISSUER) {
             sync::mbar_arrive_expect_tx(&sm.bar_b, REC_B_BYTES);
             sync::bulk_load(sm.rec_b, rec_of(blk + 1) + REC_KP_HI, REC_B_BYTES, &sm.bar_b);
         }
@@ -1041,7 +1051,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         out_pending = true;
 
         // ---- the next piece's S~^T tiles, or the final write-back -----------
-        for (int k0 = kh; k0 < kh + KP; k0 += 16) {
+        for (int k0 = kh; k0 < kh + KP && worker; k0 += 16) {
             float x[16];
             tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
             tc::tmem_wait_ld();
