@@ -326,7 +326,7 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     if tile_v:
         bv, rows = tile_v, tile_rows or 16
     else:
-        bv, rows = (64, 32) if one_token else ((32, 32) if pairs >= 2048 else (16, 16))
+        bv, rows = (64, 32) if one_token else ((32, 32) if pairs >= 2048 else ((8, 8) if pairs <= 64 else (16, 16)))
         rows = tile_rows or rows
     return f"gdn::gdn_decode_kernel<128,128,{bv},{128 // rows}>"
 

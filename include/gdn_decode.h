@@ -137,12 +137,13 @@ extern "C" {
                                     GDN_SCHEDULE_PER_TILE */
 #define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
                                     state tile moves through registers.  Tiles
-                                    (tile_v x tile_rows): 16x16, 32x16, 32x32,
-                                    64x16, 64x32.  Library choice: 64x32 when
-                                    every sequence has one token, else 32x32
-                                    with >= 2048 (sequence, value head) pairs,
-                                    else 16x16; with fp32 activations 32x16
-                                    for one token, else 16x16 */
+                                    (tile_v x tile_rows): 8x8, 16x16, 32x16,
+                                    32x32, 64x16, 64x32.  Library choice: 64x32
+                                    when every sequence has one token, else
+                                    32x32 with >= 2048 (sequence, value head)
+                                    pairs, 8x8 with <= 64, else 16x16; with
+                                    fp32 activations 32x16 for one token, else
+                                    16x16 */
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
                                     tiles stream through a shared-memory ring of
                                     bulk async copies (cp.async.bulk) */

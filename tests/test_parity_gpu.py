@@ -32,8 +32,8 @@ PER_TILE = binding.SCHEDULE_PER_TILE
 PIPELINED = binding.SCHEDULE_PIPELINED
 # (schedule, V-tile width, rows per thread) of every kernel the library can launch
 KERNELS = [(PER_TILE, 16, 16), (PER_TILE, 32, 16), (PER_TILE, 32, 32), (PER_TILE, 64, 16), (PER_TILE, 64, 32),
-           (PIPELINED, 0, 0)]
-KERNEL_IDS = ["tile16x16", "tile32x16", "tile32x32", "tile64x16", "tile64x32", "pipelined"]
+           (PIPELINED, 0, 0), (PER_TILE, 8, 8)]
+KERNEL_IDS = ["tile16x16", "tile32x16", "tile32x32", "tile64x16", "tile64x32", "pipelined", "tile8x8"]
 # the library's two default tiles and the pipelined schedule
 MAIN = [KERNELS[0], KERNELS[4], KERNELS[5]]
 MAIN_IDS = ["tile16x16", "tile64x32", "pipelined"]

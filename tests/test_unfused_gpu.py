@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 L2 = binding.L2NORM_QK
 INTER = binding.WRITE_INTERMEDIATE
-TILES = [(16, 16), (32, 16), (32, 32), (64, 16), (64, 32)]
+TILES = [(8, 8), (16, 16), (32, 16), (32, 32), (64, 16), (64, 32)]
 
 
 @pytest.fixture(scope="module", autouse=True)
