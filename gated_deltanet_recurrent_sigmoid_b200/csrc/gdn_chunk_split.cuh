@@ -12,9 +12,10 @@
 //
 //   gdn_chunk_wy_kernel     one CTA per (64-token block of the packed token
 //                           range, value head), all in parallel: writes the
-//                           block's W, U^T, P, K'^T = (diag(fd) K)^T and raw Q
+//                           block's W^T, Q^T, K' = diag(fd) K, P^T and U^T
 //                           into the workspace as the byte images of the
-//                           operand tiles the second kernel feeds to tcgen05.
+//                           operand tiles the second kernel feeds to tcgen05
+//                           (row by row, as the block kernel produces them).
 //   gdn_chunk_state_kernel  one 544-thread CTA per (sequence, value head) (or, for
 //                           many short sequences, gdn_chunk_state_compact_kernel:
 //                           256 threads, two CTAs per SM): walks the
