@@ -716,8 +716,8 @@ __device__ __forceinline__ void state_product2(uint32_t tmem, uint32_t s_col, co
 }
 struct StSmem {
     alignas(1024) unsigned char st[2][128 * 128 * 2];   // S~^T hi / lo [v][k]
-    alignas(1024) unsigned char rec_a[REC_A_BYTES];     // W hi, Q, W lo of the piece (record bytes 0 .. 49151)
-    alignas(1024) unsigned char rec_b[REC_B_BYTES];     // K'^T hi, P hi, K'^T lo, P lo (record bytes 49152 .. 98303)
+    alignas(1024) unsigned char rec_a[REC_A_BYTES];     // [W^T hi | Q^T], W^T lo of the piece (record bytes 0 .. 49151)
+    alignas(1024) unsigned char rec_b[REC_B_BYTES];     // [K' | P^T] hi, lo (record bytes 49152 .. 98303)
     alignas(1024) unsigned char dt[2][128 * 64 * 2];    // Delta~^T hi / lo [v][i]
     alignas(16) float rec_s[REC_S_BYTES / 4];           // fo, gamma of the piece (record tail)
     float fo[2][C];                                     // fo of the last two pieces (by piece parity)
@@ -1021,7 +1021,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         tc::tmem_wait_st();
         publish_smem();
 
-        // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T (3 split products;
+        // ---- product 2: [S~^T | O2] += Delta~^T [K' | P^T] (3 split products;
         // bar_s) ------------------------------------------------------------
         if (tid == ST_ISSUER) {
             state_product2(tmem, ST_COL_S, sm.dt[0], sm.dt[1], kp_hi, kp_lo, &sm.bar_s);
@@ -1109,7 +1109,7 @@ struct StSmemCompact {
     // S~^T hi / lo [v][k]; between product 1 and product 2 the first 32 KB
     // hold Delta~^T hi / lo [v][i]
     alignas(1024) unsigned char st[2][128 * 128 * 2];
-    alignas(1024) unsigned char rec[REC_A_BYTES];        // W hi, Q, W lo; then K'^T hi, P hi, K'^T lo, P lo
+    alignas(1024) unsigned char rec[REC_A_BYTES];        // [W^T hi | Q^T], W^T lo; then [K' | P^T] hi, lo
     alignas(16) float rec_s[REC_S_BYTES / 4];            // fo, gamma of the piece
     float fo[C];
     // products; copies of W / Q, K' / P, fo / gamma, and of the state at the start
@@ -1342,7 +1342,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
         const float cs_new = rescale ? 1.f : cn;
         publish_smem();
 
-        // ---- product 2: [S~^T | O2] += Delta~^T [K'^T; P]^T ----------------
+        // ---- product 2: [S~^T | O2] += Delta~^T [K' | P^T] -----------------
         wait_bar(&sm.bar_b, ph_b);
         if (!ok)
             break;
