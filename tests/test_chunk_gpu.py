@@ -205,6 +205,20 @@ def test_chunked_strided_views_of_packed_projections(sched):
     assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
 
 
+@pytest.mark.parametrize("lens", [[200, 37, 130, 64, 5] * 3, [int(x) for x in np.random.default_rng(71).integers(1, 65, 320)]],
+                         ids=["full_form", "compact_form"])
+def test_split_is_deterministic(lens):
+    """Five runs of the split schedule on the same inputs give the same bits
+    (no atomics or order-dependent sums in either kernel: a race between the
+    kernels' reuse of shared memory or TMEM would show here)."""
+    w = problem(lens, seed=72)
+    ref, _, _ = run_gpu(w, schedule=SPLIT)
+    for _ in range(4):
+        d, status, _ = run_gpu(w, schedule=SPLIT)
+        assert status == 0
+        assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
+
+
 def test_split_compact_many_short_sequences():
     """Enough short sequences (320 x 8 heads) that the split schedule runs its
     compact state kernel: empty sequences, padded slots, weak and strong
