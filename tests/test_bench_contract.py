@@ -1,0 +1,57 @@
+"""bench.py's command-line contract, on the CPU.
+
+The reference arm (the oracle on the host cores) prints the one JSON line the
+driver parses, with the keys the base contract and the reference arm require;
+the kernel-name mirror follows the library's documented choices (the names
+are what the bench line reports as the dominant kernel)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from gated_deltanet_recurrent_sigmoid_b200 import binding  # noqa: E402
+
+
+def test_reference_arm_prints_the_contract_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny_b4", "--steps", "2",
+                        "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "gpu_launches"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "tiny_b4" and d["value"] > 0 and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["gpu_launches"] == 0
+
+
+@pytest.mark.parametrize("one_token,pairs,mean,expected", [
+    (True, 4096, 1.0, "gdn::gdn_decode_kernel<128,128,64,4>"),                  # decode: 64x32
+    (False, 4096, 4.0, "gdn::gdn_decode_kernel<128,128,32,4>"),                 # many short chains: 32x32
+    (False, 1024, 4.0, "gdn::gdn_decode_kernel<128,128,16,8>"),                 # spec decode: 16x16
+    (False, 8, 29.0, "gdn::gdn_decode_kernel<128,128,8,16>"),                   # few chains: 8x8
+    (False, 8, 48.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
+    (False, 8192, 32.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_compact_kernel"),
+    (False, 512, 480.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
+])
+def test_kernel_name_mirrors_the_documented_choice(one_token, pairs, mean, expected):
+    assert bench.kernel_name(binding.SCHEDULE_AUTO, 0, 0, one_token, pairs, mean, chunk_ok=not one_token,
+                             sms=148) == expected
+
+
+def test_split_thresholds_match_the_header():
+    """The thresholds the bench mirrors are the ones the header documents."""
+    header = open(os.path.join(ROOT, "include", "gdn_decode.h")).read()
+    assert ">= 40 tokens" in header and ">= 30 (N * HV < 512) or >= 18" in header
+    assert [bench.chunked_min_mean_tokens(p) for p in (8, 63, 64, 511, 512, 8192)] == [40, 40, 30, 30, 18, 18]
