@@ -73,6 +73,17 @@ __device__ __forceinline__ void mma_tiles_bmn(uint32_t d, const unsigned char *a
                      idesc, (accumulate || s > 0) ? 1u : 0u);
 }
 
+// 2^x with the hardware approximation (PTX ex2.approx.ftz: a few ulp of
+// relative error; results below 2^-126 flush to zero), for the A and P
+// factors: values that small are far below what the fp32 products resolve,
+// and entries outside the masks are discarded by a select, whatever they are.
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 constexpr int K = 128;
 constexpr int V = 128;
 constexpr int C = 64;            // tokens per block
@@ -401,10 +412,10 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                     const int j0 = jb + 4 * e4;
                     const float4 u4 = *reinterpret_cast<const float4 *>(sm.ua + j0);
                     float4 a4;
-                    a4.x = (j0 > c && j0 < ce) ? kk16[4 * e4] * exp2f(u4.x - w) : 0.f;
-                    a4.y = (j0 + 1 > c && j0 + 1 < ce) ? kk16[4 * e4 + 1] * exp2f(u4.y - w) : 0.f;
-                    a4.z = (j0 + 2 > c && j0 + 2 < ce) ? kk16[4 * e4 + 2] * exp2f(u4.z - w) : 0.f;
-                    a4.w = (j0 + 3 > c && j0 + 3 < ce) ? kk16[4 * e4 + 3] * exp2f(u4.w - w) : 0.f;
+                    a4.x = (j0 > c && j0 < ce) ? kk16[4 * e4] * ex2_approx(u4.x - w) : 0.f;
+                    a4.y = (j0 + 1 > c && j0 + 1 < ce) ? kk16[4 * e4 + 1] * ex2_approx(u4.y - w) : 0.f;
+                    a4.z = (j0 + 2 > c && j0 + 2 < ce) ? kk16[4 * e4 + 2] * ex2_approx(u4.z - w) : 0.f;
+                    a4.w = (j0 + 3 > c && j0 + 3 < ce) ? kk16[4 * e4 + 3] * ex2_approx(u4.w - w) : 0.f;
                     *reinterpret_cast<float4 *>(At + c * A_LD + j0) = a4;
                 }
             }
@@ -420,7 +431,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = jb + 4 * e4 + e;
-                        pt[4 * e4 + e] = (j >= c && j < ce) ? pt[4 * e4 + e] * exp2f(uv[e] - w) : 0.f;
+                        pt[4 * e4 + e] = (j >= c && j < ce) ? pt[4 * e4 + e] * ex2_approx(uv[e] - w) : 0.f;
                     }
                 }
                 st_row8(rec + REC_KP_HI, c, K + jb, KP_COLS, pt, false);
