@@ -205,3 +205,31 @@ def test_host_step_rejects_missing_pointers(gdn_lib):
     st.host_in = st.dev_in = st.dev_out = st.host_out = ctypes.addressof(buf)
     st.ev_h2d = st.ev_ran = None
     assert gdn_lib.gdn_host_step_issue(ctypes.byref(st)) == binding.ERR_NULL_ARG
+
+
+def test_struct_layouts_match_the_c_header(tmp_path):
+    """Every field offset and struct size of the ctypes mirrors equals what a
+    C compiler makes of include/gdn_decode.h."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"gdn_tensor": binding.GdnTensor, "gdn_extra": binding.GdnExtra, "gdn_host_step": binding.GdnHostStep}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "gdn_decode.h"', "int main(void) {"]
+    for cname, py in structs.items():
+        lines.append(f'    printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'    printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
