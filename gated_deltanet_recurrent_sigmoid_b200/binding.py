@@ -37,7 +37,8 @@ OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5
 ERR_UNSUPPORTED, ERR_ARG, ERR_INDICES, ERR_CUDA = -6, -7, -8, -9
 ERR_SCRATCH = -10
-STATIC_SCRATCH_BYTES = 64 << 20     # gdn_decode_update_static_scratch's built-in array
+STATIC_SCRATCH_BYTES = 64 << 20     # gdn_decode_update_static_scratch's built-in array (checked
+                                    # against the library's gdn_static_scratch_bytes() by the tests)
 
 _DTYPE_CODES = {torch.bfloat16: 1, torch.float32: 2, torch.int32: 3}
 
@@ -104,6 +105,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_chunked_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
         lib.gdn_host_step_issue.restype = ctypes.c_int
         lib.gdn_host_step_issue.argtypes = [ctypes.POINTER(GdnHostStep)]
+        lib.gdn_static_scratch_bytes.restype = ctypes.c_uint64
+        lib.gdn_static_scratch_bytes.argtypes = []
         lib.gdn_decode_update_static_scratch.restype = ctypes.c_int
         lib.gdn_decode_update_static_scratch.argtypes = [P] * 11 + [ctypes.c_float, ctypes.c_uint32,
                                                                     ctypes.POINTER(GdnExtra)]

@@ -7,6 +7,7 @@
 // of the update's arithmetic; the kernel does all of it.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include <cmath>
@@ -167,6 +168,47 @@ bool stride_ok(int64_t extent, int64_t stride, int64_t multiple)
             return rc_;            \
     } while (0)
 
+// Workspace bytes of the split schedule for T_tot tokens and HV value heads
+// (both >= 0), saturating at UINT64_MAX instead of wrapping for sizes no
+// device could hold.
+uint64_t split_workspace_bytes(int64_t T_tot, int64_t HV)
+{
+    const uint64_t blocks = static_cast<uint64_t>((T_tot + gdn::split::C - 1) / gdn::split::C);
+    uint64_t recs = 0, bytes = 0;
+    if (__builtin_mul_overflow(blocks, static_cast<uint64_t>(HV), &recs) ||
+        __builtin_mul_overflow(recs, static_cast<uint64_t>(gdn::split::REC_BYTES), &bytes))
+        return UINT64_MAX;
+    return bytes;
+}
+
+// One-time set-up per device (shared-memory opt-ins, SM counts), safe when
+// several host threads make their first call on a device at once: the first
+// caller runs `init` under the lock; the flag is published with release
+// order after everything `init` wrote, so a thread that sees it set also
+// sees those writes.  A failed `init` leaves the flag clear (the next call
+// tries again).
+struct PerDevice {
+    static constexpr int kMaxDevices = 64;
+    std::mutex lock;
+    std::atomic<bool> ready[kMaxDevices] = {};
+};
+
+template <typename Init>
+cudaError_t once_per_device(PerDevice &pd, int dev, Init &&init)
+{
+    if (dev < 0 || dev >= PerDevice::kMaxDevices)
+        return cudaErrorInvalidDevice;
+    if (pd.ready[dev].load(std::memory_order_acquire))
+        return cudaSuccess;
+    std::lock_guard<std::mutex> guard(pd.lock);
+    if (pd.ready[dev].load(std::memory_order_relaxed))
+        return cudaSuccess;
+    const cudaError_t err = init();
+    if (err == cudaSuccess)
+        pd.ready[dev].store(true, std::memory_order_release);
+    return err;
+}
+
 // Host-side index check (GDN_CHECK_INDICES).
 int check_indices_on_host(const int32_t *d_idx, const int32_t *d_cu, int64_t N, int64_t num_slots,
                           int64_t T_tot, cudaStream_t stream)
@@ -234,21 +276,22 @@ cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t strea
 // memory opted in once per device.
 cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
 {
-    static bool ready[64][2];
+    static PerDevice once;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)
         return err;
-    if (dev < 0 || dev >= 64)
-        return cudaErrorInvalidDevice;
     const size_t smem = sizeof(gdn::chunk::Smem);
-    if (!ready[dev][l2norm]) {
-        err = cudaFuncSetAttribute(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (err != cudaSuccess)
-            return err;
-        ready[dev][l2norm] = true;
-    }
+    err = once_per_device(once, dev, [&]() {
+        cudaError_t e = cudaFuncSetAttribute(gdn::chunk::gdn_chunk_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::chunk::gdn_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem));
+        return e;
+    });
+    if (err != cudaSuccess)
+        return err;
     return launch_ex(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
                      dim3(static_cast<unsigned>(units)), dim3(gdn::chunk::THREADS), smem, stream, pdl, p);
 }
@@ -260,42 +303,40 @@ cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream
 cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t units, cudaStream_t stream,
                          bool pdl, bool l2norm)
 {
-    static bool ready[64];
-    static int sm_count[64];
+    static PerDevice once;
+    static int sm_count[PerDevice::kMaxDevices];      // written once per device, inside `once`
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)
         return err;
-    if (dev < 0 || dev >= 64)
-        return cudaErrorInvalidDevice;
     const size_t smem_wy = sizeof(gdn::split::WySmem), smem_st = sizeof(gdn::split::StSmem);
-    if (!ready[dev]) {
-        err = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem_wy));
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_wy));
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem_st));
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sizeof(gdn::split::StSmemCompact)));
+    err = once_per_device(once, dev, [&]() {
+        cudaError_t e = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_wy));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::split::gdn_chunk_wy_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_wy));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_st));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(sizeof(gdn::split::StSmemCompact)));
         // the largest shared-memory carveout, so that four block-kernel CTAs
         // (two compact state-kernel CTAs) fit on an SM
-        for (int l2 = 0; l2 < 2 && err == cudaSuccess; ++l2)
-            err = cudaFuncSetAttribute(l2 ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
-                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
-                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (err == cudaSuccess)
-            err = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (err != cudaSuccess)
-            return err;
-        ready[dev] = true;
-    }
+        for (int l2 = 0; l2 < 2 && e == cudaSuccess; ++l2)
+            e = cudaFuncSetAttribute(l2 ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
+                                     cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
+                                     cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+        return e;
+    });
+    if (err != cudaSuccess)
+        return err;
     const int64_t blocks = (static_cast<int64_t>(p.T_tot) + gdn::split::C - 1) / gdn::split::C * p.HV;
     err = launch_ex(l2norm ? gdn::split::gdn_chunk_wy_kernel<true> : gdn::split::gdn_chunk_wy_kernel<false>,
                     dim3(static_cast<unsigned>(blocks)), dim3(gdn::split::THREADS), smem_wy, stream, pdl, p, ws);
@@ -330,35 +371,27 @@ cudaError_t launch_tile(const gdn::DecodeParams &p, int64_t units, cudaStream_t 
 
 constexpr int kPipeStages = 3;
 
-// Per-device one-time setup of the pipelined kernel: its dynamic shared
-// memory opt-in and the SM count that sizes its persistent grid.
-struct PipeDevice {
-    int sms = 0;
-    bool ready = false;
-};
-
 cudaError_t launch_pipelined(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl)
 {
-    static PipeDevice devices[64];
+    // per device, once: the dynamic shared memory opt-in and the SM count
+    // that sizes the persistent grid
+    static PerDevice once;
+    static int sms[PerDevice::kMaxDevices];           // written once per device, inside `once`
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)
         return err;
-    if (dev < 0 || dev >= 64)
-        return cudaErrorInvalidDevice;
     const size_t smem = sizeof(gdn::pipe::Smem<kPipeStages>);
-    PipeDevice &d = devices[dev];
-    if (!d.ready) {
-        err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        if (err != cudaSuccess)
-            return err;
-        err = cudaFuncSetAttribute(gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (err != cudaSuccess)
-            return err;
-        d.ready = true;
-    }
-    const int64_t grid = units < d.sms ? units : d.sms;
+    err = once_per_device(once, dev, [&]() {
+        cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        return e;
+    });
+    if (err != cudaSuccess)
+        return err;
+    const int64_t grid = units < sms[dev] ? units : sms[dev];
     return launch_ex(gdn::pipe::gdn_decode_pipelined_kernel<kPipeStages>, dim3(static_cast<unsigned>(grid)),
                      dim3(gdn::pipe::THREADS), smem, stream, pdl, p);
 }
@@ -553,7 +586,7 @@ int run_update(const UpdateArgs &c)
                 return GDN_ERR_ALIAS;
         }
     }
-    const bool ws_fits = ws && ws_bytes >= gdn::split::workspace_bytes(T_tot, HV);
+    const bool ws_fits = ws && ws_bytes >= split_workspace_bytes(T_tot, HV);
     if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT && !ws)
         return GDN_ERR_NULL_ARG;
     if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT && !ws_fits)
@@ -711,11 +744,13 @@ extern "C" {
 
 GDN_API int gdn_version(void) { return GDN_DECODE_ABI_VERSION; }
 
+GDN_API uint64_t gdn_static_scratch_bytes(void) { return GDN_STATIC_SCRATCH_BYTES; }
+
 GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV)
 {
     if (T_tot <= 0 || HV <= 0)
         return 0;
-    return gdn::split::workspace_bytes(T_tot, HV);
+    return split_workspace_bytes(T_tot, HV);
 }
 
 GDN_API const char *gdn_status_string(int status)
@@ -844,22 +879,33 @@ static __device__ __align__(256) unsigned char g_static_scratch[GDN_STATIC_SCRAT
 
 namespace {
 
-// Device address of g_static_scratch on the current device, looked up on the
-// first call there.  Returns nullptr (and the CUDA error in *err) on failure.
-void *static_scratch_address(cudaError_t *err)
+// Device address of g_static_scratch on the current device.  The address
+// belongs to the module the CUDA runtime loaded into the device's current
+// context, and a context that is torn down and created again (e.g. after
+// cudaDeviceReset) loads the module afresh, possibly elsewhere: so every call
+// outside stream capture looks the address up again (a host-side table
+// lookup once the module is loaded) and records it; a call made while its
+// stream is capturing uses the address recorded by the last call on this
+// device outside capture (capture must not load modules).  Returns nullptr
+// (and the CUDA error in *err) on failure.
+void *static_scratch_address(cudaStream_t stream, cudaError_t *err)
 {
     static std::mutex lock;
-    static void *addr[64];
+    static void *addr[PerDevice::kMaxDevices];
     int dev = 0;
     *err = cudaGetDevice(&dev);
     if (*err != cudaSuccess)
         return nullptr;
-    if (dev < 0 || dev >= 64) {
+    if (dev < 0 || dev >= PerDevice::kMaxDevices) {
         *err = cudaErrorInvalidDevice;
         return nullptr;
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    // the legacy stream cannot be queried while another stream captures
+    // (an error): treat that as capturing
+    const bool capturing = cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
     std::lock_guard<std::mutex> guard(lock);
-    if (!addr[dev]) {
+    if (!capturing || !addr[dev]) {
         void *ptr = nullptr;
         *err = cudaGetSymbolAddress(&ptr, g_static_scratch);
         if (*err != cudaSuccess)
@@ -885,19 +931,24 @@ GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tens
     if (extra && (extra->workspace || extra->workspace_bytes ||
                   (extra->schedule != GDN_SCHEDULE_AUTO && extra->schedule != GDN_SCHEDULE_CHUNKED_SPLIT)))
         return GDN_ERR_ARG;
-    // size check first: T_tot = all leading dims of v, HV = its second-to-last
+    // size check first: T_tot = all leading dims of v, HV = its second-to-last.
+    // Each dim is checked before it enters a product, so hostile shapes cannot
+    // overflow it (T_tot <= INT32_MAX^2 fits in int64_t).
     if (v->ndim < 2 || v->ndim > 4)
         return GDN_ERR_SHAPE;
     int64_t T_tot = 1;
-    for (int d = 0; d < v->ndim - 2; ++d)
+    for (int d = 0; d < v->ndim - 2; ++d) {
+        if (v->shape[d] < 0 || v->shape[d] > INT32_MAX || (d > 0 && T_tot > INT32_MAX))
+            return GDN_ERR_SHAPE;
         T_tot *= v->shape[d];
+    }
     const int64_t HV = v->shape[v->ndim - 2];
-    if (T_tot < 0 || HV < 0)
+    if (T_tot > INT32_MAX || HV < 0 || HV > INT32_MAX)
         return GDN_ERR_SHAPE;
-    if (T_tot > 0 && HV > 0 && gdn::split::workspace_bytes(T_tot, HV) > GDN_STATIC_SCRATCH_BYTES)
+    if (T_tot > 0 && HV > 0 && split_workspace_bytes(T_tot, HV) > GDN_STATIC_SCRATCH_BYTES)
         return GDN_ERR_SCRATCH;
     cudaError_t err = cudaSuccess;
-    void *scratch = static_scratch_address(&err);
+    void *scratch = static_scratch_address(extra ? static_cast<cudaStream_t>(extra->stream) : nullptr, &err);
     if (!scratch)
         return GDN_ERR_CUDA;
     gdn_extra x;

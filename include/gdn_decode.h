@@ -210,7 +210,6 @@ GDN_API int gdn_decode_update(const gdn_tensor *q, const gdn_tensor *k, const gd
                       const gdn_tensor *cu_seqlens, const gdn_tensor *out,
                       float scale, uint32_t flags, const gdn_extra *extra);
 
-/* Static text for a gdn_status value (never NULL). */
 /*
  * The recurrence of the unfused pair: the pages name the two kernels the
  * fused op replaces, fused_gdn_gating then fused_recurrent_gated_delta_rule
@@ -248,6 +247,8 @@ GDN_API int gdn_gating(const gdn_tensor *A_log, const gdn_tensor *a, const gdn_t
                        const gdn_tensor *b, const gdn_tensor *g, const gdn_tensor *beta,
                        const gdn_extra *extra);
 
+/* Static text for a gdn_status value (never NULL; "unknown gdn status" for
+   a value that is not one). */
 GDN_API const char *gdn_status_string(int status);
 
 /* GDN_DECODE_ABI_VERSION of the loaded library. */
@@ -257,12 +258,16 @@ GDN_API int gdn_version(void);
  * Bytes of workspace GDN_SCHEDULE_CHUNKED_SPLIT needs for a call with T_tot
  * tokens and HV value heads (K = V = 128): one 131,584-byte record per
  * (64-token block of the packed token range, value head).  0 for T_tot <= 0
- * or HV <= 0.  Host-only arithmetic, no CUDA call.
+ * or HV <= 0; UINT64_MAX when the size does not fit in 64 bits.  Host-only
+ * arithmetic, no CUDA call.
  */
 GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV);
 
 /* Size of the library's built-in scratch array (64 MiB; see below). */
 #define GDN_STATIC_SCRATCH_BYTES (64ull << 20)
+
+/* GDN_STATIC_SCRATCH_BYTES of the loaded library (host-only, no CUDA call). */
+GDN_API uint64_t gdn_static_scratch_bytes(void);
 
 /*
  * gdn_decode_update on the split chunked schedule, with NO device allocation
@@ -290,9 +295,18 @@ GDN_API uint64_t gdn_chunked_workspace_bytes(int64_t T_tot, int64_t HV);
  *     every workspace byte it reads before reading it), but two calls that
  *     can overlap on the GPU (different streams, or different host threads,
  *     on the same device) race on it: order such calls, e.g. on one stream;
- *   - the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
+ *   - the array's device address is looked up (cudaGetSymbolAddress, with
+ *     the call's device current) on every call whose stream is not
+ *     capturing, so it follows the module if the device's context is torn
+ *     down and created again; a call inside a stream capture reuses the
+ *     address found by the last call on that device outside capture.  The
+ *     first call on a device may load the library's module there: make it
  *     before any stream capture on the device.
+ *   - sizes are checked before anything else: a shape whose dims exceed
+ *     INT32_MAX returns GDN_ERR_SHAPE, a call too large for the array
+ *     GDN_ERR_SCRATCH, and a non-NULL extra->workspace, a nonzero
+ *     extra->workspace_bytes or a schedule other than 0 /
+ *     GDN_SCHEDULE_CHUNKED_SPLIT GDN_ERR_ARG, all before any CUDA call.
  * The library allocates no device memory for this call.
  */
 GDN_API int gdn_decode_update_static_scratch(const gdn_tensor *q, const gdn_tensor *k, const gdn_tensor *v,

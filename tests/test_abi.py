@@ -25,7 +25,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     assert set(declared_functions()) == {"gdn_decode_update", "gdn_recurrent_update", "gdn_gating",
                                          "gdn_status_string", "gdn_version", "gdn_chunked_workspace_bytes",
-                                         "gdn_decode_update_static_scratch", "gdn_host_step_issue"}
+                                         "gdn_decode_update_static_scratch", "gdn_host_step_issue",
+                                         "gdn_static_scratch_bytes"}
 
 
 def test_library_exports_every_declared_symbol(gdn_lib):
@@ -233,3 +234,58 @@ def test_struct_layouts_match_the_c_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_static_scratch_size_matches_binding(gdn_lib):
+    """The binding's constant equals the array size the library was built
+    with (gdn_static_scratch_bytes) and the header's #define."""
+    assert gdn_lib.gdn_static_scratch_bytes() == binding.STATIC_SCRATCH_BYTES
+    m = re.search(r"#define GDN_STATIC_SCRATCH_BYTES \((\d+)ull << (\d+)\)", open(HEADER).read())
+    assert int(m.group(1)) << int(m.group(2)) == binding.STATIC_SCRATCH_BYTES
+
+
+def _static_call(gdn_lib, t, extra=None):
+    descs = [binding.describe(t[n]) for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias", "state_pool",
+                                                "state_indices", "cu_seqlens", "out")]
+    return gdn_lib.gdn_decode_update_static_scratch(*[binding._ref(d) for d in descs], ctypes.c_float(0.088),
+                                                    ctypes.c_uint32(binding.L2NORM_QK),
+                                                    ctypes.byref(extra) if extra is not None else None)
+
+
+def test_static_scratch_guards_run_before_any_cuda_call(gdn_lib):
+    """gdn_decode_update_static_scratch rejects a caller workspace, a nonzero
+    workspace size, a schedule other than AUTO / CHUNKED_SPLIT, a call too
+    large for its array and hostile shapes -- all before any CUDA call (so
+    on this GPU-less host), leaving `out` untouched."""
+    for field, value in [("workspace", 256), ("workspace_bytes", 4096),
+                         ("schedule", binding.SCHEDULE_PER_TILE), ("schedule", binding.SCHEDULE_CHUNKED),
+                         ("schedule", 9)]:
+        t = make(N=2, T=3)
+        t["out"].fill_(7.0)
+        extra = binding.GdnExtra()
+        setattr(extra, field, value)
+        assert _static_call(gdn_lib, t, extra) == binding.ERR_ARG, (field, value)
+        assert bool((t["out"] == 7.0).all())
+    # 4160 tokens x 8 heads need 520 records > the 510 that fit in 64 MiB:
+    # strides of zero give a large shape with no storage behind it
+    T, H, HV = 4160, 4, 8
+    assert binding.chunked_workspace_bytes(T, HV) > binding.STATIC_SCRATCH_BYTES
+    t = make(N=2, T=3, H=H, HV=HV)
+    t["v"] = torch.zeros(1, HV, 128, dtype=torch.bfloat16).expand(T, HV, 128)
+    assert _static_call(gdn_lib, t) == binding.ERR_SCRATCH
+    # leading dims whose product overflows 64 bits are a shape error, not a
+    # wrapped size that slips past the check
+    d = binding.describe(torch.zeros(1, 1, HV, 128, dtype=torch.bfloat16))
+    for shape in [(1 << 40, 1 << 40), (-1, 4), (1 << 31, 1), (65536, 65536)]:
+        d.shape[0], d.shape[1] = shape
+        descs = [binding.describe(t[n]) for n in ("q", "k")] + [d] + \
+                [binding.describe(t[n]) for n in ("a", "b", "A_log", "dt_bias", "state_pool", "state_indices",
+                                                  "cu_seqlens", "out")]
+        rc = gdn_lib.gdn_decode_update_static_scratch(*[ctypes.byref(x) for x in descs], ctypes.c_float(0.088),
+                                                      ctypes.c_uint32(1), None)
+        assert rc == binding.ERR_SHAPE, shape
+
+
+def test_chunked_workspace_bytes_saturates(gdn_lib):
+    assert binding.chunked_workspace_bytes(1 << 62, 1 << 30) == (1 << 64) - 1
+    assert binding.chunked_workspace_bytes((1 << 31) - 1, (1 << 31) - 1) == (1 << 64) - 1
