@@ -107,3 +107,67 @@ def assert_state_close(s_gpu: np.ndarray, s_ref: np.ndarray, what="state"):
     err = np.abs(s_gpu.astype(np.float64) - s_ref)
     assert np.isfinite(s_gpu).all(), f"{what}: non-finite values"
     assert err.max() <= STATE_ATOL, f"{what}: max abs err {err.max():.3e} > {STATE_ATOL}"
+
+
+def max_errors(o_gpu: np.ndarray, o_ref: np.ndarray, s_gpu=None, s_ref=None) -> dict:
+    """Largest output and state errors of a comparison (for the drift log)."""
+    o_gpu = o_gpu.reshape(o_ref.shape).astype(np.float64)
+    written = ~np.isnan(o_ref)
+    res = {"out": float(np.abs(o_gpu - o_ref)[written].max()) if written.any() else 0.0}
+    if s_gpu is not None and s_ref is not None and np.size(s_ref):
+        res["state"] = float(np.abs(s_gpu.astype(np.float64) - s_ref).max())
+    return res
+
+
+def log_errors(case: str, **fields) -> None:
+    """Append one case's largest errors to the JSON-lines file named by the
+    GDN_PARITY_LOG environment variable (nothing when it is unset): the
+    record of how far from the tolerances each long-sequence case lands."""
+    import json
+    import os
+    path = os.environ.get("GDN_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, **fields}) + "\n")
+
+
+def oracle_chain(steps, pool0: np.ndarray, flags=oracle.L2NORM_QK):
+    """The oracle over successive calls that share one fp32 state pool: each
+    step's inputs are a dict of oracle arrays (without state_pool); the pool
+    after a step is rounded to fp32, as the library stores it, before the
+    next step reads it.  Returns (outputs per step, pool after the last step
+    in fp64)."""
+    pool = np.ascontiguousarray(pool0, dtype=np.float32)
+    outs, s_ref = [], pool.astype(np.float64)
+    for arrays in steps:
+        st, o_ref, s_ref, _ = oracle.update(arrays["q"], arrays["k"], arrays["v"], arrays["a"], arrays["b"],
+                                            arrays["A_log"], arrays["dt_bias"], pool, arrays["state_indices"],
+                                            arrays.get("cu_seqlens"), flags=flags)
+        assert st == 0
+        outs.append(o_ref)
+        pool = s_ref.astype(np.float32)
+    return outs, s_ref
+
+
+def workload_arrays(w: Workload) -> dict:
+    """A workload's inputs as the oracle takes them (pool excluded)."""
+    return dict(q=w.q, k=w.k, v=w.v, a=w.a, b=w.b, A_log=w.A_log, dt_bias=w.dt_bias,
+                state_indices=w.state_indices, cu_seqlens=w.cu_seqlens)
+
+
+def random_workload(lens, H, HV, seed, weak_heads=(), pad=()) -> Workload:
+    """A random problem with the workloads' distributions and the given
+    sequence lengths (K = V = 128); value heads in `weak_heads` get
+    A_log = -9 (decay within 1e-4 of 1 per token)."""
+    from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl
+    from helpers import random_problem
+    rng = np.random.default_rng(seed)
+    p = random_problem(rng, lens=lens, H=H, HV=HV, K=128, V=128, pad=pad)
+    spec = wl.WorkloadSpec(f"random_{len(lens)}x{max(lens)}", N=len(lens), H=H, HV=HV,
+                           num_slots=p["state_pool"].shape[0], seed=seed, T=None)
+    w = Workload(spec, p["q"], p["k"], p["v"], p["a"], p["b"], p["A_log"], p["dt_bias"], p["state_pool"],
+                 p["state_indices"], p["cu_seqlens"])
+    w.A_log = w.A_log.copy()
+    for h in weak_heads:
+        w.A_log[h] = -9.0
+    return w

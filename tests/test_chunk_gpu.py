@@ -11,8 +11,8 @@ import torch
 import oracle
 from gated_deltanet_recurrent_sigmoid_b200 import binding
 from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl
-from gpu_helpers import (assert_out_close, assert_state_close, oracle_on, out_as_f32, run_gpu, run_oracle,
-                         sample_subproblem, to_device)
+from gpu_helpers import (assert_out_close, assert_state_close, oracle_chain, oracle_on, out_as_f32, run_gpu,
+                         run_oracle, sample_subproblem, to_device, workload_arrays)
 from helpers import random_problem
 
 pytestmark = pytest.mark.gpu
@@ -183,8 +183,9 @@ def test_auto_schedule_picks_chunked_for_long_sequences():
 
 def test_chunked_strided_views_of_packed_projections(sched):
     """q, k, v as column slices of one packed projection row (token stride
-    wider than a head's row) and a, b interleaved per value head: the same
-    bits as contiguous inputs, on both chunked schedules."""
+    wider than a head's row) and a, b interleaved per value head: the
+    oracle's results, and the same bits as contiguous inputs, on both
+    chunked schedules."""
     w = problem([200, 37, 130, 64, 5], seed=61)
     ref, _, _ = run_gpu(w, schedule=sched)
     d = to_device(w)
@@ -202,6 +203,11 @@ def test_chunked_strided_views_of_packed_projections(sched):
     binding.decode_update(q, k, v, a, b, d["A_log"], d["dt_bias"], d["state_pool"], d["state_indices"],
                           d["cu_seqlens"], d["out"], schedule=sched)
     torch.cuda.synchronize()
+    ost, o_ref, s_ref, _ = run_oracle(w)
+    assert ost == 0
+    assert_out_close(out_as_f32(d["out"]), o_ref, "strided out")
+    live = w.state_indices[w.state_indices >= 0]
+    assert_state_close(d["state_pool"].cpu().numpy()[live], s_ref[live], "strided state")
     assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
 
 
@@ -242,7 +248,8 @@ def _args(d):
 def test_split_graph_capture_and_pdl_chain():
     """The split schedule (two kernels) captures in a CUDA graph and chains
     with programmatic dependent launch: two chained calls replayed from a
-    graph, and two chained PDL calls, give the bits of two eager calls."""
+    graph, and two chained PDL calls, match two chained oracle calls and give
+    the bits of two eager calls."""
     w = problem([150, 40, 90], seed=51)
     eager = to_device(w)
     for _ in range(2):
@@ -269,9 +276,16 @@ def test_split_graph_capture_and_pdl_chain():
     assert torch.equal(d["out"], eager["out"]) and torch.equal(d["state_pool"], eager["state_pool"])
 
     p = to_device(w)
-    for _ in range(2):
-        binding.decode_update(*_args(p), schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
+    first = torch.empty_like(p["out"])
+    binding.decode_update(*_args(p)[:-1], first, schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
+    binding.decode_update(*_args(p), schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
     torch.cuda.synchronize()
+    o_refs, s_ref = oracle_chain([workload_arrays(w)] * 2, w.state_pool)
+    live = w.state_indices[w.state_indices >= 0]
+    for name, got in (("graph", d), ("pdl", p)):
+        assert_out_close(out_as_f32(got["out"]), o_refs[1], f"{name} chain out")
+        assert_state_close(got["state_pool"].cpu().numpy()[live], s_ref[live], f"{name} chain state")
+    assert_out_close(out_as_f32(first), o_refs[0], "pdl chain first out")
     assert torch.equal(p["out"], eager["out"]) and torch.equal(p["state_pool"], eager["state_pool"])
 
 

@@ -1,0 +1,116 @@
+"""Long sequences against the oracle: every schedule at prefill lengths.
+
+The per-token kernels carry the state in fp32 registers (scaled by a running
+decay factor that is renormalised when it leaves [2^-60, 2^60]) across the
+whole sequence; the chunked kernels carry it through tensor memory as bf16
+hi / lo operand pairs, 64 tokens at a time.  Rounding accumulates with the
+length, so these cases run sequences of 200 to 2,048 tokens -- the prefill
+lengths of the chunked workload ("sglang PR #21411 summary", 实现拆解:
+chunked prefill, CHUNK_SIZE 64) and the long end of the per-token paths
+("vLLM PR #35777 summary", 实现拆解: spec / non-spec paths) -- with weak
+decay (A_log = -9: e^g within 1e-4 of 1, so the state keeps everything it
+has seen) beside the workloads' strong decays, at the same tolerances as
+every other parity test: state max abs 1e-4, output 1e-2 + 1e-2 |o_ref|.
+
+With GDN_PARITY_LOG=<path> each case appends its largest errors to <path>.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_recurrent_sigmoid_b200 import binding
+from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl
+from gpu_helpers import (assert_out_close, assert_state_close, log_errors, max_errors, oracle_on, out_as_f32,
+                         random_workload, run_gpu, run_oracle, sample_subproblem)
+
+pytestmark = pytest.mark.gpu
+
+L2 = binding.L2NORM_QK
+INTER = binding.WRITE_INTERMEDIATE
+PER_TILE = binding.SCHEDULE_PER_TILE
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(gdn_lib):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return gdn_lib
+
+
+def check_whole(w, name, flags=L2, **kw):
+    """Whole-problem comparison (outputs, every written slot, intermediates)."""
+    inter = bool(flags & INTER)
+    d, status, inter_t = run_gpu(w, flags=flags, inter=inter, **kw)
+    ost, o_ref, s_ref, i_ref = run_oracle(w, flags=flags)
+    assert status == ost == 0
+    o_gpu = out_as_f32(d["out"])
+    assert_out_close(o_gpu, o_ref)
+    pool = d["state_pool"].cpu().numpy()
+    live = w.state_indices[(w.state_indices >= 0) & (w.seq_lens > 0)]
+    untouched = np.ones(w.spec.num_slots, bool)
+    untouched[live] = False
+    assert np.array_equal(pool[untouched], w.state_pool[untouched])
+    assert_state_close(pool[live], s_ref[live])
+    errs = max_errors(o_gpu, o_ref, pool[live], s_ref[live])
+    if inter:
+        it = inter_t.cpu().numpy()
+        del inter_t
+        nan_ref = np.isnan(i_ref)
+        assert np.array_equal(np.isnan(it), nan_ref), "intermediate rows written differ"
+        assert_state_close(it[~nan_ref], i_ref[~nan_ref], "intermediate")
+        errs["intermediate"] = float(np.abs(it[~nan_ref].astype(np.float64) - i_ref[~nan_ref]).max())
+    log_errors(name, lens=[int(x) for x in w.seq_lens], **errs)
+    return errs
+
+
+# per-token kernel forced, two tiles; one weak and one strong head per key head
+@pytest.mark.parametrize("tile", [(16, 16), (32, 32)], ids=["tile16x16", "tile32x32"])
+def test_per_tile_long_sequences(tile):
+    w = random_workload([2048, 700, 200, 1], H=2, HV=4, seed=101, weak_heads=(0, 2))
+    check_whole(w, f"per_tile_{tile[0]}x{tile[1]}", schedule=PER_TILE, tile_v=tile[0], tile_rows=tile[1])
+
+
+def test_auto_with_intermediates_long_sequences():
+    """GDN_WRITE_INTERMEDIATE keeps AUTO on the per-token kernel at any
+    length: every token's state is compared, up to 2,048 tokens."""
+    w = random_workload([2048, 300], H=1, HV=2, seed=102, weak_heads=(0,))
+    check_whole(w, "auto_intermediate", flags=L2 | INTER)
+
+
+def test_auto_without_workspace_short_mean_long_sequence():
+    """Without a workspace AUTO keeps the per-token kernel below 128 tokens
+    per sequence on average, so one 2,048-token sequence among short ones
+    runs there."""
+    lens = [2048] + [3, 9, 17, 1, 30] * 6
+    w = random_workload(lens, H=2, HV=4, seed=103, weak_heads=(1, 3), pad=(4,))
+    check_whole(w, "auto_no_workspace_per_tile", workspace=None)
+
+
+@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT],
+                         ids=["single", "split"])
+def test_chunked_long_weak_decay(sched):
+    """The chunked schedules at 2,048 tokens with weak and strong heads, whole."""
+    w = random_workload([2048, 1500, 64, 65], H=2, HV=4, seed=104, weak_heads=(0, 3))
+    check_whole(w, f"chunked_{sched}", schedule=sched)
+
+
+@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT],
+                         ids=["single", "split"])
+def test_prefill_b8_t2k_sampled(sched):
+    """The full prefill workload (8 sequences of 1-2K tokens) in the
+    benchmark's configuration; the oracle recomputes three sequences, the
+    longest among them."""
+    w = wl.generate(wl.PREFILL_B8)
+    d, status, _ = run_gpu(w, schedule=sched)
+    assert status == 0
+    order = np.argsort(-w.seq_lens, kind="stable")
+    seqs = np.sort(np.array([order[0], order[len(order) // 2], order[-1]]))
+    arrays, rows, slots = sample_subproblem(w, seqs)
+    _, o_ref, s_ref, _ = oracle_on(arrays)
+    out = d["out"].view(w.T_tot, w.spec.HV, w.spec.V)
+    o_gpu = out[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    assert_out_close(o_gpu, o_ref, "sampled out")
+    live = slots >= 0
+    got = d["state_pool"][torch.from_numpy(slots[live].astype(np.int64)).cuda()].cpu().numpy()
+    assert_state_close(got, s_ref, "sampled state")
+    log_errors(f"prefill_b8_t2k_{sched}", lens=[int(x) for x in w.seq_lens[seqs]],
+               **max_errors(o_gpu, o_ref, got, s_ref))

@@ -12,8 +12,8 @@ import torch
 import oracle
 from gated_deltanet_recurrent_sigmoid_b200 import binding
 from gated_deltanet_recurrent_sigmoid_b200 import workloads as wl
-from gpu_helpers import (assert_out_close, assert_state_close, bf16_tensor, oracle_on, out_as_f32,
-                         run_gpu, run_oracle, sample_subproblem, to_device)
+from gpu_helpers import (assert_out_close, assert_state_close, bf16_tensor, oracle_chain, oracle_on, out_as_f32,
+                         run_gpu, run_oracle, sample_subproblem, to_device, workload_arrays)
 from helpers import BF16_NEG_INF, BF16_POS_INF, bf16, random_problem
 
 pytestmark = pytest.mark.gpu
@@ -244,6 +244,11 @@ def test_strided_views_of_packed_projections():
     binding.decode_update(q, k, v, a, b, d["A_log"], d["dt_bias"], d["state_pool"], d["state_indices"],
                           d["cu_seqlens"], d["out"])
     torch.cuda.synchronize()
+    ost, o_ref, s_ref, _ = run_oracle(w)
+    assert ost == 0
+    assert_out_close(out_as_f32(d["out"]), o_ref, "strided out")
+    live = w.state_indices[w.state_indices >= 0]
+    assert_state_close(d["state_pool"].cpu().numpy()[live], s_ref[live], "strided state")
     assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
 
 
@@ -382,6 +387,11 @@ def test_host_staged_decode_matches_device_call(spec):
             getattr(staged, name).copy_(d[name].cpu())
     out = staged.step()
     torch.cuda.synchronize()
+    ost, o_ref, s_ref, _ = run_oracle(w)
+    assert ost == 0
+    assert_out_close(out.float().numpy(), o_ref, "host-staged out")
+    live = w.state_indices[w.state_indices >= 0]
+    assert_state_close(d["state_pool"].cpu().numpy()[live], s_ref[live], "host-staged state")
     assert torch.equal(out, ref["out"].cpu())
     assert torch.equal(d["state_pool"], ref["state_pool"])
     assert staged.h2d_bytes >= sum(d[n].numel() * d[n].element_size() for n in ("q", "k", "v", "a", "b"))
@@ -393,8 +403,9 @@ def test_host_staged_decode_matches_device_call(spec):
 def test_pipelined_host_decode_matches_device_calls(spec, depth):
     """Five host-fed steps with different inputs, copies overlapped across
     steps (2, 3 or 4 slots in flight): every step's host output and the final
-    pool are the bits of the same five steps run as device-resident calls, in
-    order."""
+    pool match five chained oracle calls (each reading the pool the previous
+    one left), and are the bits of the same five steps run as
+    device-resident calls, in order."""
     ws = [wl.generate(dataclasses.replace(spec, seed=spec.seed + 100 * n)) for n in range(5)]
     ref = to_device(ws[0])
     ref_outs = []
@@ -421,6 +432,12 @@ def test_pipelined_host_decode_matches_device_calls(spec, depth):
     outs.extend(o.clone() for o in pipe.finish())
     torch.cuda.synchronize()
     assert len(outs) == len(ref_outs)
+    steps = [dict(workload_arrays(w), A_log=ws[0].A_log, dt_bias=ws[0].dt_bias) for w in ws]
+    o_refs, s_ref = oracle_chain(steps, ws[0].state_pool)
+    for n, (got, o_ref) in enumerate(zip(outs, o_refs)):
+        assert_out_close(got.float().numpy(), o_ref, f"pipelined step {n} out")
+    touched = np.unique(np.concatenate([w.state_indices[w.state_indices >= 0] for w in ws]))
+    assert_state_close(d0["state_pool"].cpu().numpy()[touched], s_ref[touched], "pipelined final state")
     for got, exp in zip(outs, ref_outs):
         assert torch.equal(got, exp)
     assert torch.equal(d0["state_pool"], ref["state_pool"])
@@ -429,7 +446,8 @@ def test_pipelined_host_decode_matches_device_calls(spec, depth):
 @pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
 def test_cuda_graph_capture_replays_the_same_update(kernel):
     """The launch is capturable: a graph of two chained updates replays to
-    the same bits as the same two updates run eagerly."""
+    two chained oracle calls, and to the bits of the same two updates run
+    eagerly."""
     w = wl.generate(wl.shrink(wl.SPEC_B128_T4, 12))
     kw = kw_of(kernel)
     eager = to_device(w)
@@ -455,22 +473,37 @@ def test_cuda_graph_capture_replays_the_same_update(kernel):
     torch.cuda.synchronize()
     graph.replay()
     torch.cuda.synchronize()
+    o_refs, s_ref = oracle_chain([workload_arrays(w)] * 2, w.state_pool)
+    assert_out_close(out_as_f32(d["out"]), o_refs[1], "graph replay out")
+    live = w.state_indices[w.state_indices >= 0]
+    assert_state_close(d["state_pool"].cpu().numpy()[live], s_ref[live], "graph replay state")
     assert torch.equal(d["out"], eager["out"]) and torch.equal(d["state_pool"], eager["state_pool"])
 
 
 @pytest.mark.parametrize("kernel", MAIN, ids=MAIN_IDS)
 def test_programmatic_dependent_launch_keeps_results(kernel):
     """With GDN_LAUNCH_PDL every launch still waits for the previous kernel
-    before reading: a chain of launches over the same pool (each reads the
-    state the previous one wrote) equals the chain without PDL."""
+    before reading: a chain of six launches over the same pool (each reads
+    the state the previous one wrote) matches six chained oracle calls, step
+    by step, and equals the chain without PDL bit for bit."""
     w = wl.generate(wl.shrink(wl.DECODE_B512, 200))
     kw = kw_of(kernel)
+    steps = 6
     results = []
     for flags in (L2, L2 | binding.LAUNCH_PDL):
         d = to_device(w)
-        for _ in range(6):
+        outs = [torch.empty_like(d["out"]) for _ in range(steps)]
+        for o in outs:
             binding.decode_update(d["q"], d["k"], d["v"], d["a"], d["b"], d["A_log"], d["dt_bias"],
-                                  d["state_pool"], d["state_indices"], d["cu_seqlens"], d["out"], flags=flags, **kw)
+                                  d["state_pool"], d["state_indices"], d["cu_seqlens"], o, flags=flags, **kw)
         torch.cuda.synchronize()
-        results.append((d["out"].clone(), d["state_pool"].clone()))
-    assert torch.equal(results[0][0], results[1][0]) and torch.equal(results[0][1], results[1][1])
+        results.append(([o.clone() for o in outs], d["state_pool"].clone()))
+    o_refs, s_ref = oracle_chain([workload_arrays(w)] * steps, w.state_pool)
+    outs, pool = results[1]
+    for n in range(steps):
+        assert_out_close(out_as_f32(outs[n]), o_refs[n], f"PDL chain step {n} out")
+    live = w.state_indices[w.state_indices >= 0]
+    assert_state_close(pool.cpu().numpy()[live], s_ref[live], "PDL chain state")
+    for a_, b_ in zip(results[0][0], results[1][0]):
+        assert torch.equal(a_, b_)
+    assert torch.equal(results[0][1], results[1][1])
