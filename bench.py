@@ -323,6 +323,8 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
     if schedule == binding.SCHEDULE_CHUNKED:
         return "gdn::chunk::gdn_chunk_kernel<true>"
+    if schedule == binding.SCHEDULE_CHUNKED_LOCAL:
+        return "gdn::local::gdn_chunk_local_kernel<true>"
     if tile_v:
         bv, rows = tile_v, tile_rows or 16
     else:
@@ -355,6 +357,83 @@ def device_copy(w, torch, device):
     return d
 
 
+# the other workload families, timed after the headline one (per_config)
+PER_CONFIG = [wl.TINY.name, wl.FULLHEAD_B256.name, wl.SPEC_B128_T4.name] + [wl.sweep_spec(n).name
+                                                                             for n in wl.SWEEP_NS]
+L2_FLUSH_BYTES = 256 << 20     # twice the B200's 126 MB L2
+
+
+def oracle_sample_us(w, rng, max_seqs=16):
+    """The oracle (single thread, fp64) on a random sample of the workload's
+    sequences, scaled to the whole call by its share of the active
+    (token, value head) pairs (padded and empty sequences cost nothing);
+    returns (us per call, description of the sample)."""
+    N = w.spec.N
+    seqs = np.sort(rng.choice(N, size=min(max_seqs, N), replace=False))
+    oracle_subset_seconds(w, seqs[:1])   # untimed: loads the oracle library
+    secs = oracle_subset_seconds(w, seqs)
+    live = w.state_indices >= 0
+    work_all = int(w.seq_lens[live].sum()) + int(live.sum())
+    work_smp = int(w.seq_lens[seqs][live[seqs]].sum()) + int(live[seqs].sum())
+    scale = work_all / max(1, work_smp)
+    return secs * scale * 1e6, (f"{len(seqs)} random sequences ({int(w.seq_lens[seqs].sum())} tokens) timed, "
+                                f"scaled x{scale:.1f} by active tokens + sequences")
+
+
+def per_config_table(torch, binding, device, stream, flags, peak, sms, launches=50):
+    """Every other workload family through the library's default (AUTO) choice:
+    one fresh call checked against the oracle on a sample of sequences, then
+    `launches` isolated launches, each after an L2 flush (a 256 MB memset
+    outside the event pair) and bracketed by CUDA events on the launch stream;
+    the median launch against the measured HBM copy bandwidth, on the
+    algorithmic bytes.  Multi-token calls that run the per-token kernel also
+    report the fraction of the fp32 CUDA-core bound of their algorithmic
+    flops."""
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    rng = np.random.default_rng(0)
+    rows = []
+    for name in PER_CONFIG:
+        w = wl.generate(wl.BY_NAME[name])
+        s = w.spec
+        f = flags | (binding.WRITE_INTERMEDIATE if s.intermediate else 0)
+        c = device_copy(w, torch, device)
+        call = binding.PreparedCall(c["q"], c["k"], c["v"], c["a"], c["b"], c["A_log"], c["dt_bias"],
+                                    c["state_pool"], c["state_indices"], c["cu_seqlens"], c["out"], flags=f,
+                                    intermediate_states=c.get("inter"), stream=stream)
+        par = parity_sample(w, lambda cc: binding.PreparedCall(
+            cc["q"], cc["k"], cc["v"], cc["a"], cc["b"], cc["A_log"], cc["dt_bias"], cc["state_pool"],
+            cc["state_indices"], cc["cu_seqlens"], cc["out"], flags=f, intermediate_states=cc.get("inter"),
+            stream=stream), torch, device)
+        for _ in range(3):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+        with torch.cuda.stream(stream):
+            for a_, b_ in ev:
+                flush.zero_()
+                a_.record(stream)
+                call()
+                b_.record(stream)
+        torch.cuda.synchronize(device)
+        us = float(np.median([a_.elapsed_time(b_) * 1e3 for a_, b_ in ev]))
+        nbytes = wl.algorithmic_bytes(w)
+        one_token = w.T_tot == s.N and not s.intermediate
+        kname = kernel_name(binding.SCHEDULE_AUTO, 0, 0, one_token, s.N * s.HV, w.T_tot / max(1, s.N),
+                            not s.intermediate, sms)
+        o_us, o_how = oracle_sample_us(w, rng)
+        row = {"workload": name, "kernel": kname, "us_per_call": round(us, 3),
+               "gb_s": round(nbytes / (us * 1e-6) / 1e9, 2), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / peak, 4),
+               "algorithmic_bytes": nbytes, "oracle_us_per_call_1core": round(o_us, 1), "oracle_sample": o_how,
+               "parity": par}
+        if not one_token and "gdn_decode_kernel" in kname:
+            row["alu_frac"] = round(wl.algorithmic_flops(w) / (us * 1e-6) / 1e12 / ALU_F32_PEAK_TFLOPS, 4)
+        rows.append(row)
+        del call, c
+    del flush
+    return {"rows": rows, "how": f"AUTO schedule, PDL flag as the headline; median of {launches} isolated "
+                                 "launches, each after a 256 MB L2 flush outside its CUDA-event pair",
+            "peak_gbs": peak}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -365,10 +444,12 @@ def main():
     ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
     ap.add_argument("--tile-v", type=int, default=0)
     ap.add_argument("--tile-rows", type=int, default=0)
-    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split", "local"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-per-config", action="store_true",
+                    help="omit the table of the other workload families (timed after the headline one)")
     ap.add_argument("--unfused", action="store_true",
                     help="time the two-kernel pair (gating, then the recurrence) instead of the fused update")
     ap.add_argument("--no-final-writeback", dest="final_writeback", action="store_false",
@@ -408,7 +489,7 @@ def main():
 
     schedule = {"auto": binding.SCHEDULE_AUTO, "per_tile": binding.SCHEDULE_PER_TILE,
                 "pipelined": binding.SCHEDULE_PIPELINED, "chunked": binding.SCHEDULE_CHUNKED,
-                "split": binding.SCHEDULE_CHUNKED_SPLIT}[args.schedule]
+                "split": binding.SCHEDULE_CHUNKED_SPLIT, "local": binding.SCHEDULE_CHUNKED_LOCAL}[args.schedule]
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)
@@ -567,7 +648,6 @@ def main():
         peak, peak_src = hbm_peak()
         achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
         nflops = wl.algorithmic_flops(w)
-        alu_bound = nflops / (ALU_F32_PEAK_TFLOPS * 1e12) > nbytes / (peak * 1e9)
         traffic = None
         if (NCU_TRAFFIC["kernel_sha256"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.spec.name
                 and not args.unfused and args.schedule in ("auto", "per_tile") and not args.tile_v
@@ -587,16 +667,16 @@ def main():
             "launch_us": launch_us,
             "hbm_frac": {"of_measured": round(achieved / peak, 4), "of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
                          "peak_source": peak_src},
-            "roofline": ({"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                          "frac": round(achieved / peak, 4)} if not alu_bound else
-                         {"bound": "alu", "achieved": round(nflops / (avg_kernel_ms * 1e-3) / 1e12, 3),
-                          "peak": round(ALU_F32_PEAK_TFLOPS, 2), "unit": "TFLOP/s",
-                          "frac": round(nflops / (avg_kernel_ms * 1e-3) / 1e12 / ALU_F32_PEAK_TFLOPS, 4),
-                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-                          "hbm_frac": round(achieved / peak, 4)}) | {
-                         "traffic": traffic, "algorithmic_bytes_per_launch": nbytes,
-                         "algorithmic_flops_per_launch": nflops, "hbm_peak_source": peak_src,
-                         "kernel": kname},
+            # every shape is rated against HBM on its algorithmic bytes; a
+            # multi-token call on the per-token kernel also shows the fraction
+            # of the fp32 CUDA-core bound of its per-token arithmetic
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes_per_launch": nbytes,
+                         "algorithmic_flops_per_launch": nflops, "hbm_peak_source": peak_src, "kernel": kname} | (
+                {"alu_frac": round(nflops / (avg_kernel_ms * 1e-3) / 1e12 / ALU_F32_PEAK_TFLOPS, 4),
+                 "alu_peak_tflops": round(ALU_F32_PEAK_TFLOPS, 2),
+                 "alu_peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"}
+                if w.T_tot != w.spec.N and "gdn_decode_kernel" in kname else {}),
             "e2e": e2e,
             "e2e_serial": e2e_serial,
             "gpu_launches": args.steps * (2 if args.unfused or "+" in kname else 1),
@@ -607,6 +687,10 @@ def main():
             line["cpu_baseline"] = cpu_baseline(w)
             line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w)
             line["parity"] = parity_sample(w, prepare, torch, device, final_writeback=args.final_writeback)
+        if world == 1 and not args.skip_per_config and w.spec.name == wl.DECODE_B512.name:
+            line["per_config"] = per_config_table(torch, binding, device, stream,
+                                                  binding.L2NORM_QK | (binding.LAUNCH_PDL if args.pdl else 0), peak,
+                                                  torch.cuda.get_device_properties(device).multi_processor_count)
         print(json.dumps(line), flush=True)
 
     del calls

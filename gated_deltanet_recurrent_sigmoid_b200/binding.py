@@ -32,6 +32,7 @@ SCHEDULE_PER_TILE = 1
 SCHEDULE_PIPELINED = 2
 SCHEDULE_CHUNKED = 3
 SCHEDULE_CHUNKED_SPLIT = 4
+SCHEDULE_CHUNKED_LOCAL = 5
 
 OK = 0
 ERR_NULL_ARG, ERR_DTYPE, ERR_SHAPE, ERR_ALIGN, ERR_ALIAS = -1, -2, -3, -4, -5

@@ -113,6 +113,156 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
     return static_cast<uint64_t>((T_tot + C - 1) / C) * static_cast<uint64_t>(HV) * REC_BYTES;
 }
 
+// T = (I + A)^-1 for A strictly lower triangular (64 x 64, fp32), by
+// recursive doubling over 16 x 16 blocks:
+//   level 1: the diagonal blocks by substitution, a thread per column;
+//   level 2: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
+//   level 3: T_[23][01] = -T_[23][23] (A_[23][01] T_[01][01]) (32 x 32).
+// A is stored by columns (At[c * 64 + r] = A[r][c]); the intermediate
+// products sit in its upper triangle, whose entries (A[r][c] = 0 for r < c)
+// are never read: level 2's at column block 2p + 1, rows of block 2p; level
+// 3's at columns 32.., rows ..31.  T is written by columns with the row index
+// XOR-swizzled by the column (Tcol[c * 64 + (r ^ (c & 31))]); the diagonal
+// blocks are written in full (their upper triangles zero), the blocks above
+// them never, and every read that can reach one selects zero instead.
+// Threads 0..127 compute; every thread of the CTA must call this (it holds
+// the CTA's barriers), and it ends with one.  When only the first n rows of A
+// can be nonzero (n uniform over the CTA), the blocks of T in rows >= n --
+// rows of the identity -- are skipped: level 1's blocks starting at or past
+// n, level 2's pairs whose lower block does, and level 3 for n <= 32; the
+// caller must then take T's rows >= n as identity rows instead of reading
+// them.  n = 64 computes every block.
+__device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int tid, int n = 64)
+{
+    constexpr int A_LD = 64;
+    const int warp = tid >> 5;
+    auto T_at = [&](int r, int c) -> float & { return Tcol[c * 64 + (r ^ (c & 31))]; };
+    if (tid < 64 && 16 * (tid >> 4) < n) {
+        // level 1: thread (bw, cl) takes column cl of diagonal block bw
+        // (rows b .. b + 15, b = 16 bw), all 16 rows in registers: x = e_cl;
+        // for r = 0 .. 14, x_rho -= A[rho][r] x_r for every rho (A[rho][r] = 0
+        // unless rho > r; x_r is final once the steps before r are done).
+        // Column r of the block is read as the 16-byte groups holding rows
+        // > r; no lane exchanges, so the only dependent chain is the FMAs.
+        const int b = 16 * (tid >> 4), cl = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int rho = 0; rho < 16; ++rho)
+            x[rho] = (rho == cl) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 0; r < 15; ++r) {
+#pragma unroll
+            for (int g = (r + 1) >> 2; g < 4; ++g) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(At + (b + r) * A_LD + b + 4 * g);
+                x[4 * g] = fmaf(-a4.x, x[r], x[4 * g]);
+                x[4 * g + 1] = fmaf(-a4.y, x[r], x[4 * g + 1]);
+                x[4 * g + 2] = fmaf(-a4.z, x[r], x[4 * g + 2]);
+                x[4 * g + 3] = fmaf(-a4.w, x[r], x[4 * g + 3]);
+            }
+        }
+#pragma unroll
+        for (int rho = 0; rho < 16; ++rho)
+            T_at(b + rho, b + cl) = x[rho];
+    }
+    __syncthreads();
+    const int t64 = tid & 63, pr = warp >> 1, C0 = 32 * pr, R1 = C0 + 16;
+    const bool level2 = tid < 128 && R1 < n, level3 = n > 32;
+    if (level2) {
+        // level 2, product 1: M1 = A_[R1][C0] T_[C0][C0] (16 x 16) of pair
+        // pr; thread: column j, rows 4 rg .. 4 rg + 3
+        const int j = t64 & 15, rg = t64 >> 4;
+        float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const float t = T_at(C0 + kk, C0 + j);
+            const float4 a4 = *reinterpret_cast<const float4 *>(At + (C0 + kk) * A_LD + R1 + 4 * rg);
+            m[0] = fmaf(a4.x, t, m[0]);
+            m[1] = fmaf(a4.y, t, m[1]);
+            m[2] = fmaf(a4.z, t, m[2]);
+            m[3] = fmaf(a4.w, t, m[3]);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+            At[(R1 + 4 * rg + ii) * A_LD + C0 + j] = m[ii];      // M1[i][j]
+    }
+    __syncthreads();
+    if (level2) {
+        // level 2, product 2: T_[R1][C0] = -T_[R1][R1] M1; thread: row i,
+        // columns 4 cg .. 4 cg + 3
+        const int i = t64 & 15, cg = t64 >> 4;
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const float t = T_at(R1 + i, R1 + kk);
+            const float4 m4 = *reinterpret_cast<const float4 *>(At + (R1 + kk) * A_LD + C0 + 4 * cg);
+            o[0] = fmaf(-t, m4.x, o[0]);
+            o[1] = fmaf(-t, m4.y, o[1]);
+            o[2] = fmaf(-t, m4.z, o[2]);
+            o[3] = fmaf(-t, m4.w, o[3]);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            T_at(R1 + i, C0 + 4 * cg + jj) = o[jj];
+    }
+    __syncthreads();
+    if (!level3)
+        return;
+    if (tid < 128) {
+        // level 3, product 1: M = A_[23][01] T_[01][01] (32 x 32); thread:
+        // column j = lane, rows 8 w .. 8 w + 7
+        const int j = tid & 31;
+        float m[8];
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii)
+            m[ii] = 0.f;
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            const float t = kk >= j ? T_at(kk, j) : 0.f;
+            const float4 a0 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 32 + 8 * warp);
+            const float4 a1 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 36 + 8 * warp);
+            m[0] = fmaf(a0.x, t, m[0]);
+            m[1] = fmaf(a0.y, t, m[1]);
+            m[2] = fmaf(a0.z, t, m[2]);
+            m[3] = fmaf(a0.w, t, m[3]);
+            m[4] = fmaf(a1.x, t, m[4]);
+            m[5] = fmaf(a1.y, t, m[5]);
+            m[6] = fmaf(a1.z, t, m[6]);
+            m[7] = fmaf(a1.w, t, m[7]);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii)
+            At[(32 + 8 * warp + ii) * A_LD + j] = m[ii];       // M[i][j]
+    }
+    __syncthreads();
+    if (tid < 128) {
+        // level 3, product 2: T_[23][01] = -T_[23][23] M; thread: row
+        // 32 + i (i = lane), columns 8 w .. 8 w + 7
+        const int i = tid & 31;
+        float o[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+            o[jj] = 0.f;
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {
+            const float t = kk <= i ? T_at(32 + i, 32 + kk) : 0.f;
+            const float4 m0 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 8 * warp);
+            const float4 m1 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 4 + 8 * warp);
+            o[0] = fmaf(-t, m0.x, o[0]);
+            o[1] = fmaf(-t, m0.y, o[1]);
+            o[2] = fmaf(-t, m0.z, o[2]);
+            o[3] = fmaf(-t, m0.w, o[3]);
+            o[4] = fmaf(-t, m1.x, o[4]);
+            o[5] = fmaf(-t, m1.y, o[5]);
+            o[6] = fmaf(-t, m1.z, o[6]);
+            o[7] = fmaf(-t, m1.w, o[7]);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+            T_at(32 + i, 8 * warp + jj) = o[jj];
+    }
+    __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 // Kernel 1: the state-independent products of one (block, value head).
 // ---------------------------------------------------------------------------
@@ -456,139 +606,8 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
         }
         __syncthreads();
 
-        // ---- step 4: T = (I + A)^-1, A strictly lower triangular, by
-        // recursive doubling over 16 x 16 blocks:
-        //   level 1: the diagonal blocks by substitution, a thread per column;
-        //   level 2: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
-        //   level 3: T_[23][01] = -T_[23][23] (A_[23][01] T_[01][01]) (32 x 32).
-        // The intermediate products sit in the upper triangle of At, whose
-        // entries (A[r][c] = 0 for r < c) are never read: level 2's at column
-        // block 2p + 1, rows of block 2p; level 3's at columns 32.., rows ..31.
-        // The diagonal blocks are written in full (their upper triangles
-        // zero); the blocks above them are never written, and every read that
-        // can reach one selects zero instead.
-        auto T_at = [&](int r, int c) -> float & { return Tcol[c * 64 + (r ^ (c & 31))]; };
-        if (tid < 64) {
-            // level 1: thread (bw, cl) takes column cl of diagonal block bw
-            // (rows b .. b + 15, b = 16 bw), all 16 rows in registers: x = e_cl;
-            // for r = 0 .. 14, x_rho -= A[rho][r] x_r for every rho (A[rho][r] = 0
-            // unless rho > r; x_r is final once the steps before r are done).
-            // Column r of the block is read as the 16-byte groups holding rows
-            // > r; no lane exchanges, so the only dependent chain is the FMAs.
-            const int b = 16 * (tid >> 4), cl = tid & 15;
-            float x[16];
-#pragma unroll
-            for (int rho = 0; rho < 16; ++rho)
-                x[rho] = (rho == cl) ? 1.f : 0.f;
-#pragma unroll
-            for (int r = 0; r < 15; ++r) {
-#pragma unroll
-                for (int g = (r + 1) >> 2; g < 4; ++g) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(At + (b + r) * A_LD + b + 4 * g);
-                    x[4 * g] = fmaf(-a4.x, x[r], x[4 * g]);
-                    x[4 * g + 1] = fmaf(-a4.y, x[r], x[4 * g + 1]);
-                    x[4 * g + 2] = fmaf(-a4.z, x[r], x[4 * g + 2]);
-                    x[4 * g + 3] = fmaf(-a4.w, x[r], x[4 * g + 3]);
-                }
-            }
-#pragma unroll
-            for (int rho = 0; rho < 16; ++rho)
-                T_at(b + rho, b + cl) = x[rho];
-        }
-        __syncthreads();
-        const int t64 = tid & 63, pr = warp >> 1, C0 = 32 * pr, R1 = C0 + 16;
-        {
-            // level 2, product 1: M1 = A_[R1][C0] T_[C0][C0] (16 x 16) of pair
-            // pr; thread: column j, rows 4 rg .. 4 rg + 3
-            const int j = t64 & 15, rg = t64 >> 4;
-            float m[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                const float t = T_at(C0 + kk, C0 + j);
-                const float4 a4 = *reinterpret_cast<const float4 *>(At + (C0 + kk) * A_LD + R1 + 4 * rg);
-                m[0] = fmaf(a4.x, t, m[0]);
-                m[1] = fmaf(a4.y, t, m[1]);
-                m[2] = fmaf(a4.z, t, m[2]);
-                m[3] = fmaf(a4.w, t, m[3]);
-            }
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
-                At[(R1 + 4 * rg + ii) * A_LD + C0 + j] = m[ii];      // M1[i][j]
-        }
-        __syncthreads();
-        {
-            // level 2, product 2: T_[R1][C0] = -T_[R1][R1] M1; thread: row i,
-            // columns 4 cg .. 4 cg + 3
-            const int i = t64 & 15, cg = t64 >> 4;
-            float o[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                const float t = T_at(R1 + i, R1 + kk);
-                const float4 m4 = *reinterpret_cast<const float4 *>(At + (R1 + kk) * A_LD + C0 + 4 * cg);
-                o[0] = fmaf(-t, m4.x, o[0]);
-                o[1] = fmaf(-t, m4.y, o[1]);
-                o[2] = fmaf(-t, m4.z, o[2]);
-                o[3] = fmaf(-t, m4.w, o[3]);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                T_at(R1 + i, C0 + 4 * cg + jj) = o[jj];
-        }
-        __syncthreads();
-        {
-            // level 3, product 1: M = A_[23][01] T_[01][01] (32 x 32); thread:
-            // column j = lane, rows 8 w .. 8 w + 7
-            const int j = tid & 31;
-            float m[8];
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii)
-                m[ii] = 0.f;
-#pragma unroll 8
-            for (int kk = 0; kk < 32; ++kk) {
-                const float t = kk >= j ? T_at(kk, j) : 0.f;
-                const float4 a0 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 32 + 8 * warp);
-                const float4 a1 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 36 + 8 * warp);
-                m[0] = fmaf(a0.x, t, m[0]);
-                m[1] = fmaf(a0.y, t, m[1]);
-                m[2] = fmaf(a0.z, t, m[2]);
-                m[3] = fmaf(a0.w, t, m[3]);
-                m[4] = fmaf(a1.x, t, m[4]);
-                m[5] = fmaf(a1.y, t, m[5]);
-                m[6] = fmaf(a1.z, t, m[6]);
-                m[7] = fmaf(a1.w, t, m[7]);
-            }
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii)
-                At[(32 + 8 * warp + ii) * A_LD + j] = m[ii];       // M[i][j]
-        }
-        __syncthreads();
-        {
-            // level 3, product 2: T_[23][01] = -T_[23][23] M; thread: row
-            // 32 + i (i = lane), columns 8 w .. 8 w + 7
-            const int i = tid & 31;
-            float o[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                o[jj] = 0.f;
-#pragma unroll 8
-            for (int kk = 0; kk < 32; ++kk) {
-                const float t = kk <= i ? T_at(32 + i, 32 + kk) : 0.f;
-                const float4 m0 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 8 * warp);
-                const float4 m1 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 4 + 8 * warp);
-                o[0] = fmaf(-t, m0.x, o[0]);
-                o[1] = fmaf(-t, m0.y, o[1]);
-                o[2] = fmaf(-t, m0.z, o[2]);
-                o[3] = fmaf(-t, m0.w, o[3]);
-                o[4] = fmaf(-t, m1.x, o[4]);
-                o[5] = fmaf(-t, m1.y, o[5]);
-                o[6] = fmaf(-t, m1.z, o[6]);
-                o[7] = fmaf(-t, m1.w, o[7]);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                T_at(32 + i, 8 * warp + jj) = o[jj];
-        }
-        __syncthreads();
+        // ---- step 4: T = (I + A)^-1 (A strictly lower triangular)
+        solve_unit_lower64(At, Tcol, tid);
 
         // T diag(fw) and T diag(beta) as hi / lo operand tiles, in turn over
         // the q half of kq: each thread keeps four 8-column chunks of rows of

@@ -19,6 +19,7 @@
 #include "gdn_decode_kernel.cuh"
 #include "gdn_chunk_kernel.cuh"
 #include "gdn_chunk_split.cuh"
+#include "gdn_chunk_local.cuh"
 #include "gdn_decode_pipelined.cuh"
 
 namespace {
@@ -354,6 +355,32 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
                      static_cast<const unsigned char *>(ws));
 }
 
+// On-chip chunked schedule: one 256-thread CTA per (sequence, value head),
+// two per SM.
+cudaError_t launch_local(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
+{
+    static PerDevice once;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    const size_t smem = sizeof(gdn::local::Smem);
+    err = once_per_device(once, dev, [&]() {
+        cudaError_t e = cudaSuccess;
+        for (int l2 = 0; l2 < 2 && e == cudaSuccess; ++l2) {
+            auto kern = l2 ? gdn::local::gdn_chunk_local_kernel<true> : gdn::local::gdn_chunk_local_kernel<false>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        }
+        return e;
+    });
+    if (err != cudaSuccess)
+        return err;
+    return launch_ex(l2norm ? gdn::local::gdn_chunk_local_kernel<true> : gdn::local::gdn_chunk_local_kernel<false>,
+                     dim3(static_cast<unsigned>(units)), dim3(gdn::local::THREADS), smem, stream, pdl, p);
+}
+
 // The tile table: (V-tile width, rows per thread) -> (BV, KG = K / rows).
 template <typename TAct, bool GIVEN>
 cudaError_t launch_tile(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, int tile_v,
@@ -424,7 +451,8 @@ int run_update(const UpdateArgs &c)
         return GDN_ERR_ARG;
     int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
     if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED &&
-        schedule != GDN_SCHEDULE_CHUNKED && schedule != GDN_SCHEDULE_CHUNKED_SPLIT)
+        schedule != GDN_SCHEDULE_CHUNKED && schedule != GDN_SCHEDULE_CHUNKED_SPLIT &&
+        schedule != GDN_SCHEDULE_CHUNKED_LOCAL)
         return GDN_ERR_ARG;
     if (extra && extra->reserved != 0)
         return GDN_ERR_ARG;
@@ -657,7 +685,8 @@ int run_update(const UpdateArgs &c)
     if (schedule == GDN_SCHEDULE_PIPELINED &&
         (act != GDN_DTYPE_BF16 || c.given_gates || ga->dtype != GDN_DTYPE_BF16 || gb->dtype != GDN_DTYPE_BF16))
         return GDN_ERR_UNSUPPORTED;
-    const bool chunked = schedule == GDN_SCHEDULE_CHUNKED || schedule == GDN_SCHEDULE_CHUNKED_SPLIT;
+    const bool chunked = schedule == GDN_SCHEDULE_CHUNKED || schedule == GDN_SCHEDULE_CHUNKED_SPLIT ||
+                         schedule == GDN_SCHEDULE_CHUNKED_LOCAL;
     if (chunked && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
         return GDN_ERR_UNSUPPORTED;
     // the chunked kernels read v rows 16 bytes at a time, like q and k
@@ -727,6 +756,8 @@ int run_update(const UpdateArgs &c)
         err = launch_pipelined(p, units, stream, pdl);
     else if (schedule == GDN_SCHEDULE_CHUNKED)
         err = launch_chunked(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
+    else if (schedule == GDN_SCHEDULE_CHUNKED_LOCAL)
+        err = launch_local(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT)
         err = launch_split(p, static_cast<unsigned char *>(ws), units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (act == GDN_DTYPE_BF16)

@@ -164,6 +164,12 @@ extern "C" {
                                     GDN_SCHEDULE_CHUNKED, plus a workspace of
                                     gdn_chunked_workspace_bytes(T_tot, HV) bytes
                                     in gdn_extra */
+#define GDN_SCHEDULE_CHUNKED_LOCAL 5 /* the chunked algorithm in one kernel with
+                                    every product of a chunk kept on chip: one
+                                    CTA per (sequence, value head), 64-token
+                                    chunks aligned to the sequence, two CTAs per
+                                    SM, no workspace.  Same restrictions as
+                                    GDN_SCHEDULE_CHUNKED */
 
 /* bits OR-ed into *device_status by the kernel */
 #define GDN_DEV_BAD_SLOT    1u

@@ -22,10 +22,13 @@ SPLIT = binding.SCHEDULE_CHUNKED_SPLIT
 L2 = binding.L2NORM_QK
 
 
-@pytest.fixture(params=[CHUNKED, SPLIT], ids=["single", "split"])
+LOCAL = binding.SCHEDULE_CHUNKED_LOCAL
+
+
+@pytest.fixture(params=[CHUNKED, SPLIT, LOCAL], ids=["single", "split", "local"])
 def sched(request):
-    """Both chunked schedules: one kernel, or the block kernel + state kernel
-    around a workspace."""
+    """The chunked schedules: one kernel, the block kernel + state kernel
+    around a workspace, or one kernel with every chunk product on chip."""
     return request.param
 
 
