@@ -43,14 +43,19 @@ METRIC = "µs/call and state GB/s (% of B200 HBM peak) at B=512, HV=8, K=V=128"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 ROTATING_COPIES = 4
-# the library's GDN_SCHEDULE_AUTO thresholds (mean tokens per sequence) for
-# the chunked kernel, as documented in include/gdn_decode.h
+# the library's GDN_SCHEDULE_AUTO thresholds (mean tokens per sequence, by the
+# (sequence, value head) pair count), as documented in include/gdn_decode.h
+
+
+def split_min_mean_tokens(pairs):
+    """The split chunked kernels' threshold (the binding passes a workspace)."""
+    return 128 if pairs <= 128 else (448 if pairs <= 512 else 1024)
 
 
 def chunked_min_mean_tokens(pairs):
-    """The split chunked kernels' threshold (the binding always passes a
-    workspace)."""
-    return 40 if pairs < 64 else (30 if pairs < 512 else 18)
+    """The on-chip chunked kernel's threshold."""
+    return 20 if pairs < 64 else (14 if pairs < 512 else 12)
+
 
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
 # ncu capture summarised in profiles/ (dram__bytes_read.sum +
@@ -312,9 +317,11 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     state kernel from 2 (sequence, head) pairs per SM at <= 128 tokens per
     sequence on average)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
-    if (schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok
-            and mean_tokens >= chunked_min_mean_tokens(pairs)):
-        schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
+    if schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok:
+        if mean_tokens >= split_min_mean_tokens(pairs):
+            schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
+        elif mean_tokens >= chunked_min_mean_tokens(pairs):
+            schedule = binding.SCHEDULE_CHUNKED
     if schedule == binding.SCHEDULE_CHUNKED_SPLIT:
         state = ("gdn_chunk_state_compact_kernel" if pairs >= 2 * sms and mean_tokens <= 128
                  else "gdn_chunk_state_kernel")
@@ -322,8 +329,6 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"
     if schedule == binding.SCHEDULE_CHUNKED:
-        return "gdn::chunk::gdn_chunk_kernel<true>"
-    if schedule == binding.SCHEDULE_CHUNKED_LOCAL:
         return "gdn::local::gdn_chunk_local_kernel<true>"
     if tile_v:
         bv, rows = tile_v, tile_rows or 16
@@ -444,7 +449,7 @@ def main():
     ap.add_argument("--copies", type=int, default=ROTATING_COPIES)
     ap.add_argument("--tile-v", type=int, default=0)
     ap.add_argument("--tile-rows", type=int, default=0)
-    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split", "local"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
@@ -489,7 +494,7 @@ def main():
 
     schedule = {"auto": binding.SCHEDULE_AUTO, "per_tile": binding.SCHEDULE_PER_TILE,
                 "pipelined": binding.SCHEDULE_PIPELINED, "chunked": binding.SCHEDULE_CHUNKED,
-                "split": binding.SCHEDULE_CHUNKED_SPLIT, "local": binding.SCHEDULE_CHUNKED_LOCAL}[args.schedule]
+                "split": binding.SCHEDULE_CHUNKED_SPLIT}[args.schedule]
     stream = torch.cuda.Stream(device)
     copies = [device_copy(w, torch, device) for _ in range(max(1, args.copies))]
     flags = binding.L2NORM_QK | (binding.WRITE_INTERMEDIATE if w.spec.intermediate else 0)

@@ -1,12 +1,13 @@
 // gdn_chunk_local.cuh -- the chunked Gated DeltaNet update in ONE sm_100a
-// kernel with every product of a chunk kept on chip: one CTA per (sequence,
-// value head), chunks of 64 tokens aligned to the sequence, no workspace.
+// kernel with every product of a chunk kept on chip (GDN_SCHEDULE_CHUNKED):
+// one CTA per (sequence, value head), chunks of 64 tokens aligned to the
+// sequence, no workspace.
 //
-// Same closed form over a chunk as gdn_chunk_kernel.cuh / gdn_chunk_split.cuh
-// (the pages' chunked GDN prefill, "sglang PR #21411 summary", 实现拆解:
-// chunk_scaled_dot_kkt + solve_tril, CHUNK_SIZE 64), with the state-dependent
-// part arranged so that the state enters one product early instead of
-// through W = T diag(beta e^gamma rk) K.  With S0 the state before the chunk,
+// The closed form of the delta rule over a chunk (the pages' chunked GDN
+// prefill, "sglang PR #21411 summary", 实现拆解: chunk_scaled_dot_kkt +
+// solve_tril, CHUNK_SIZE 64; gdn_chunk_split.cuh holds its WY form), with
+// the state-dependent part arranged so that the state enters one product
+// early instead of through W = T diag(beta e^gamma rk) K.  With S0 the state before the chunk,
 // gamma_t the running sum of g from the chunk start, hats the normalised
 // vectors:
 //     A[t][i] = beta_t e^(gamma_t - gamma_i) k^_t . k^_i   (i < t),  T = (I + A)^-1
@@ -45,7 +46,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "gdn_chunk_kernel.cuh"
+#include "gdn_chunk_common.cuh"
 #include "gdn_chunk_split.cuh"
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"

@@ -1,14 +1,16 @@
 // gdn_chunk_split.cuh -- the chunked Gated DeltaNet update split into two
 // sm_100a kernels around a caller-provided workspace (GDN_SCHEDULE_CHUNKED_SPLIT).
 //
-// The chunk form of gdn_chunk_kernel.cuh has two kinds of work per chunk:
-// products that need only the chunk's own inputs (the decay scan, A, the
-// triangular solve T = (I + A)^-1, W, U and the masked q.k matrix P -- the
-// pages' chunk_scaled_dot_kkt, solve_tril and recompute_w_u steps) and the
+// The chunk form of the update (the WY representation behind the pages'
+// chunked GDN kernels) has two kinds of work per chunk: products that need
+// only the chunk's own inputs (the decay scan, A, the triangular solve
+// T = (I + A)^-1, W, U and the masked q.k matrix P -- the pages'
+// chunk_scaled_dot_kkt, solve_tril and recompute_w_u steps) and the
 // recurrence through the state (Delta = U - W S0, the outputs, the state
 // update -- chunk_gated_delta_rule_fwd_h and chunk_fwd_o).  The single-kernel
-// schedule runs both in one CTA per (sequence, head), chunk after chunk, so
-// the state-independent work sits on the sequential critical path.  Here:
+// schedule (gdn_chunk_local.cuh) runs both in one CTA per (sequence, head),
+// chunk after chunk, so the state-independent work sits on the sequential
+// critical path; with few, long sequences that path is what counts.  Here:
 //
 //   gdn_chunk_wy_kernel     one CTA per (64-token block of the packed token
 //                           range, value head), all in parallel: writes the
@@ -39,15 +41,15 @@
 //              P[j][i] = e^(gamma_j - gamma_i) rqs_j rk_i q_j . k_i  (i <= j, same segment)
 //     S'     = e^gamma_last S0 + sum_i fd_i k_i Delta_i^T,  fd_i = e^(gamma_last - gamma_i) rk_i
 // Operands that are not exact bf16 are split into bf16 hi + lo parts and
-// multiplied as hi*hi + hi*lo + lo*hi (fp32 accumulators in TMEM), as in the
-// single-kernel schedule.
+// multiplied as hi*hi + hi*lo + lo*hi (fp32 accumulators in TMEM; see
+// gdn_chunk_common.cuh).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stddef.h>
 #include <stdint.h>
 
-#include "gdn_chunk_kernel.cuh"
+#include "gdn_chunk_common.cuh"
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
 #include "mbarrier_sm100.cuh"
@@ -58,6 +60,7 @@ namespace split {
 
 using chunk::mma_tiles;
 using chunk::st_row8;
+using chunk::st_row8_hilo;
 
 // D (+)= A B^T with A a K-major [128][a_cols] tile (k-slices of 16 columns)
 // and B stored as the [kdim][b_cols] row tile of B^T, read MN-major: core
@@ -113,12 +116,18 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
     return static_cast<uint64_t>((T_tot + C - 1) / C) * static_cast<uint64_t>(HV) * REC_BYTES;
 }
 
+// Index of A[j][c] in the by-columns fp32 store of A (64 x 64): column c is
+// 64 contiguous floats.  (An XOR swizzle of its 16-byte groups removes the
+// bank conflicts of the column writes but its index arithmetic in the
+// unrolled solve cost more than it saved: 1.3 % on the split schedule.)
+__device__ __forceinline__ int at_idx(int c, int j) { return c * 64 + j; }
+
 // T = (I + A)^-1 for A strictly lower triangular (64 x 64, fp32), by
 // recursive doubling over 16 x 16 blocks:
 //   level 1: the diagonal blocks by substitution, a thread per column;
 //   level 2: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
 //   level 3: T_[23][01] = -T_[23][23] (A_[23][01] T_[01][01]) (32 x 32).
-// A is stored by columns (At[c * 64 + r] = A[r][c]); the intermediate
+// A is stored by columns (At[at_idx(c, r)] = A[r][c]); the intermediate
 // products sit in its upper triangle, whose entries (A[r][c] = 0 for r < c)
 // are never read: level 2's at column block 2p + 1, rows of block 2p; level
 // 3's at columns 32.., rows ..31.  T is written by columns with the row index
@@ -134,7 +143,6 @@ __host__ __device__ constexpr uint64_t workspace_bytes(int64_t T_tot, int64_t HV
 // them.  n = 64 computes every block.
 __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int tid, int n = 64)
 {
-    constexpr int A_LD = 64;
     const int warp = tid >> 5;
     auto T_at = [&](int r, int c) -> float & { return Tcol[c * 64 + (r ^ (c & 31))]; };
     if (tid < 64 && 16 * (tid >> 4) < n) {
@@ -153,7 +161,7 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
         for (int r = 0; r < 15; ++r) {
 #pragma unroll
             for (int g = (r + 1) >> 2; g < 4; ++g) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(At + (b + r) * A_LD + b + 4 * g);
+                const float4 a4 = *reinterpret_cast<const float4 *>(At + at_idx(b + r, b + 4 * g));
                 x[4 * g] = fmaf(-a4.x, x[r], x[4 * g]);
                 x[4 * g + 1] = fmaf(-a4.y, x[r], x[4 * g + 1]);
                 x[4 * g + 2] = fmaf(-a4.z, x[r], x[4 * g + 2]);
@@ -175,7 +183,7 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
             const float t = T_at(C0 + kk, C0 + j);
-            const float4 a4 = *reinterpret_cast<const float4 *>(At + (C0 + kk) * A_LD + R1 + 4 * rg);
+            const float4 a4 = *reinterpret_cast<const float4 *>(At + at_idx(C0 + kk, R1 + 4 * rg));
             m[0] = fmaf(a4.x, t, m[0]);
             m[1] = fmaf(a4.y, t, m[1]);
             m[2] = fmaf(a4.z, t, m[2]);
@@ -183,7 +191,7 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
         }
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii)
-            At[(R1 + 4 * rg + ii) * A_LD + C0 + j] = m[ii];      // M1[i][j]
+            At[at_idx(R1 + 4 * rg + ii, C0 + j)] = m[ii];      // M1[i][j]
     }
     __syncthreads();
     if (level2) {
@@ -194,7 +202,7 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
             const float t = T_at(R1 + i, R1 + kk);
-            const float4 m4 = *reinterpret_cast<const float4 *>(At + (R1 + kk) * A_LD + C0 + 4 * cg);
+            const float4 m4 = *reinterpret_cast<const float4 *>(At + at_idx(R1 + kk, C0 + 4 * cg));
             o[0] = fmaf(-t, m4.x, o[0]);
             o[1] = fmaf(-t, m4.y, o[1]);
             o[2] = fmaf(-t, m4.z, o[2]);
@@ -218,8 +226,8 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
 #pragma unroll 8
         for (int kk = 0; kk < 32; ++kk) {
             const float t = kk >= j ? T_at(kk, j) : 0.f;
-            const float4 a0 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 32 + 8 * warp);
-            const float4 a1 = *reinterpret_cast<const float4 *>(At + kk * A_LD + 36 + 8 * warp);
+            const float4 a0 = *reinterpret_cast<const float4 *>(At + at_idx(kk, 32 + 8 * warp));
+            const float4 a1 = *reinterpret_cast<const float4 *>(At + at_idx(kk, 36 + 8 * warp));
             m[0] = fmaf(a0.x, t, m[0]);
             m[1] = fmaf(a0.y, t, m[1]);
             m[2] = fmaf(a0.z, t, m[2]);
@@ -231,7 +239,7 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
         }
 #pragma unroll
         for (int ii = 0; ii < 8; ++ii)
-            At[(32 + 8 * warp + ii) * A_LD + j] = m[ii];       // M[i][j]
+            At[at_idx(32 + 8 * warp + ii, j)] = m[ii];       // M[i][j]
     }
     __syncthreads();
     if (tid < 128) {
@@ -245,8 +253,8 @@ __device__ __forceinline__ void solve_unit_lower64(float *At, float *Tcol, int t
 #pragma unroll 8
         for (int kk = 0; kk < 32; ++kk) {
             const float t = kk <= i ? T_at(32 + i, 32 + kk) : 0.f;
-            const float4 m0 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 8 * warp);
-            const float4 m1 = *reinterpret_cast<const float4 *>(At + (32 + kk) * A_LD + 4 + 8 * warp);
+            const float4 m0 = *reinterpret_cast<const float4 *>(At + at_idx(32 + kk, 8 * warp));
+            const float4 m1 = *reinterpret_cast<const float4 *>(At + at_idx(32 + kk, 4 + 8 * warp));
             o[0] = fmaf(-t, m0.x, o[0]);
             o[1] = fmaf(-t, m0.y, o[1]);
             o[2] = fmaf(-t, m0.z, o[2]);
@@ -535,10 +543,9 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     }
     wait_mma();
 
-    // A stored by columns, At[c][j] = A[j][c] (fp32 [64][64], over the q half
-    // of kq, consumed by the product above), and T by columns with the row
-    // index XOR-swizzled by the column (fp32 [64][64], in r2)
-    constexpr int A_LD = 64;
+    // A stored by columns, At[at_idx(c, j)] = A[j][c] (fp32 [64][64], over the
+    // q half of kq, consumed by the product above), and T by columns with the
+    // row index XOR-swizzled by the column (fp32 [64][64], in r2)
     float *At = reinterpret_cast<float *>(qhalf);
     float *Tcol = reinterpret_cast<float *>(sm.r2);
     float t8[4][8];     // rows of T, kept for the two T diag() tile pairs
@@ -566,7 +573,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                     a4.y = (j0 + 1 > c && j0 + 1 < ce) ? kk16[4 * e4 + 1] * ex2_approx(u4.y - w) : 0.f;
                     a4.z = (j0 + 2 > c && j0 + 2 < ce) ? kk16[4 * e4 + 2] * ex2_approx(u4.z - w) : 0.f;
                     a4.w = (j0 + 3 > c && j0 + 3 < ce) ? kk16[4 * e4 + 3] * ex2_approx(u4.w - w) : 0.f;
-                    *reinterpret_cast<float4 *>(At + c * A_LD + j0) = a4;
+                    *reinterpret_cast<float4 *>(At + at_idx(c, j0)) = a4;
                 }
             }
 #pragma unroll 1
@@ -584,10 +591,8 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
                         pt[4 * e4 + e] = (j >= c && j < ce) ? pt[4 * e4 + e] * ex2_approx(uv[e] - w) : 0.f;
                     }
                 }
-                st_row8(rec + REC_KP_HI, c, K + jb, KP_COLS, pt, false);
-                st_row8(rec + REC_KP_HI, c, K + jb + 8, KP_COLS, pt + 8, false);
-                st_row8(rec + REC_KP_LO, c, K + jb, KP_COLS, pt, true);
-                st_row8(rec + REC_KP_LO, c, K + jb + 8, KP_COLS, pt + 8, true);
+                st_row8_hilo(rec + REC_KP_HI, rec + REC_KP_LO, c, K + jb, KP_COLS, pt);
+                st_row8_hilo(rec + REC_KP_HI, rec + REC_KP_LO, c, K + jb + 8, KP_COLS, pt + 8);
             }
         } else {
             // K' = diag(fd) K: row j of the raw k rows, scaled, hi / lo
@@ -600,8 +605,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     x[e] *= f;
-                st_row8(rec + REC_KP_HI, j, col, KP_COLS, x, false);
-                st_row8(rec + REC_KP_LO, j, col, KP_COLS, x, true);
+                st_row8_hilo(rec + REC_KP_HI, rec + REC_KP_LO, j, col, KP_COLS, x);
             }
         }
         __syncthreads();
@@ -637,8 +641,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 x8[e] = t8[ch][e] * sm.fw[c0 + e];
-            st_row8(tw_hi, r, c0, C, x8, false);
-            st_row8(tw_lo, r, c0, C, x8, true);
+            st_row8_hilo(tw_hi, tw_lo, r, c0, C, x8);
         }
         publish_smem();
 
@@ -661,8 +664,7 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 x8[e] = t8[ch][e] * sm.beta[c0 + e];
-            st_row8(tu_hi, r, c0, C, x8, false);
-            st_row8(tu_lo, r, c0, C, x8, true);
+            st_row8_hilo(tu_hi, tu_lo, r, c0, C, x8);
         }
         sync::cp_async_wait_all();
         publish_smem();
@@ -903,10 +905,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
 #pragma unroll
             for (int c = 0; c < KP; c += 16) {
                 tc::tmem_st16(my_lane + ST_COL_S + kh + c, x + c);
-                st_row8(sm.st[0], v, kh + c, K, x + c, false);
-                st_row8(sm.st[0], v, kh + c + 8, K, x + c + 8, false);
-                st_row8(sm.st[1], v, kh + c, K, x + c, true);
-                st_row8(sm.st[1], v, kh + c + 8, K, x + c + 8, true);
+                st_row8_hilo(sm.st[0], sm.st[1], v, kh + c, K, x + c);
+                st_row8_hilo(sm.st[0], sm.st[1], v, kh + c + 8, K, x + c + 8);
             }
             tc::tmem_wait_st();
         }
@@ -1020,10 +1020,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
                 const int ii = cb + e;
                 d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[cl + e]) * dscale : 0.f;
             }
-            st_row8(sm.dt[0], v, cb, C, d, false);
-            st_row8(sm.dt[0], v, cb + 8, C, d + 8, false);
-            st_row8(sm.dt[1], v, cb, C, d, true);
-            st_row8(sm.dt[1], v, cb + 8, C, d + 8, true);
+            st_row8_hilo(sm.dt[0], sm.dt[1], v, cb, C, d);
+            st_row8_hilo(sm.dt[0], sm.dt[1], v, cb + 8, C, d + 8);
         }
         {                            // O2 accumulates from zero in product 2
             float z[16];
@@ -1087,10 +1085,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
             tc::tmem_ld16(my_lane + ST_COL_S + k0, x);
             tc::tmem_wait_ld();
             if (more) {
-                st_row8(sm.st[0], v, k0, K, x, false);
-                st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
-                st_row8(sm.st[1], v, k0, K, x, true);
-                st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
+                st_row8_hilo(sm.st[0], sm.st[1], v, k0, K, x);
+                st_row8_hilo(sm.st[0], sm.st[1], v, k0 + 8, K, x + 8);
             } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -1266,10 +1262,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
 #pragma unroll
         for (int c = 0; c < KP; c += 16) {
             tc::tmem_st16(my_lane + SC_COL_S + kh + c, x + c);
-            st_row8(sm.st[0], v, kh + c, K, x + c, false);
-            st_row8(sm.st[0], v, kh + c + 8, K, x + c + 8, false);
-            st_row8(sm.st[1], v, kh + c, K, x + c, true);
-            st_row8(sm.st[1], v, kh + c + 8, K, x + c + 8, true);
+            st_row8_hilo(sm.st[0], sm.st[1], v, kh + c, K, x + c);
+            st_row8_hilo(sm.st[0], sm.st[1], v, kh + c + 8, K, x + c + 8);
         }
         tc::tmem_wait_st();
     }
@@ -1347,10 +1341,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
                 const int ii = cb + e;
                 d[e] = (ii >= r0 && ii < r1) ? fmaf(cs, d[e], u[cl + e]) * dscale : 0.f;
             }
-            st_row8(dt_hi, v, cb, C, d, false);
-            st_row8(dt_hi, v, cb + 8, C, d + 8, false);
-            st_row8(dt_lo, v, cb, C, d, true);
-            st_row8(dt_lo, v, cb + 8, C, d + 8, true);
+            st_row8_hilo(dt_hi, dt_lo, v, cb, C, d);
+            st_row8_hilo(dt_hi, dt_lo, v, cb + 8, C, d + 8);
 #pragma unroll
             for (int e = 0; e < 16; ++e)
                 d[e] = 0.f;
@@ -1420,10 +1412,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
             tc::tmem_ld16(my_lane + SC_COL_S + k0, x);
             tc::tmem_wait_ld();
             if (more) {
-                st_row8(sm.st[0], v, k0, K, x, false);
-                st_row8(sm.st[0], v, k0 + 8, K, x + 8, false);
-                st_row8(sm.st[1], v, k0, K, x, true);
-                st_row8(sm.st[1], v, k0 + 8, K, x + 8, true);
+                st_row8_hilo(sm.st[0], sm.st[1], v, k0, K, x);
+                st_row8_hilo(sm.st[0], sm.st[1], v, k0 + 8, K, x + 8);
             } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e)

@@ -17,7 +17,6 @@
 
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
-#include "gdn_chunk_kernel.cuh"
 #include "gdn_chunk_split.cuh"
 #include "gdn_chunk_local.cuh"
 #include "gdn_decode_pipelined.cuh"
@@ -26,21 +25,24 @@ namespace {
 
 constexpr int kHeadK = 128;
 constexpr int kHeadV = 128;
-// GDN_SCHEDULE_AUTO takes the chunked kernel when the batch holds at least
-// this many tokens per sequence on average: 128 while there are at most 1024
-// (sequence, value head) pairs, 256 beyond (the measured B200 crossovers:
-// with 64-1024 pairs the chunked kernel is 0.82-0.97 of the per-tile time at
-// ~128 tokens; with 4096 pairs it needs ~250).
-constexpr int64_t kChunkedMinMeanTokensFew = 128;
-constexpr int64_t kChunkedMinMeanTokensMany = 256;
-constexpr int64_t kChunkedFewPairs = 1024;
-// With a workspace, AUTO takes the split chunked kernels from a lower mean
-// length (measured B200 crossovers against the per-tile kernel, lengths
-// spread over [L/2, 3L/2]): 40 tokens below 64 (sequence, value head)
-// pairs, 30 below 512, 18 from 512 on (split / per-tile time: 1 sequence
-// 1.04 at 36 tokens, 0.81 at 48; 8 sequences 1.23 at 23, 0.90 at 33; 64-1024
-// sequences 0.98-1.06 at 16, 0.88-0.92 at 20).
-int64_t split_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 40 : (pairs < 512 ? 30 : 18); }
+// GDN_SCHEDULE_AUTO, for calls the chunked kernels are built for, by the
+// mean sequence length L = T_tot / N and the (sequence, value head) pair
+// count P = N * HV (measured B200 crossovers, lengths spread over
+// [L/2, 3L/2], isolated launches):
+//   - the split kernels (with a large enough caller workspace) from L >= 128
+//     when P <= 128, L >= 448 when P <= 512, L >= 1024 beyond: only few,
+//     long sequences gain from computing every block's products in parallel
+//     first (4 sequences: 50 vs 53 us at L = 132; 16: 77 vs 84 us at 193;
+//     64: 459 vs 511 us at 481, but 372 vs 335 us at 365; 256: the on-chip
+//     kernel is faster at every measured length up to 392);
+//   - the on-chip chunked kernel from L >= 20 when P < 64, L >= 14 when
+//     P < 512, L >= 12 beyond (its one-CTA chain costs ~20 us, so with few
+//     pairs the per-token kernel wins longer: 1 sequence 28.7 vs 22.5 us at
+//     L = 32, 8: 26.6 vs 21.4 at 19, 64 - 1024: within 4 % at 12, the
+//     chunked kernel ahead from 16);
+//   - the per-token kernel otherwise.
+int64_t split_min_mean_tokens(int64_t pairs) { return pairs <= 128 ? 128 : (pairs <= 512 ? 448 : 1024); }
+int64_t chunked_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 20 : (pairs < 512 ? 14 : 12); }
 // The split schedule's state kernel in its compact form (two CTAs per SM)
 // from this many (sequence, value head) pairs per SM, for sequences of at
 // most this many tokens on average (measured on B200: 0.89-0.92x the time of
@@ -273,30 +275,6 @@ cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t strea
                      stream, pdl, p);
 }
 
-// Chunked schedule: one CTA per (sequence, value head), dynamic shared
-// memory opted in once per device.
-cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
-{
-    static PerDevice once;
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess)
-        return err;
-    const size_t smem = sizeof(gdn::chunk::Smem);
-    err = once_per_device(once, dev, [&]() {
-        cudaError_t e = cudaFuncSetAttribute(gdn::chunk::gdn_chunk_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn::chunk::gdn_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem));
-        return e;
-    });
-    if (err != cudaSuccess)
-        return err;
-    return launch_ex(l2norm ? gdn::chunk::gdn_chunk_kernel<true> : gdn::chunk::gdn_chunk_kernel<false>,
-                     dim3(static_cast<unsigned>(units)), dim3(gdn::chunk::THREADS), smem, stream, pdl, p);
-}
-
 // Split chunked schedule: the block kernel over ceil(T_tot / 64) x HV CTAs,
 // then the state kernel over the (sequence, value head) pairs.  The state
 // kernel always uses programmatic dependent launch behind the block kernel
@@ -355,9 +333,9 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
                      static_cast<const unsigned char *>(ws));
 }
 
-// On-chip chunked schedule: one 256-thread CTA per (sequence, value head),
-// two per SM.
-cudaError_t launch_local(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
+// Chunked schedule: one 256-thread CTA per (sequence, value head), two per
+// SM, every chunk product on chip (gdn_chunk_local.cuh).
+cudaError_t launch_chunked(const gdn::DecodeParams &p, int64_t units, cudaStream_t stream, bool pdl, bool l2norm)
 {
     static PerDevice once;
     int dev = 0;
@@ -370,6 +348,7 @@ cudaError_t launch_local(const gdn::DecodeParams &p, int64_t units, cudaStream_t
         for (int l2 = 0; l2 < 2 && e == cudaSuccess; ++l2) {
             auto kern = l2 ? gdn::local::gdn_chunk_local_kernel<true> : gdn::local::gdn_chunk_local_kernel<false>;
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            // the largest shared-memory carveout, so that two CTAs fit on an SM
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         }
@@ -451,8 +430,7 @@ int run_update(const UpdateArgs &c)
         return GDN_ERR_ARG;
     int schedule = extra ? extra->schedule : GDN_SCHEDULE_AUTO;
     if (schedule != GDN_SCHEDULE_AUTO && schedule != GDN_SCHEDULE_PER_TILE && schedule != GDN_SCHEDULE_PIPELINED &&
-        schedule != GDN_SCHEDULE_CHUNKED && schedule != GDN_SCHEDULE_CHUNKED_SPLIT &&
-        schedule != GDN_SCHEDULE_CHUNKED_LOCAL)
+        schedule != GDN_SCHEDULE_CHUNKED && schedule != GDN_SCHEDULE_CHUNKED_SPLIT)
         return GDN_ERR_ARG;
     if (extra && extra->reserved != 0)
         return GDN_ERR_ARG;
@@ -667,16 +645,16 @@ int run_update(const UpdateArgs &c)
                          (tile_v == 64 && (tile_rows == 16 || tile_rows == 32));
     if (!tile_ok)
         return GDN_ERR_UNSUPPORTED;
-    // The library's schedule: the chunked tensor-core kernel when the
-    // sequences are long on average (and it is built for the call), else the
-    // per-tile kernel.
+    // The library's schedule (thresholds above): the split kernels for few,
+    // long sequences, the on-chip chunked kernel from a dozen or so tokens per
+    // sequence on average, else the per-tile kernel.
     const bool v_rows_16b =
         aligned(v->data, 16) && stride_ok(T_tot, Lv.tok, 8) && stride_ok(HV, v->stride[v->ndim - 2], 8);
     if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
         act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0) {
         if (ws_fits && T_tot >= split_min_mean_tokens(N * HV) * N)
             schedule = GDN_SCHEDULE_CHUNKED_SPLIT;
-        else if (T_tot >= (N * HV <= kChunkedFewPairs ? kChunkedMinMeanTokensFew : kChunkedMinMeanTokensMany) * N)
+        else if (T_tot >= chunked_min_mean_tokens(N * HV) * N)
             schedule = GDN_SCHEDULE_CHUNKED;
     }
     // The pipelined schedule is built for bf16 activations and fused bf16
@@ -685,8 +663,7 @@ int run_update(const UpdateArgs &c)
     if (schedule == GDN_SCHEDULE_PIPELINED &&
         (act != GDN_DTYPE_BF16 || c.given_gates || ga->dtype != GDN_DTYPE_BF16 || gb->dtype != GDN_DTYPE_BF16))
         return GDN_ERR_UNSUPPORTED;
-    const bool chunked = schedule == GDN_SCHEDULE_CHUNKED || schedule == GDN_SCHEDULE_CHUNKED_SPLIT ||
-                         schedule == GDN_SCHEDULE_CHUNKED_LOCAL;
+    const bool chunked = schedule == GDN_SCHEDULE_CHUNKED || schedule == GDN_SCHEDULE_CHUNKED_SPLIT;
     if (chunked && (act != GDN_DTYPE_BF16 || c.given_gates || want_inter))
         return GDN_ERR_UNSUPPORTED;
     // the chunked kernels read v rows 16 bytes at a time, like q and k
@@ -756,8 +733,6 @@ int run_update(const UpdateArgs &c)
         err = launch_pipelined(p, units, stream, pdl);
     else if (schedule == GDN_SCHEDULE_CHUNKED)
         err = launch_chunked(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
-    else if (schedule == GDN_SCHEDULE_CHUNKED_LOCAL)
-        err = launch_local(p, units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (schedule == GDN_SCHEDULE_CHUNKED_SPLIT)
         err = launch_split(p, static_cast<unsigned char *>(ws), units, stream, pdl, (flags & GDN_L2NORM_QK) != 0);
     else if (act == GDN_DTYPE_BF16)

@@ -124,16 +124,16 @@ extern "C" {
                                      more scratch than GDN_STATIC_SCRATCH_BYTES */
 
 /* work schedules (gdn_extra.schedule); all compute the same update */
-#define GDN_SCHEDULE_AUTO      0 /* library choice.  When the call qualifies for
-                                    the chunked kernels (bf16 activations, fused
-                                    gates, no per-token states, v rows 16-byte
-                                    aligned): GDN_SCHEDULE_CHUNKED_SPLIT if the
-                                    caller gives a large enough workspace and
-                                    the sequences hold, on average, >= 40 tokens
-                                    (N * HV < 64), >= 30 (N * HV < 512) or >= 18
-                                    (otherwise); without a workspace
-                                    GDN_SCHEDULE_CHUNKED from >= 128 tokens
-                                    (N * HV <= 1024) or >= 256.  Otherwise
+#define GDN_SCHEDULE_AUTO      0 /* library choice, by the mean tokens per sequence
+                                    L = T_tot / N and the pair count P = N * HV.
+                                    When the call qualifies for the chunked
+                                    kernels (bf16 activations, fused gates, no
+                                    per-token states, v rows 16-byte aligned):
+                                    GDN_SCHEDULE_CHUNKED_SPLIT if the caller gives
+                                    a large enough workspace and L >= 128
+                                    (P <= 128), >= 448 (P <= 512) or >= 1024;
+                                    else GDN_SCHEDULE_CHUNKED if L >= 20 (P < 64),
+                                    >= 14 (P < 512) or >= 12.  Otherwise
                                     GDN_SCHEDULE_PER_TILE */
 #define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
                                     state tile moves through registers.  Tiles
@@ -147,10 +147,11 @@ extern "C" {
 #define GDN_SCHEDULE_PIPELINED 2 /* one persistent CTA per SM; whole-head state
                                     tiles stream through a shared-memory ring of
                                     bulk async copies (cp.async.bulk) */
-#define GDN_SCHEDULE_CHUNKED   3 /* one CTA per (sequence, value head); tokens in
-                                    chunks of 64 through the closed form of the
-                                    delta rule over a chunk, every matrix product
-                                    on the tcgen05 tensor cores (prefill-style);
+#define GDN_SCHEDULE_CHUNKED   3 /* one CTA per (sequence, value head), two per SM;
+                                    tokens in chunks of 64 through the closed
+                                    form of the delta rule over a chunk, every
+                                    matrix product on the tcgen05 tensor cores and
+                                    every intermediate on chip (no workspace);
                                     bf16 activations, gates from A_log/a/b/dt_bias,
                                     no GDN_WRITE_INTERMEDIATE; v aligned like q */
 #define GDN_SCHEDULE_CHUNKED_SPLIT 4 /* the same chunked algorithm as two kernels:
@@ -164,12 +165,6 @@ extern "C" {
                                     GDN_SCHEDULE_CHUNKED, plus a workspace of
                                     gdn_chunked_workspace_bytes(T_tot, HV) bytes
                                     in gdn_extra */
-#define GDN_SCHEDULE_CHUNKED_LOCAL 5 /* the chunked algorithm in one kernel with
-                                    every product of a chunk kept on chip: one
-                                    CTA per (sequence, value head), 64-token
-                                    chunks aligned to the sequence, two CTAs per
-                                    SM, no workspace.  Same restrictions as
-                                    GDN_SCHEDULE_CHUNKED */
 
 /* bits OR-ed into *device_status by the kernel */
 #define GDN_DEV_BAD_SLOT    1u

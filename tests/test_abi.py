@@ -62,7 +62,7 @@ def test_header_constants_match_binding():
     assert define("GDN_NO_FINAL_WRITEBACK") == binding.NO_FINAL_WRITEBACK
     assert define("GDN_CHECK_INDICES") == binding.CHECK_INDICES
     assert define("GDN_LAUNCH_PDL") == binding.LAUNCH_PDL
-    for name in ("AUTO", "PER_TILE", "PIPELINED", "CHUNKED", "CHUNKED_SPLIT", "CHUNKED_LOCAL"):
+    for name in ("AUTO", "PER_TILE", "PIPELINED", "CHUNKED", "CHUNKED_SPLIT"):
         assert define(f"GDN_SCHEDULE_{name}") == getattr(binding, f"SCHEDULE_{name}")
     for name, val in [("GDN_ERR_NULL_ARG", -1), ("GDN_ERR_DTYPE", -2), ("GDN_ERR_SHAPE", -3),
                       ("GDN_ERR_ALIGN", -4), ("GDN_ERR_ALIAS", -5), ("GDN_ERR_UNSUPPORTED", -6),

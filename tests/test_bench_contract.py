@@ -40,18 +40,27 @@ def test_reference_arm_prints_the_contract_line():
     (True, 4096, 1.0, "gdn::gdn_decode_kernel<128,128,64,4>"),                  # decode: 64x32
     (False, 4096, 4.0, "gdn::gdn_decode_kernel<128,128,32,4>"),                 # many short chains: 32x32
     (False, 1024, 4.0, "gdn::gdn_decode_kernel<128,128,16,8>"),                 # spec decode: 16x16
-    (False, 8, 29.0, "gdn::gdn_decode_kernel<128,128,8,16>"),                   # few chains: 8x8
-    (False, 8, 48.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
-    (False, 8192, 32.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_compact_kernel"),
+    (False, 8, 12.0, "gdn::gdn_decode_kernel<128,128,8,16>"),                   # few short chains: 8x8
+    (False, 8, 29.0, "gdn::local::gdn_chunk_local_kernel<true>"),               # sweep_b1
+    (False, 8192, 31.8, "gdn::local::gdn_chunk_local_kernel<true>"),            # sweep_b1024
+    (False, 64, 1686.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
     (False, 512, 480.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
+    (False, 512, 365.0, "gdn::local::gdn_chunk_local_kernel<true>"),
 ])
 def test_kernel_name_mirrors_the_documented_choice(one_token, pairs, mean, expected):
     assert bench.kernel_name(binding.SCHEDULE_AUTO, 0, 0, one_token, pairs, mean, chunk_ok=not one_token,
                              sms=148) == expected
 
 
-def test_split_thresholds_match_the_header():
+def test_split_schedule_names_its_compact_state_kernel():
+    assert bench.kernel_name(binding.SCHEDULE_CHUNKED_SPLIT, 0, 0, False, 8192, 32.0, sms=148) == \
+        "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_compact_kernel"
+
+
+def test_auto_thresholds_match_the_header():
     """The thresholds the bench mirrors are the ones the header documents."""
-    header = open(os.path.join(ROOT, "include", "gdn_decode.h")).read()
-    assert ">= 40 tokens" in header and ">= 30 (N * HV < 512) or >= 18" in header
-    assert [bench.chunked_min_mean_tokens(p) for p in (8, 63, 64, 511, 512, 8192)] == [40, 40, 30, 30, 18, 18]
+    header = " ".join(open(os.path.join(ROOT, "include", "gdn_decode.h")).read().split())
+    assert "L >= 128 (P <= 128), >= 448 (P <= 512) or >= 1024" in header
+    assert "L >= 20 (P < 64), >= 14 (P < 512) or >= 12" in header
+    assert [bench.split_min_mean_tokens(p) for p in (8, 128, 129, 512, 513)] == [128, 128, 448, 448, 1024]
+    assert [bench.chunked_min_mean_tokens(p) for p in (8, 63, 64, 511, 512, 8192)] == [20, 20, 14, 14, 12, 12]

@@ -22,13 +22,10 @@ SPLIT = binding.SCHEDULE_CHUNKED_SPLIT
 L2 = binding.L2NORM_QK
 
 
-LOCAL = binding.SCHEDULE_CHUNKED_LOCAL
-
-
-@pytest.fixture(params=[CHUNKED, SPLIT, LOCAL], ids=["single", "split", "local"])
+@pytest.fixture(params=[CHUNKED, SPLIT], ids=["single", "split"])
 def sched(request):
-    """The chunked schedules: one kernel, the block kernel + state kernel
-    around a workspace, or one kernel with every chunk product on chip."""
+    """Both chunked schedules: one kernel with every chunk product on chip, or
+    the block kernel + state kernel around a workspace."""
     return request.param
 
 
@@ -158,13 +155,13 @@ def _bits_equal(a, b):
     return torch.equal(a["state_pool"], b["state_pool"]) and torch.equal(a["out"], b["out"])
 
 
-def test_auto_schedule_picks_chunked_for_long_sequences():
-    """GDN_SCHEDULE_AUTO: mean length >= 128 with few (sequence, head) pairs
-    runs the split chunked kernels when a workspace is given (the binding
-    allocates one) and the single chunked kernel without one (bit-identical
-    to asking for them); short sequences, or a call with per-token states,
-    run the per-tile kernel."""
-    long_w = problem([200, 150, 300], seed=21)
+def test_auto_schedule_picks_by_length_and_pairs():
+    """GDN_SCHEDULE_AUTO (bit-identical to asking for the schedule it picks):
+    few long sequences run the split kernels when a workspace is given (the
+    binding allocates one) and the on-chip chunked kernel without one;
+    sequences of a few dozen tokens run the on-chip chunked kernel either
+    way; short ones, or a call with per-token states, the per-tile kernel."""
+    long_w = problem([200, 150, 300], seed=21)                 # 24 pairs, mean 217
     auto, _, _ = run_gpu(long_w)
     split, _, _ = run_gpu(long_w, schedule=SPLIT)
     assert _bits_equal(auto, split)
@@ -174,7 +171,12 @@ def test_auto_schedule_picks_chunked_for_long_sequences():
     per_tile, _, _ = run_gpu(long_w, schedule=binding.SCHEDULE_PER_TILE)
     assert not _bits_equal(auto, per_tile) and not _bits_equal(auto, chunked)
 
-    short_w = problem([3, 60, 10], seed=22)
+    mid_w = problem([30, 60, 10, 45], seed=23)                # 32 pairs, mean 36
+    auto, _, _ = run_gpu(mid_w)
+    chunked, _, _ = run_gpu(mid_w, schedule=CHUNKED)
+    assert _bits_equal(auto, chunked)
+
+    short_w = problem([3, 20, 10], seed=22)                   # 24 pairs, mean 11
     auto, _, _ = run_gpu(short_w)
     per_tile, _, _ = run_gpu(short_w, schedule=binding.SCHEDULE_PER_TILE)
     assert _bits_equal(auto, per_tile)

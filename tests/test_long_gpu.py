@@ -85,16 +85,16 @@ def test_auto_without_workspace_short_mean_long_sequence():
     check_whole(w, "auto_no_workspace_per_tile", workspace=None)
 
 
-@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT,
-                                   binding.SCHEDULE_CHUNKED_LOCAL], ids=["single", "split", "local"])
+@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT],
+                         ids=["single", "split"])
 def test_chunked_long_weak_decay(sched):
     """The chunked schedules at 2,048 tokens with weak and strong heads, whole."""
     w = random_workload([2048, 1500, 64, 65], H=2, HV=4, seed=104, weak_heads=(0, 3))
     check_whole(w, f"chunked_{sched}", schedule=sched)
 
 
-@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT,
-                                   binding.SCHEDULE_CHUNKED_LOCAL], ids=["single", "split", "local"])
+@pytest.mark.parametrize("sched", [binding.SCHEDULE_CHUNKED, binding.SCHEDULE_CHUNKED_SPLIT],
+                         ids=["single", "split"])
 def test_prefill_b8_t2k_sampled(sched):
     """The full prefill workload (8 sequences of 1-2K tokens) in the
     benchmark's configuration; the oracle recomputes three sequences, the
