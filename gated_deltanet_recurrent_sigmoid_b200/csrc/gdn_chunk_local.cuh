@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_chunk_local_kernel(const __gri
         sm.failed = 0;
         sync::fence_barrier_init();
         // the state S [k][v] (64 KB, contiguous) in one bulk copy
-        sync::mbar_arrive_expect_tx(&sm.bar_x, K * V * 4);
+        sync::mbar_arrive_expect_state_tx(&sm.bar_x, K * V * 4);
         sync::bulk_load(sm.s, s_gmem, K * V * 4, &sm.bar_x);
     }
     if (warp == 0) {

@@ -849,7 +849,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1) gdn_chunk_state_kernel(const __
         sync::fence_barrier_init();
         // the state S [k][v] (64 KB, contiguous) into the state-tile region in
         // one bulk copy, beside the first piece's records
-        sync::mbar_arrive_expect_tx(&sm.bar_x, K * V * 4);
+        sync::mbar_arrive_expect_state_tx(&sm.bar_x, K * V * 4);
         sync::bulk_load(sm.st, s_gmem, K * V * 4, &sm.bar_x);
         const unsigned char *r = rec_of(blk);
         sync::mbar_arrive_expect_tx(&sm.bar_a, REC_A_BYTES);
@@ -1211,7 +1211,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) gdn_chunk_state_compact_kernel(
         sync::fence_barrier_init();
         // the state S [k][v] (64 KB, contiguous) into the state-tile region in
         // one bulk copy, beside the first piece's W / Q and fo / gamma
-        sync::mbar_arrive_expect_tx(&sm.bar_x, K * V * 4);
+        sync::mbar_arrive_expect_state_tx(&sm.bar_x, K * V * 4);
         sync::bulk_load(sm.st, s_gmem, K * V * 4, &sm.bar_x);
         const unsigned char *r = rec_of(blk);
         sync::prefetch_l2(r + REC_UT, REC_FO - REC_UT);     // U^T of the first piece (read per thread)

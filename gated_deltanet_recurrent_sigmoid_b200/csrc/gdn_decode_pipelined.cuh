@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(THREADS, 1) gdn_decode_pipelined_kernel(const 
             const int s = j % STAGES;
             const Unit u = classify(p, blockIdx.x + j * gridDim.x);
             if (u.kind == 0 && !*failed) {
-                mbar_arrive_expect_tx(&sm.full[s], TILE_BYTES);
+                sync::mbar_arrive_expect_state_tx(&sm.full[s], TILE_BYTES);
                 const float *src = state_ptr(u);
 #pragma unroll
                 for (int c = 0; c < CHUNKS; ++c)

@@ -8,7 +8,12 @@
 namespace gdn {
 namespace sync {
 
-constexpr uint64_t WAIT_LIMIT_NS = 500ull * 1000ull * 1000ull;   // 0.5 s
+// Time limit of every bounded wait: 0.5 s.  The timeout tests build a copy
+// of the library (tests/timeout_probe/) with a limit of a few milliseconds.
+#ifndef GDN_WAIT_LIMIT_NS
+#define GDN_WAIT_LIMIT_NS (500ull * 1000ull * 1000ull)
+#endif
+constexpr uint64_t WAIT_LIMIT_NS = GDN_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -36,6 +41,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, u
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                  : "memory");
+}
+
+// The expect-tx arrival paired with the bulk copy of a sequence's state (the
+// barrier phase completes when this arrival and the copy's bytes are both
+// in).  The test copy of the library (tests/timeout_probe/) is compiled with
+// GDN_TEST_WITHHOLD_STATE_ARRIVAL, which drops the arrival: the copy still
+// lands, its phase never completes, and the kernel's bounded wait for it runs
+// out -- how the timeout paths are made to fire on a GPU without a fault.
+// Product builds never define it.
+__device__ __forceinline__ void mbar_arrive_expect_state_tx(unsigned long long *bar, uint32_t bytes)
+{
+#ifdef GDN_TEST_WITHHOLD_STATE_ARRIVAL
+    (void)bar;
+    (void)bytes;
+#else
+    mbar_arrive_expect_tx(bar, bytes);
+#endif
 }
 
 __device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t parity)

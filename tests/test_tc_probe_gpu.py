@@ -2,19 +2,28 @@
 checked through a test-only one-tile probe against a plain matrix product."""
 import ctypes
 import os
-import sys
 
 import pytest
 import torch
 
 pytestmark = pytest.mark.gpu
 
-sys.path.insert(0, os.path.join(os.path.dirname(os.path.abspath(__file__)), "tc_probe"))
+
+def _load_builder():
+    """The probe's build module, loaded by path under its own name (both
+    probe directories have a build.py)."""
+    import importlib.util
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tc_probe", "build.py")
+    spec = importlib.util.spec_from_file_location("tc_probe_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
 
 
 @pytest.fixture(scope="module")
 def probe():
-    import build as probe_build
+    probe_build = _load_builder()
     lib = ctypes.CDLL(probe_build.build())
     lib.tc_gemm_probe.restype = ctypes.c_int
     lib.tc_gemm_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [ctypes.c_void_p] * 2
