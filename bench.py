@@ -47,14 +47,20 @@ ROTATING_COPIES = 4
 # (sequence, value head) pair count), as documented in include/gdn_decode.h
 
 
-def split_min_mean_tokens(pairs):
-    """The split chunked kernels' threshold (the binding passes a workspace)."""
-    return 128 if pairs <= 128 else (448 if pairs <= 512 else 1024)
+def split_pays(pairs, mean_tokens):
+    """Whether AUTO runs the split chunked kernels (the binding passes a workspace)."""
+    if pairs < 128:
+        return mean_tokens >= 128
+    if pairs < 256:
+        return mean_tokens >= 192
+    if pairs < 512:
+        return mean_tokens >= 512
+    return False
 
 
 def chunked_min_mean_tokens(pairs):
     """The on-chip chunked kernel's threshold."""
-    return 20 if pairs < 64 else (14 if pairs < 512 else 12)
+    return 20 if pairs < 64 else (14 if pairs < 512 else 13)
 
 
 # DRAM traffic of one launch of the fused kernel on decode_b512_hv8, from the
@@ -318,7 +324,7 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     sequence on average)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok:
-        if mean_tokens >= split_min_mean_tokens(pairs):
+        if split_pays(pairs, mean_tokens):
             schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
         elif mean_tokens >= chunked_min_mean_tokens(pairs):
             schedule = binding.SCHEDULE_CHUNKED

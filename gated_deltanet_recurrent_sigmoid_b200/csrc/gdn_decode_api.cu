@@ -28,21 +28,31 @@ constexpr int kHeadV = 128;
 // GDN_SCHEDULE_AUTO, for calls the chunked kernels are built for, by the
 // mean sequence length L = T_tot / N and the (sequence, value head) pair
 // count P = N * HV (measured B200 crossovers, lengths spread over
-// [L/2, 3L/2], isolated launches):
+// [L/2, 3L/2]):
 //   - the split kernels (with a large enough caller workspace) from L >= 128
-//     when P <= 128, L >= 448 when P <= 512, L >= 1024 beyond: only few,
-//     long sequences gain from computing every block's products in parallel
-//     first (4 sequences: 50 vs 53 us at L = 132; 16: 77 vs 84 us at 193;
-//     64: 459 vs 511 us at 481, but 372 vs 335 us at 365; 256: the on-chip
-//     kernel is faster at every measured length up to 392);
+//     when P < 128, L >= 192 when P < 256, L >= 512 when P < 512, never
+//     beyond: only few, long sequences gain from computing every block's
+//     products in parallel first (back-to-back calls: 8 sequences at
+//     L = 470, 116 vs 183 us; 16 at 130, 54 vs 51, at 283, 85 vs 98; 32 at
+//     506, 255 vs 261; 64 sequences: the on-chip kernel is 4-10 % faster at
+//     every length up to 2,085, 128 sequences 16-20 %);
 //   - the on-chip chunked kernel from L >= 20 when P < 64, L >= 14 when
-//     P < 512, L >= 12 beyond (its one-CTA chain costs ~20 us, so with few
+//     P < 512, L >= 13 beyond (its one-CTA chain costs ~20 us, so with few
 //     pairs the per-token kernel wins longer: 1 sequence 28.7 vs 22.5 us at
-//     L = 32, 8: 26.6 vs 21.4 at 19, 64 - 1024: within 4 % at 12, the
-//     chunked kernel ahead from 16);
+//     L = 32, 8: 26.6 vs 21.4 at 19; 1024 sequences 513 vs 539 us at 11.9,
+//     663 vs 550 at 16);
 //   - the per-token kernel otherwise.
-int64_t split_min_mean_tokens(int64_t pairs) { return pairs <= 128 ? 128 : (pairs <= 512 ? 448 : 1024); }
-int64_t chunked_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 20 : (pairs < 512 ? 14 : 12); }
+bool split_pays(int64_t pairs, int64_t T_tot, int64_t N)
+{
+    if (pairs < 128)
+        return T_tot >= 128 * N;
+    if (pairs < 256)
+        return T_tot >= 192 * N;
+    if (pairs < 512)
+        return T_tot >= 512 * N;
+    return false;
+}
+int64_t chunked_min_mean_tokens(int64_t pairs) { return pairs < 64 ? 20 : (pairs < 512 ? 14 : 13); }
 // The split schedule's state kernel in its compact form (two CTAs per SM)
 // from this many (sequence, value head) pairs per SM, for sequences of at
 // most this many tokens on average (measured on B200: 0.89-0.92x the time of
@@ -652,7 +662,7 @@ int run_update(const UpdateArgs &c)
         aligned(v->data, 16) && stride_ok(T_tot, Lv.tok, 8) && stride_ok(HV, v->stride[v->ndim - 2], 8);
     if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
         act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0) {
-        if (ws_fits && T_tot >= split_min_mean_tokens(N * HV) * N)
+        if (ws_fits && split_pays(N * HV, T_tot, N))
             schedule = GDN_SCHEDULE_CHUNKED_SPLIT;
         else if (T_tot >= chunked_min_mean_tokens(N * HV) * N)
             schedule = GDN_SCHEDULE_CHUNKED;

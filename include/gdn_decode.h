@@ -131,10 +131,10 @@ extern "C" {
                                     per-token states, v rows 16-byte aligned):
                                     GDN_SCHEDULE_CHUNKED_SPLIT if the caller gives
                                     a large enough workspace and L >= 128
-                                    (P <= 128), >= 448 (P <= 512) or >= 1024;
-                                    else GDN_SCHEDULE_CHUNKED if L >= 20 (P < 64),
-                                    >= 14 (P < 512) or >= 12.  Otherwise
-                                    GDN_SCHEDULE_PER_TILE */
+                                    (P < 128), >= 192 (P < 256) or >= 512
+                                    (P < 512); else GDN_SCHEDULE_CHUNKED if
+                                    L >= 20 (P < 64), >= 14 (P < 512) or >= 13.
+                                    Otherwise GDN_SCHEDULE_PER_TILE */
 #define GDN_SCHEDULE_PER_TILE  1 /* one CTA per (sequence, value head, V-tile); the
                                     state tile moves through registers.  Tiles
                                     (tile_v x tile_rows): 8x8, 16x16, 32x16,
