@@ -250,22 +250,22 @@ def _args(d):
             d["cu_seqlens"], d["out"])
 
 
-def test_split_graph_capture_and_pdl_chain():
-    """The split schedule (two kernels) captures in a CUDA graph and chains
-    with programmatic dependent launch: two chained calls replayed from a
-    graph, and two chained PDL calls, match two chained oracle calls and give
-    the bits of two eager calls."""
+def test_graph_capture_and_pdl_chain(sched):
+    """Both chunked schedules capture in a CUDA graph and chain with
+    programmatic dependent launch (the split one as two kernels): two chained
+    calls replayed from a graph, and two chained PDL calls, match two chained
+    oracle calls and give the bits of two eager calls."""
     w = problem([150, 40, 90], seed=51)
     eager = to_device(w)
     for _ in range(2):
-        binding.decode_update(*_args(eager), schedule=SPLIT)
+        binding.decode_update(*_args(eager), schedule=sched)
     torch.cuda.synchronize()
 
     d = to_device(w)
     pool0 = d["state_pool"].clone()
     ws = torch.empty(binding.chunked_workspace_bytes(w.T_tot, w.spec.HV), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
-    call = binding.PreparedCall(*_args(d), stream=stream, schedule=SPLIT, workspace=ws)
+    call = binding.PreparedCall(*_args(d), stream=stream, schedule=sched, workspace=ws)
     call()                                   # one-time per-device set-up outside the capture
     torch.cuda.synchronize()
     d["state_pool"].copy_(pool0)
@@ -282,8 +282,8 @@ def test_split_graph_capture_and_pdl_chain():
 
     p = to_device(w)
     first = torch.empty_like(p["out"])
-    binding.decode_update(*_args(p)[:-1], first, schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
-    binding.decode_update(*_args(p), schedule=SPLIT, flags=L2 | binding.LAUNCH_PDL)
+    binding.decode_update(*_args(p)[:-1], first, schedule=sched, flags=L2 | binding.LAUNCH_PDL)
+    binding.decode_update(*_args(p), schedule=sched, flags=L2 | binding.LAUNCH_PDL)
     torch.cuda.synchronize()
     o_refs, s_ref = oracle_chain([workload_arrays(w)] * 2, w.state_pool)
     live = w.state_indices[w.state_indices >= 0]
