@@ -26,6 +26,18 @@ __device__ __forceinline__ void split2(float x, __nv_bfloat16 &hi, __nv_bfloat16
     lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
+// The hi and lo parts of two values at once, packed as bf16 pairs (x0 in the
+// low half): the paired conversion rounds each value to nearest even, exactly
+// as split2 does one at a time, in half the instructions.
+__device__ __forceinline__ void split2x2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // Eight consecutive columns c0..c0+7 (c0 % 8 == 0) of row r: one 16-byte store
 // of their hi or lo parts into a K-major tile whose rows have `cols` columns.
 __device__ __forceinline__ void st_row8(unsigned char *tile, uint32_t r, uint32_t c0, uint32_t cols, const float *x,
@@ -34,29 +46,22 @@ __device__ __forceinline__ void st_row8(unsigned char *tile, uint32_t r, uint32_
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split2(x[2 * e], h0, l0);
-        split2(x[2 * e + 1], h1, l1);
-        const __nv_bfloat16 a = lo_part ? l0 : h0, b = lo_part ? l1 : h1;
-        w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
+        uint32_t hi, lo;
+        split2x2(x[2 * e], x[2 * e + 1], hi, lo);
+        w[e] = lo_part ? lo : hi;
     }
     *reinterpret_cast<uint4 *>(tile + tc::kmajor_offset(r, c0, cols)) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // The same eight columns of row r into a hi tile and a lo tile of the same
-// layout at once (one split per element, two 16-byte stores).
+// layout at once (one split per pair of elements, two 16-byte stores).
 __device__ __forceinline__ void st_row8_hilo(unsigned char *hi_tile, unsigned char *lo_tile, uint32_t r, uint32_t c0,
                                              uint32_t cols, const float *x)
 {
     uint32_t wh[4], wl[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        split2(x[2 * e], h0, l0);
-        split2(x[2 * e + 1], h1, l1);
-        wh[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-        wl[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-    }
+    for (int e = 0; e < 4; ++e)
+        split2x2(x[2 * e], x[2 * e + 1], wh[e], wl[e]);
     const uint32_t off = tc::kmajor_offset(r, c0, cols);
     *reinterpret_cast<uint4 *>(hi_tile + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
     *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
@@ -67,6 +72,7 @@ __device__ __forceinline__ void st_row8_hilo(unsigned char *hi_tile, unsigned ch
 __device__ __forceinline__ void mma_tiles(uint32_t d, const unsigned char *a, uint32_t a_cols, const unsigned char *b,
                                           uint32_t b_cols, uint32_t slices, uint32_t idesc, bool accumulate)
 {
+#pragma unroll 1
     for (uint32_t s = 0; s < slices; ++s)
         tc::mma_bf16(d, tc::kslice_desc(a, a_cols, s), tc::kslice_desc(b, b_cols, s), idesc,
                      (accumulate || s > 0) ? 1u : 0u);

@@ -71,6 +71,7 @@ __device__ __forceinline__ void mma_tiles_bmn(uint32_t d, const unsigned char *a
                                               uint32_t idesc, bool accumulate)
 {
     const uint32_t kstride = (b_cols >> 3) * 128u;
+#pragma unroll 1
     for (uint32_t s = 0; s < slices; ++s)
         tc::mma_bf16(d, tc::kslice_desc(a, a_cols, s), tc::mn_desc(tc::smem_u32(b) + s * 2u * kstride, kstride, 128u),
                      idesc, (accumulate || s > 0) ? 1u : 0u);
