@@ -319,9 +319,10 @@ def run_reference(args, w):
 
 def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, chunk_ok=False, sms=148):
     """Name of the kernel the library launches for these settings (mirrors
-    the library's documented choice, including the split schedule's compact
-    state kernel from 2 (sequence, head) pairs per SM at <= 128 tokens per
-    sequence on average)."""
+    the library's documented choice, including the split schedule's state
+    kernel: two CTAs per (sequence, head) pair while they fit one wave, the
+    compact form from 2 pairs per SM at <= 128 tokens per sequence on
+    average, else the full-width form)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok:
         if split_pays(pairs, mean_tokens):
@@ -329,8 +330,12 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
         elif mean_tokens >= chunked_min_mean_tokens(pairs):
             schedule = binding.SCHEDULE_CHUNKED
     if schedule == binding.SCHEDULE_CHUNKED_SPLIT:
-        state = ("gdn_chunk_state_compact_kernel" if pairs >= 2 * sms and mean_tokens <= 128
-                 else "gdn_chunk_state_kernel")
+        if 2 * pairs <= sms:
+            state = "gdn_chunk_state_half_kernel"
+        elif pairs >= 2 * sms and mean_tokens <= 128:
+            state = "gdn_chunk_state_compact_kernel"
+        else:
+            state = "gdn_chunk_state_kernel"
         return f"gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::{state}"
     if schedule == binding.SCHEDULE_PIPELINED:
         return "gdn::pipe::gdn_decode_pipelined_kernel<3>"

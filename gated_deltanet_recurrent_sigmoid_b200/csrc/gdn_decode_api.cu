@@ -18,6 +18,7 @@
 #include "gdn_decode.h"
 #include "gdn_decode_kernel.cuh"
 #include "gdn_chunk_split.cuh"
+#include "gdn_chunk_state_half.cuh"
 #include "gdn_chunk_local.cuh"
 #include "gdn_decode_pipelined.cuh"
 
@@ -312,6 +313,10 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
             e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(sizeof(gdn::split::StSmemCompact)));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_half_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(sizeof(gdn::split::ShSmem)));
         // the largest shared-memory carveout, so that four block-kernel CTAs
         // (two compact state-kernel CTAs) fit on an SM
         for (int l2 = 0; l2 < 2 && e == cudaSuccess; ++l2)
@@ -331,8 +336,13 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
                     dim3(static_cast<unsigned>(blocks)), dim3(gdn::split::THREADS), smem_wy, stream, pdl, p, ws);
     if (err != cudaSuccess)
         return err;
-    // Many (sequence, head) pairs: the compact state kernel (two CTAs per SM);
-    // otherwise the one with more threads and deeper prefetching.
+    // Few (sequence, head) pairs: two CTAs per pair, each on half the state
+    // columns, as long as they fit one wave; many pairs: the compact state
+    // kernel (two CTAs per SM); otherwise the full-width kernel.
+    if (2 * units <= sm_count[dev])
+        return launch_ex(gdn::split::gdn_chunk_state_half_kernel, dim3(static_cast<unsigned>(2 * units)),
+                         dim3(gdn::split::SH_THREADS), sizeof(gdn::split::ShSmem), stream, true, p,
+                         static_cast<const unsigned char *>(ws));
     if (units >= kSplitCompactMinUnitsPerSm * sm_count[dev] &&
         static_cast<int64_t>(p.T_tot) <= kSplitCompactMaxMeanTokens * p.N)
         return launch_ex(gdn::split::gdn_chunk_state_compact_kernel, dim3(static_cast<unsigned>(units)),

@@ -43,9 +43,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, u
                  : "memory");
 }
 
-// The expect-tx arrival paired with the bulk copy of a sequence's state (the
-// barrier phase completes when this arrival and the copy's bytes are both
-// in).  The test copy of the library (tests/timeout_probe/) is compiled with
+// The expect-tx arrival paired with a kernel's first bulk copy of a
+// sequence's data -- its state, or the first piece's record for a kernel that
+// loads the state with plain loads (the barrier phase completes when this
+// arrival and the copy's bytes are both in).  The test copy of the library (tests/timeout_probe/) is compiled with
 // GDN_TEST_WITHHOLD_STATE_ARRIVAL, which drops the arrival: the copy still
 // lands, its phase never completes, and the kernel's bounded wait for it runs
 // out -- how the timeout paths are made to fire on a GPU without a fault.

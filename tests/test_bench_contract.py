@@ -43,7 +43,7 @@ def test_reference_arm_prints_the_contract_line():
     (False, 8, 12.0, "gdn::gdn_decode_kernel<128,128,8,16>"),                   # few short chains: 8x8
     (False, 8, 29.0, "gdn::local::gdn_chunk_local_kernel<true>"),               # sweep_b1
     (False, 8192, 31.8, "gdn::local::gdn_chunk_local_kernel<true>"),            # sweep_b1024
-    (False, 64, 1686.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
+    (False, 64, 1686.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_half_kernel"),
     (False, 512, 480.0, "gdn::local::gdn_chunk_local_kernel<true>"),           # prefill_b64_t512
     (False, 256, 600.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
     (False, 128, 150.0, "gdn::local::gdn_chunk_local_kernel<true>"),
@@ -54,9 +54,13 @@ def test_kernel_name_mirrors_the_documented_choice(one_token, pairs, mean, expec
                              sms=148) == expected
 
 
-def test_split_schedule_names_its_compact_state_kernel():
-    assert bench.kernel_name(binding.SCHEDULE_CHUNKED_SPLIT, 0, 0, False, 8192, 32.0, sms=148) == \
-        "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_compact_kernel"
+def test_split_schedule_names_its_state_kernel():
+    def name(pairs, mean):
+        return bench.kernel_name(binding.SCHEDULE_CHUNKED_SPLIT, 0, 0, False, pairs, mean, sms=148).split("::")[-1]
+    assert name(8192, 32.0) == "gdn_chunk_state_compact_kernel"     # many short sequences
+    assert name(74, 32.0) == "gdn_chunk_state_half_kernel"          # two CTAs per pair fit one wave
+    assert name(75, 2000.0) == "gdn_chunk_state_kernel"
+    assert name(296, 129.0) == "gdn_chunk_state_kernel"
 
 
 def test_auto_thresholds_match_the_header():

@@ -216,8 +216,9 @@ def test_chunked_strided_views_of_packed_projections(sched):
     assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
 
 
-@pytest.mark.parametrize("lens", [[200, 37, 130, 64, 5] * 3, [int(x) for x in np.random.default_rng(71).integers(1, 65, 320)]],
-                         ids=["full_form", "compact_form"])
+@pytest.mark.parametrize("lens", [[200, 37, 130, 64, 5], [200, 37, 130, 64, 5] * 3,
+                                  [int(x) for x in np.random.default_rng(71).integers(1, 65, 320)]],
+                         ids=["two_cta_form", "full_form", "compact_form"])
 def test_split_is_deterministic(lens):
     """Five runs of the split schedule on the same inputs give the same bits
     (no atomics or order-dependent sums in either kernel: a race between the
@@ -228,6 +229,18 @@ def test_split_is_deterministic(lens):
         d, status, _ = run_gpu(w, schedule=SPLIT)
         assert status == 0
         assert torch.equal(d["out"], ref["out"]) and torch.equal(d["state_pool"], ref["state_pool"])
+
+
+def test_split_full_width_state_kernel_mid_batch():
+    """96 (sequence, head) pairs -- more than one wave of two-CTA pairs on 148
+    SMs, fewer than the compact form's 296 -- run the full-width state kernel:
+    ragged lengths, an empty and a padded sequence, weak and strong decays,
+    compared whole with the oracle."""
+    lens = [200, 37, 130, 64, 5, 1, 300, 65, 128, 0, 90, 150]
+    w = problem(lens, pad=(4,), seed=73)
+    w.A_log = w.A_log.copy()
+    w.A_log[::2] = -9.0
+    check(w, SPLIT)
 
 
 def test_split_compact_many_short_sequences():

@@ -1,10 +1,13 @@
 """The kernels' bounded waits, made to run out on purpose.
 
 A test-only copy of the library (tests/timeout_probe/) withholds the arrival
-that pairs with each bulk copy of a sequence's state and limits every wait
-to 2 ms, so each kernel that waits for a state copy gives up.  For the
-on-chip chunked kernel, both split state kernels (full and compact) and the
-pipelined kernel, one call through that copy must
+that pairs with each kernel's first bulk copy of a sequence's data (its
+state, or for the two-CTA split state kernel, which loads the state with
+plain loads, the first piece's U / fo / gamma) and limits every wait to
+2 ms, so each kernel gives up at its first wait.  For the on-chip chunked
+kernel, the three split state kernels (two CTAs per pair -- 12 pairs --,
+full-width -- 84 pairs, more than fit one wave of two-CTA pairs on 148 SMs --
+and compact) and the pipelined kernel, one call through that copy must
 
   - return GDN_OK and report GDN_DEV_TIMEOUT in the status word,
   - leave every byte outside its buffers alone (guard bands around the pool,
@@ -60,7 +63,8 @@ def timeout_lib(gdn_lib):
 CASES = {
     # schedule, lengths, heads: each reaches the named kernel's state wait
     "chunked": (binding.SCHEDULE_CHUNKED, [70, 3, 130, 64], 2, 4),
-    "split_full": (binding.SCHEDULE_CHUNKED_SPLIT, [150, 40, 90], 2, 4),
+    "split_half": (binding.SCHEDULE_CHUNKED_SPLIT, [150, 40, 90], 2, 4),
+    "split_full": (binding.SCHEDULE_CHUNKED_SPLIT, [150, 40, 90] * 7, 2, 4),
     "split_compact": (binding.SCHEDULE_CHUNKED_SPLIT, [int(x) for x in np.random.default_rng(5).integers(1, 65, 40)],
                       4, 8),
     "pipelined": (binding.SCHEDULE_PIPELINED, [1] * 24, 2, 4),

@@ -3,11 +3,11 @@
 
 The library's own sources, compiled with two switches that product builds
 never set: GDN_TEST_WITHHOLD_STATE_ARRIVAL drops the expect-tx arrival that
-pairs with each bulk copy of a sequence's state (the copy still lands, but
-the barrier phase it belongs to never completes), and GDN_WAIT_LIMIT_NS
-shortens every bounded wait to 2 ms.  Every kernel that waits for a state
-copy (the on-chip chunked kernel, both split state kernels, the pipelined
-kernel) then takes its timeout path: GDN_DEV_TIMEOUT in the status word, no
+pairs with each kernel's first bulk copy of a sequence's data (the copy
+still lands, but the barrier phase it belongs to never completes), and
+GDN_WAIT_LIMIT_NS shortens every bounded wait to 2 ms.  Every kernel that
+waits for such a copy (the on-chip chunked kernel, the three split state
+kernels, the pipelined kernel) then takes its timeout path: GDN_DEV_TIMEOUT in the status word, no
 further work, its copies allowed to land (bounded), TMEM freed."""
 import os
 import subprocess
