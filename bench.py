@@ -47,10 +47,12 @@ ROTATING_COPIES = 4
 # (sequence, value head) pair count), as documented in include/gdn_decode.h
 
 
-def split_pays(pairs, mean_tokens):
+def split_pays(pairs, mean_tokens, sms=148):
     """Whether AUTO runs the split chunked kernels (the binding passes a workspace)."""
+    if 2 * pairs <= sms:
+        return mean_tokens >= 80
     if pairs < 128:
-        return mean_tokens >= 128
+        return mean_tokens >= 144
     if pairs < 256:
         return mean_tokens >= 192
     if pairs < 512:
@@ -325,7 +327,7 @@ def kernel_name(schedule, tile_v, tile_rows, one_token, pairs, mean_tokens=1.0, 
     average, else the full-width form)."""
     from gated_deltanet_recurrent_sigmoid_b200 import binding
     if schedule == binding.SCHEDULE_AUTO and not tile_v and not tile_rows and chunk_ok:
-        if split_pays(pairs, mean_tokens):
+        if split_pays(pairs, mean_tokens, sms):
             schedule = binding.SCHEDULE_CHUNKED_SPLIT      # the binding passes a workspace
         elif mean_tokens >= chunked_min_mean_tokens(pairs):
             schedule = binding.SCHEDULE_CHUNKED

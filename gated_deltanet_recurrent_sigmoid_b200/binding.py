@@ -147,7 +147,7 @@ def _workspace_for(workspace, schedule: int, q: torch.Tensor, v: torch.Tensor, N
     """The workspace to pass: the caller's tensor, or (workspace="auto") one
     allocated here when the split chunked schedule is asked for, or when the
     library may choose it (AUTO with fewer than 512 (sequence, value head)
-    pairs and at least 128 tokens per sequence on average -- the library's
+    pairs and at least 80 tokens per sequence on average -- the library's
     widest range for the split kernels)."""
     if workspace is None or isinstance(workspace, torch.Tensor):
         return workspace
@@ -155,7 +155,7 @@ def _workspace_for(workspace, schedule: int, q: torch.Tensor, v: torch.Tensor, N
         raise ValueError("workspace must be a tensor, None or 'auto'")
     T_tot = v.numel() // (v.shape[-1] * v.shape[-2]) if v.dim() >= 2 else 0
     HV = v.shape[-2] if v.dim() >= 2 else 0
-    if not (schedule == SCHEDULE_CHUNKED_SPLIT or (schedule == SCHEDULE_AUTO and N > 0 and N * HV < 512 and T_tot >= 128 * N)):
+    if not (schedule == SCHEDULE_CHUNKED_SPLIT or (schedule == SCHEDULE_AUTO and N > 0 and N * HV < 512 and T_tot >= 80 * N)):
         return None
     nbytes = chunked_workspace_bytes(T_tot, HV)
     return torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None

@@ -47,7 +47,7 @@ constexpr uint32_t SH_COL_DL = 64;             // -W lo S~hi     lanes i        
 constexpr uint32_t SH_COL_O2 = 128;            // P Delta~       lanes 64 + j   64
 constexpr uint32_t SH_COL_DQ = 256;            // [D | O1], hi and lo halves: 128 per piece parity (2 x 128)
 
-enum { SH_BAR_A, SH_BAR_B, SH_BAR_R, SH_BAR_D, SH_BAR_S, SH_BAR_O };
+enum { SH_BAR_A, SH_BAR_B, SH_BAR_R, SH_BAR_D, SH_BAR_S, SH_BAR_O, SH_BAR_DR, SH_BAR_TR, SH_NBAR };
 
 struct ShSmem {
     // [S~hi | S~lo] [k][v' | v'], the MN-major B operand of product 1 (64 KB
@@ -58,10 +58,10 @@ struct ShSmem {
     alignas(1024) unsigned char dt[2][C * SH_COLS * 2]; // Delta~ hi / lo [i][v'], MN-major B of product 2
     alignas(16) float ut[SH_COLS * C];                  // this CTA's rows of U^T [v'][i]
     alignas(16) float rec_s[REC_S_BYTES / 4];           // fo, gamma of the piece
-    float fo[2][C];                                     // fo of the last two pieces (by piece parity)
     // mbarriers, by SH_BAR_*: the bulk copies of W / Q, K' / P and U / fo /
-    // gamma; product 1, product 2a and product 2b done
-    unsigned long long bar[6];
+    // gamma; product 1, product 2a and product 2b done; every worker warp's
+    // Delta~ tiles (and rescale), and its next state tiles, written
+    unsigned long long bar[SH_NBAR];
     uint32_t tmem_base;
     int failed;
 };
@@ -103,7 +103,6 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
     const bool worker = tid < SH_WORKERS;
     const int row = (warp & 3) * 32 + (tid & 31);       // TMEM lane
     const int cb = SH_CP * (warp >> 2);                   // first of this thread's columns
-    const bool delta_warp = worker && (warp & 3) < 2;
     const bool out_warp = worker && (warp & 3) >= 2;
     const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;
     const int i = pair / p.HV;
@@ -159,12 +158,8 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
     // thread's state row part into registers -----------------------------
     int64_t blk = bos / C;
     if (tid == SH_ISSUER) {
-        sync::mbar_init(&sm.bar[SH_BAR_D], 1);
-        sync::mbar_init(&sm.bar[SH_BAR_S], 1);
-        sync::mbar_init(&sm.bar[SH_BAR_O], 1);
-        sync::mbar_init(&sm.bar[SH_BAR_A], 1);
-        sync::mbar_init(&sm.bar[SH_BAR_B], 1);
-        sync::mbar_init(&sm.bar[SH_BAR_R], 1);
+        for (int m = 0; m < SH_NBAR; ++m)
+            sync::mbar_init(&sm.bar[m], m == SH_BAR_DR || m == SH_BAR_TR ? SH_WORKERS / 32 : 1);
         sm.failed = 0;
         sync::fence_barrier_init();
         const unsigned char *r = rec_of(blk);
@@ -201,26 +196,12 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t my_lane = tc::tmem_addr(tmem, (warp & 3) * 32, 0);
-    if (worker) {          // S~ = S (cs = 1) into TMEM and the hi / lo tiles
-        tc::tmem_st16(my_lane + SH_COL_S + cb, x);
-        st_row8_hilo(sm.st, sm.st + 1024, row, cb, 2 * SH_COLS, x);
-        st_row8_hilo(sm.st, sm.st + 1024, row, cb + 8, 2 * SH_COLS, x + 8);
-        tc::tmem_wait_st();
-    }
-    auto publish = [&](bool mine) {      // smem tiles -> tensor cores; uniform verdict
-        tc::fence_proxy_async_smem();
-        tc::fence_before_sync();
-        const bool all = __syncthreads_and(mine) != 0;
-        tc::fence_after_sync();
-        return all;
-    };
-    bool ok = publish(true);
-
-    // Barrier m (B_*) below: bit m of `phase` is the parity this thread waits
-    // for next.  The issuer also records, per barrier, whether it has issued
-    // a copy or committed a product to it (bit m of `used`) and the parity of
-    // the last such phase (bit m of `last`).
-    enum { B_A = SH_BAR_A, B_B = SH_BAR_B, B_R = SH_BAR_R, B_D = SH_BAR_D, B_S = SH_BAR_S, B_O = SH_BAR_O };
+    // Barrier m (B_*): bit m of `phase` is the parity this thread waits for
+    // next.  The issuer also records, per copy / product barrier, whether it
+    // has used it (bit m of `used`) and the parity of its last phase (bit m
+    // of `last`), for the drain after a failure.
+    enum { B_A = SH_BAR_A, B_B = SH_BAR_B, B_R = SH_BAR_R, B_D = SH_BAR_D, B_S = SH_BAR_S, B_O = SH_BAR_O,
+           B_DR = SH_BAR_DR, B_TR = SH_BAR_TR };
     uint32_t phase = 0, used = (1u << B_A) | (1u << B_B) | (1u << B_R), last = 0;
     auto wait_one = [&](int m) {          // bounded, this thread only
         const bool w = sync::mbar_wait(&sm.bar[m], (phase >> m) & 1u, &sm.failed);
@@ -229,18 +210,35 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
             sm.failed = 1;
             report(p.status, GDN_DEV_TIMEOUT);
         }
+        tc::fence_after_sync();
         return w;
     };
     auto note = [&](int m) {              // issuer: one more phase of barrier m used
         last ^= (used >> m) & 1u ? 1u << m : 0u;
         used |= 1u << m;
     };
+    // a worker warp's shared-memory tiles and TMEM stores, handed to the issuer
+    auto arrive = [&](int m) {
+        tc::fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if ((tid & 31) == 0)
+            sync::mbar_arrive(&sm.bar[m]);
+    };
+    bool mine = true;
+    if (worker) {          // S~ = S (cs = 1) into TMEM and the hi / lo tiles
+        tc::tmem_st16(my_lane + SH_COL_S + cb, x);
+        st_row8_hilo(sm.st, sm.st + 1024, row, cb, 2 * SH_COLS, x);
+        st_row8_hilo(sm.st, sm.st + 1024, row, cb + 8, 2 * SH_COLS, x + 8);
+        tc::tmem_wait_st();
+        arrive(B_TR);
+    }
 
     // A piece's outputs (rows j, lanes 64..127) are written while the next
-    // piece's product 1 runs, or after the last piece: rows [ob, oe) of block
-    // ob_blk, from [D | O1] buffer obuf, with the scales before (ocs) and
+    // piece's product 1 runs, or after the last piece: rows of block o_blk,
+    // from [D | O1] buffer obuf, with fo_j, and the scales before (ocs) and
     // after (ocs_new) the piece.
-    auto write_outputs = [&](int64_t o_blk, int obuf, float ocs, float ocs_new) {
+    auto write_outputs = [&](int64_t o_blk, int obuf, float fo_j, float ocs, float ocs_new) {
         const bool w = wait_one(B_O);         // product 2b of that piece
         if (w) {
             const int64_t obase = o_blk * C;
@@ -254,7 +252,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
             tc::tmem_wait_ld();
             const int j = row - C;
             if (j >= out_r0 && j < out_r1) {
-                const float f1 = -sm.fo[obuf][j] * ocs;
+                const float f1 = -fo_j * ocs;
                 uint32_t pk[SH_CP / 2];
 #pragma unroll
                 for (int e = 0; e < SH_CP; e += 2) {
@@ -271,98 +269,44 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
         return w;
     };
 
+    // The loop runs without CTA-wide barriers: workers hand their tiles to
+    // the issuer through bar_dr / bar_tr, the issuer hands products back
+    // through bar_d / bar_s / bar_o; a thread whose wait fails (or that sees
+    // another one's failure) leaves the loop.
     float cs = 1.f, prev_cs = 1.f;       // the scale before this piece and before the last one
+    float fo_j = 0.f;                    // output rows: fo of the piece whose outputs are pending
     int buf = 0;
-    for (int64_t t = bos; t < eos && ok; ++blk, buf ^= 1) {
+    for (int64_t t = bos; t < eos; ++blk, buf ^= 1) {
         const int64_t base = blk * C;
         const int r0 = static_cast<int>(t - base);
         const int r1 = static_cast<int>((eos < base + C ? eos : base + C) - base);
         const bool more = base + r1 < eos;
         const uint32_t dq = SH_COL_DQ + 128u * buf;
-        bool mine = true;
 
-        // ---- product 1 (bar_d) --------------------------------------------
         if (tid == SH_ISSUER) {
-            mine = wait_one(B_A);
-            if (mine) {
-                const uint32_t ID_DQ = tc::idesc_bf16_f32(128, 2 * SH_COLS, true, true, true);
-                const uint32_t ID_DL = tc::idesc_bf16_f32(128, SH_COLS, true, true, true);
-                mma_mn_mn<K / 16>(tmem + dq, sm.rec_a + REC_WQ_HI, WQ_COLS, sm.st, 2 * SH_COLS, ID_DQ, false);
-                mma_mn_mn<K / 16>(tmem + SH_COL_DL, sm.rec_a + REC_W_LO, C, sm.st, 2 * SH_COLS, ID_DL, false);
-                tc::mma_commit(&sm.bar[SH_BAR_D]);
-                note(B_D);
-            }
-        }
-        // the piece's decay and scale (every worker: the rescale is shared)
-        float cn = 0.f, dscale = 0.f;
-        bool rescale = false;
-        if (worker) {
-            mine = wait_one(B_R);
-            if (mine) {
-                cn = cs * expf(sm.rec_s[C + r1 - 1]);         // e^gamma at the piece's last row
-                rescale = !(cn >= 0x1p-60f && cn <= 0x1p60f);
-                dscale = rescale ? 1.f : __fdividef(1.f, cn);
-            }
-        }
-        if (out_warp && t > bos && mine)
-            mine = write_outputs(blk - 1, buf ^ 1, prev_cs, cs);
-        if (delta_warp && mine) {
-            // ---- Delta~ rows i (thread: row i, columns cb..) ----------------
-            if (warp < 4)
-                sm.fo[buf][row] = sm.rec_s[row];
-            mine = wait_one(B_D);
-            if (mine) {
-                float dh[SH_CP], dl[SH_CP], dw[SH_CP];
-                tc::tmem_ld16(my_lane + dq + cb, dh);
-                tc::tmem_ld16(my_lane + dq + SH_COLS + cb, dl);
-                tc::tmem_ld16(my_lane + SH_COL_DL + cb, dw);
-                tc::tmem_wait_ld();
-                const bool live = row >= r0 && row < r1;
-#pragma unroll
-                for (int e = 0; e < SH_CP; ++e)
-                    dh[e] = live ? fmaf(cs, (dh[e] + dl[e]) + dw[e], sm.ut[(cb + e) * C + row]) * dscale : 0.f;
-                st_row8_hilo(sm.dt[0], sm.dt[1], row, cb, SH_COLS, dh);
-                st_row8_hilo(sm.dt[0], sm.dt[1], row, cb + 8, SH_COLS, dh + 8);
-            }
-        }
-        if (worker && mine && rescale) {      // S~ <- cs' S~ in TMEM; the scale returns to 1
-            float y[SH_CP];
-            tc::tmem_ld16(my_lane + SH_COL_S + cb, y);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < SH_CP; ++e)
-                y[e] *= cn;
-            tc::tmem_st16(my_lane + SH_COL_S + cb, y);
-            tc::tmem_wait_st();
-        }
-        const float cs_new = rescale ? 1.f : cn;
-        ok = publish(mine);
-        if (!ok)
-            break;
+            // ---- product 1 (bar_d) once this piece's state tiles and W / Q are in
+            mine = wait_one(B_TR) && wait_one(B_A);
+            if (!mine)
+                break;
+            const uint32_t ID_DQ = tc::idesc_bf16_f32(128, 2 * SH_COLS, true, true, true);
+            const uint32_t ID_DL = tc::idesc_bf16_f32(128, SH_COLS, true, true, true);
+            mma_mn_mn<K / 16>(tmem + dq, sm.rec_a + REC_WQ_HI, WQ_COLS, sm.st, 2 * SH_COLS, ID_DQ, false);
+            mma_mn_mn<K / 16>(tmem + SH_COL_DL, sm.rec_a + REC_W_LO, C, sm.st, 2 * SH_COLS, ID_DL, false);
+            tc::mma_commit(&sm.bar[SH_BAR_D]);
+            note(B_D);
 
-        // ---- product 2a: S~ += K'^T Delta~ (bar_s); 2b: O2 = P Delta~ (bar_o)
-        if (tid == SH_ISSUER) {
-            mine = wait_one(B_B);
-            if (mine) {
-                const uint32_t ID = tc::idesc_bf16_f32(128, SH_COLS, false, true, true);
-                const unsigned char *kp_hi = sm.rec_b[buf], *kp_lo = sm.rec_b[buf] + (REC_KP_LO - REC_KP_HI);
-                mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_hi, KP_COLS, sm.dt[0], SH_COLS, ID, true);
-                mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_hi, KP_COLS, sm.dt[1], SH_COLS, ID, true);
-                mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_lo, KP_COLS, sm.dt[0], SH_COLS, ID, true);
-                tc::mma_commit(&sm.bar[SH_BAR_S]);
-                note(B_S);
-                mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_hi + 1024, KP_COLS, sm.dt[0], SH_COLS, ID, false);
-                mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_hi + 1024, KP_COLS, sm.dt[1], SH_COLS, ID, true);
-                mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_lo + 1024, KP_COLS, sm.dt[0], SH_COLS, ID, true);
-                tc::mma_commit(&sm.bar[SH_BAR_O]);
-                note(B_O);
-            }
-            if (mine && more) {
-                // the next piece's copies: product 1 is done and U / fo / gamma
-                // were read (both before the barrier above); the other K' / P
-                // buffer was last read by the previous piece's product 2b, which
-                // the output warps waited for before that barrier; and the
-                // piece after next into L2
+            // ---- product 2a: S~ += K'^T Delta~ (bar_s); 2b: O2 = P Delta~
+            // (bar_o), once every worker's Delta~ tiles and rescale are in
+            mine = wait_one(B_DR) && wait_one(B_B);
+            if (!mine)
+                break;
+            if (more) {
+                // the next piece's copies, ahead of this piece's product 2:
+                // product 1 is done and U / fo / gamma were read (both before
+                // every worker's arrival on bar_dr); the other K' / P buffer was
+                // last read by the previous piece's product 2b, issued before
+                // this piece's product 1, whose completion bar_d reported; and
+                // the piece after next into L2
                 const unsigned char *rn = rec_of(blk + 1);
                 sync::mbar_arrive_expect_tx(&sm.bar[SH_BAR_A], REC_A_BYTES);
                 sync::bulk_load(sm.rec_a, rn, REC_A_BYTES, &sm.bar[SH_BAR_A]);
@@ -377,34 +321,84 @@ __global__ void __launch_bounds__(SH_THREADS, 1) gdn_chunk_state_half_kernel(con
                 if ((blk + 2) * C < eos)
                     prefetch_piece(blk + 2);
             }
-        }
-
-        // ---- the next piece's state tiles, or the final write-back --------
-        if (worker) {
-            mine = wait_one(B_S);
-            if (mine) {
+            const uint32_t ID = tc::idesc_bf16_f32(128, SH_COLS, false, true, true);
+            const unsigned char *kp_hi = sm.rec_b[buf], *kp_lo = sm.rec_b[buf] + (REC_KP_LO - REC_KP_HI);
+            mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_hi, KP_COLS, sm.dt[0], SH_COLS, ID, true);
+            mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_hi, KP_COLS, sm.dt[1], SH_COLS, ID, true);
+            mma_mn_mn<C / 16>(tmem + SH_COL_S, kp_lo, KP_COLS, sm.dt[0], SH_COLS, ID, true);
+            tc::mma_commit(&sm.bar[SH_BAR_S]);
+            note(B_S);
+            mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_hi + 1024, KP_COLS, sm.dt[0], SH_COLS, ID, false);
+            mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_hi + 1024, KP_COLS, sm.dt[1], SH_COLS, ID, true);
+            mma_mn_mn<C / 16>(tmem + SH_COL_O2, kp_lo + 1024, KP_COLS, sm.dt[0], SH_COLS, ID, true);
+            tc::mma_commit(&sm.bar[SH_BAR_O]);
+            note(B_O);
+        } else if (worker) {
+            // ---- the piece's decay and scale (every worker: the rescale is shared)
+            mine = wait_one(B_R);
+            if (!mine)
+                break;
+            const float cn = cs * expf(sm.rec_s[C + r1 - 1]);     // e^gamma at the piece's last row
+            const bool rescale = !(cn >= 0x1p-60f && cn <= 0x1p60f);
+            const float dscale = rescale ? 1.f : __fdividef(1.f, cn);
+            const float cs_new = rescale ? 1.f : cn;
+            if (out_warp) {
+                if (t > bos && !(mine = write_outputs(blk - 1, buf ^ 1, fo_j, prev_cs, cs)))
+                    break;
+                fo_j = sm.rec_s[row - C];
+            } else {
+                // ---- Delta~ rows i (thread: row i, columns cb..) ------------
+                if (!(mine = wait_one(B_D)))
+                    break;
+                float dh[SH_CP], dl[SH_CP], dw[SH_CP];
+                tc::tmem_ld16(my_lane + dq + cb, dh);
+                tc::tmem_ld16(my_lane + dq + SH_COLS + cb, dl);
+                tc::tmem_ld16(my_lane + SH_COL_DL + cb, dw);
+                tc::tmem_wait_ld();
+                const bool live = row >= r0 && row < r1;
+#pragma unroll
+                for (int e = 0; e < SH_CP; ++e)
+                    dh[e] = live ? fmaf(cs, (dh[e] + dl[e]) + dw[e], sm.ut[(cb + e) * C + row]) * dscale : 0.f;
+                st_row8_hilo(sm.dt[0], sm.dt[1], row, cb, SH_COLS, dh);
+                st_row8_hilo(sm.dt[0], sm.dt[1], row, cb + 8, SH_COLS, dh + 8);
+            }
+            if (rescale) {      // S~ <- cs' S~ in TMEM; the scale returns to 1
                 float y[SH_CP];
                 tc::tmem_ld16(my_lane + SH_COL_S + cb, y);
                 tc::tmem_wait_ld();
-                if (more) {
-                    st_row8_hilo(sm.st, sm.st + 1024, row, cb, 2 * SH_COLS, y);
-                    st_row8_hilo(sm.st, sm.st + 1024, row, cb + 8, 2 * SH_COLS, y + 8);
-                } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
-                    float4 *dst = reinterpret_cast<float4 *>(s_gmem + static_cast<int64_t>(row) * V + v0 + cb);
 #pragma unroll
-                    for (int m = 0; m < SH_CP / 4; ++m)
-                        __stcs(dst + m, make_float4(cs_new * y[4 * m], cs_new * y[4 * m + 1], cs_new * y[4 * m + 2],
-                                                    cs_new * y[4 * m + 3]));
-                }
+                for (int e = 0; e < SH_CP; ++e)
+                    y[e] *= cn;
+                tc::tmem_st16(my_lane + SH_COL_S + cb, y);
+                tc::tmem_wait_st();
             }
+            arrive(B_DR);
+
+            // ---- the next piece's state tiles, or the final write-back ----
+            if (!(mine = wait_one(B_S)))
+                break;
+            float y[SH_CP];
+            tc::tmem_ld16(my_lane + SH_COL_S + cb, y);
+            tc::tmem_wait_ld();
+            if (more) {
+                st_row8_hilo(sm.st, sm.st + 1024, row, cb, 2 * SH_COLS, y);
+                st_row8_hilo(sm.st, sm.st + 1024, row, cb + 8, 2 * SH_COLS, y + 8);
+                arrive(B_TR);
+            } else if (!(p.flags & GDN_NO_FINAL_WRITEBACK)) {
+                float4 *dst = reinterpret_cast<float4 *>(s_gmem + static_cast<int64_t>(row) * V + v0 + cb);
+#pragma unroll
+                for (int m = 0; m < SH_CP / 4; ++m)
+                    __stcs(dst + m, make_float4(cs_new * y[4 * m], cs_new * y[4 * m + 1], cs_new * y[4 * m + 2],
+                                                cs_new * y[4 * m + 3]));
+            }
+            prev_cs = cs;
+            cs = cs_new;
         }
-        prev_cs = cs;
-        cs = cs_new;
         t = base + r1;
-        ok = publish(mine);
     }
-    if (ok && out_warp)
-        write_outputs(blk - 1, buf ^ 1, prev_cs, cs);
+    if (mine && out_warp)
+        mine = write_outputs(blk - 1, buf ^ 1, fo_j, prev_cs, cs);
+    const bool ok = __syncthreads_and(mine) != 0;
 
     // after a failed wait, copies or products may still be in flight: let
     // them finish (bounded) before the shared and tensor memory is released

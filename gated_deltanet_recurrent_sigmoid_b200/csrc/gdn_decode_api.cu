@@ -30,23 +30,31 @@ constexpr int kHeadV = 128;
 // mean sequence length L = T_tot / N and the (sequence, value head) pair
 // count P = N * HV (measured B200 crossovers, lengths spread over
 // [L/2, 3L/2]):
-//   - the split kernels (with a large enough caller workspace) from L >= 128
-//     when P < 128, L >= 192 when P < 256, L >= 512 when P < 512, never
-//     beyond: only few, long sequences gain from computing every block's
-//     products in parallel first (back-to-back calls: 8 sequences at
-//     L = 470, 116 vs 183 us; 16 at 130, 54 vs 51, at 283, 85 vs 98; 32 at
-//     506, 255 vs 261; 64 sequences: the on-chip kernel is 4-10 % faster at
-//     every length up to 2,085, 128 sequences 16-20 %);
+//   - the split kernels (with a large enough caller workspace) from L >= 80
+//     while two state CTAs per pair fit one wave (2 P <= the SM count), from
+//     L >= 144 when P < 128, L >= 192 when P < 256, L >= 512 when P < 512,
+//     never beyond: only few, long sequences gain from computing every
+//     block's products in parallel first.  The on-chip kernel's time steps
+//     with the longest sequence's chunk count (~13 us a chunk), the split
+//     schedule's grows by ~3 us a piece from ~22 us (device-timed graphs of
+//     24 calls: 8 pairs at L = 84, 25.5 vs 28.0 us; 64 pairs at L = 94, 29.5
+//     vs 40.0, at 70, 26.4 vs 28.0; 80 pairs at 131, 46.0 vs 44.1, at 177,
+//     53.2 vs 59.2; 120 pairs at 135, 48.9 vs 46.9, at 147, 53.6 vs 59.5;
+//     back-to-back calls: 32 sequences at L = 506, 255 vs 261 us; 64
+//     sequences: the on-chip kernel is 4-10 % faster at every length up to
+//     2,085, 128 sequences 16-20 %);
 //   - the on-chip chunked kernel from L >= 20 when P < 64, L >= 14 when
 //     P < 512, L >= 13 beyond (its one-CTA chain costs ~20 us, so with few
 //     pairs the per-token kernel wins longer: 1 sequence 28.7 vs 22.5 us at
 //     L = 32, 8: 26.6 vs 21.4 at 19; 1024 sequences 513 vs 539 us at 11.9,
 //     663 vs 550 at 16);
 //   - the per-token kernel otherwise.
-bool split_pays(int64_t pairs, int64_t T_tot, int64_t N)
+bool split_pays(int64_t pairs, int64_t T_tot, int64_t N, int sms)
 {
+    if (2 * pairs <= sms)
+        return T_tot >= 80 * N;
     if (pairs < 128)
-        return T_tot >= 128 * N;
+        return T_tot >= 144 * N;
     if (pairs < 256)
         return T_tot >= 192 * N;
     if (pairs < 512)
@@ -223,6 +231,22 @@ cudaError_t once_per_device(PerDevice &pd, int dev, Init &&init)
     return err;
 }
 
+// Streaming multiprocessors of the current device (read once per device).
+cudaError_t current_sm_count(int *sms)
+{
+    static PerDevice once;
+    static int count[PerDevice::kMaxDevices];      // written once per device, inside `once`
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess)
+        err = once_per_device(once, dev, [&]() {
+            return cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+        });
+    if (err == cudaSuccess)
+        *sms = count[dev];
+    return err;
+}
+
 // Host-side index check (GDN_CHECK_INDICES).
 int check_indices_on_host(const int32_t *d_idx, const int32_t *d_cu, int64_t N, int64_t num_slots,
                           int64_t T_tot, cudaStream_t stream)
@@ -287,16 +311,19 @@ cudaError_t launch(const gdn::DecodeParams &p, int64_t units, cudaStream_t strea
 }
 
 // Split chunked schedule: the block kernel over ceil(T_tot / 64) x HV CTAs,
-// then the state kernel over the (sequence, value head) pairs.  The state
+// then a state kernel over the (sequence, value head) pairs: two CTAs per
+// pair (half the state columns each) while they fit one wave, the compact
+// form for many short sequences, else the full-width form.  The state
 // kernel always uses programmatic dependent launch behind the block kernel
 // (it waits for the block kernel's completion before reading anything).
 cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t units, cudaStream_t stream,
                          bool pdl, bool l2norm)
 {
     static PerDevice once;
-    static int sm_count[PerDevice::kMaxDevices];      // written once per device, inside `once`
-    int dev = 0;
+    int dev = 0, sms = 0;
     cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess)
+        err = current_sm_count(&sms);
     if (err != cudaSuccess)
         return err;
     const size_t smem_wy = sizeof(gdn::split::WySmem), smem_st = sizeof(gdn::split::StSmem);
@@ -325,8 +352,6 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(gdn::split::gdn_chunk_state_compact_kernel,
                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (e == cudaSuccess)
-            e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
         return e;
     });
     if (err != cudaSuccess)
@@ -339,11 +364,11 @@ cudaError_t launch_split(const gdn::DecodeParams &p, unsigned char *ws, int64_t 
     // Few (sequence, head) pairs: two CTAs per pair, each on half the state
     // columns, as long as they fit one wave; many pairs: the compact state
     // kernel (two CTAs per SM); otherwise the full-width kernel.
-    if (2 * units <= sm_count[dev])
+    if (2 * units <= sms)
         return launch_ex(gdn::split::gdn_chunk_state_half_kernel, dim3(static_cast<unsigned>(2 * units)),
                          dim3(gdn::split::SH_THREADS), sizeof(gdn::split::ShSmem), stream, true, p,
                          static_cast<const unsigned char *>(ws));
-    if (units >= kSplitCompactMinUnitsPerSm * sm_count[dev] &&
+    if (units >= kSplitCompactMinUnitsPerSm * sms &&
         static_cast<int64_t>(p.T_tot) <= kSplitCompactMaxMeanTokens * p.N)
         return launch_ex(gdn::split::gdn_chunk_state_compact_kernel, dim3(static_cast<unsigned>(units)),
                          dim3(gdn::split::SC_THREADS), sizeof(gdn::split::StSmemCompact), stream, true, p,
@@ -672,7 +697,10 @@ int run_update(const UpdateArgs &c)
         aligned(v->data, 16) && stride_ok(T_tot, Lv.tok, 8) && stride_ok(HV, v->stride[v->ndim - 2], 8);
     if (schedule == GDN_SCHEDULE_AUTO && !(extra && (extra->tile_v || extra->tile_rows)) &&
         act == GDN_DTYPE_BF16 && !c.given_gates && !want_inter && v_rows_16b && N > 0) {
-        if (ws_fits && split_pays(N * HV, T_tot, N))
+        int sms = 0;
+        if (ws_fits && current_sm_count(&sms) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        if (ws_fits && split_pays(N * HV, T_tot, N, sms))
             schedule = GDN_SCHEDULE_CHUNKED_SPLIT;
         else if (T_tot >= chunked_min_mean_tokens(N * HV) * N)
             schedule = GDN_SCHEDULE_CHUNKED;

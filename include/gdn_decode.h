@@ -130,7 +130,8 @@ extern "C" {
                                     kernels (bf16 activations, fused gates, no
                                     per-token states, v rows 16-byte aligned):
                                     GDN_SCHEDULE_CHUNKED_SPLIT if the caller gives
-                                    a large enough workspace and L >= 128
+                                    a large enough workspace and L >= 80
+                                    (2 P <= the device's SM count), >= 144
                                     (P < 128), >= 192 (P < 256) or >= 512
                                     (P < 512); else GDN_SCHEDULE_CHUNKED if
                                     L >= 20 (P < 64), >= 14 (P < 512) or >= 13.

@@ -47,6 +47,9 @@ def test_reference_arm_prints_the_contract_line():
     (False, 512, 480.0, "gdn::local::gdn_chunk_local_kernel<true>"),           # prefill_b64_t512
     (False, 256, 600.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
     (False, 128, 150.0, "gdn::local::gdn_chunk_local_kernel<true>"),
+    (False, 64, 90.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_half_kernel"),
+    (False, 96, 130.0, "gdn::local::gdn_chunk_local_kernel<true>"),
+    (False, 96, 150.0, "gdn::split::gdn_chunk_wy_kernel<true> + gdn::split::gdn_chunk_state_kernel"),
     (False, 1024, 12.0, "gdn::gdn_decode_kernel<128,128,16,8>"),
 ])
 def test_kernel_name_mirrors_the_documented_choice(one_token, pairs, mean, expected):
@@ -66,9 +69,12 @@ def test_split_schedule_names_its_state_kernel():
 def test_auto_thresholds_match_the_header():
     """The thresholds the bench mirrors are the ones the header documents."""
     header = " ".join(open(os.path.join(ROOT, "include", "gdn_decode.h")).read().split())
-    assert "L >= 128 (P < 128), >= 192 (P < 256) or >= 512 (P < 512)" in header
+    assert ("L >= 80 (2 P <= the device's SM count), >= 144 (P < 128), >= 192 (P < 256) or >= 512 (P < 512)"
+            in header)
     assert "L >= 20 (P < 64), >= 14 (P < 512) or >= 13" in header
-    assert [bench.split_pays(p, m) for p, m in ((127, 128), (127, 127), (128, 192), (128, 191), (511, 512),
-                                                (511, 511), (512, 100000))] == [True, False, True, False, True,
-                                                                                 False, False]
+    assert [bench.split_pays(p, m) for p, m in ((74, 80), (74, 79), (75, 144), (75, 143), (127, 144), (127, 143),
+                                                (128, 192), (128, 191), (511, 512), (511, 511),
+                                                (512, 100000))] == [True, False, True, False, True, False, True,
+                                                                    False, True, False, False]
+    assert bench.split_pays(64, 100, sms=120) is False and bench.split_pays(64, 100, sms=128) is True
     assert [bench.chunked_min_mean_tokens(p) for p in (8, 63, 64, 511, 512, 8192)] == [20, 20, 14, 14, 13, 13]

@@ -158,7 +158,8 @@ def _bits_equal(a, b):
 def test_auto_schedule_picks_by_length_and_pairs():
     """GDN_SCHEDULE_AUTO (bit-identical to asking for the schedule it picks):
     few long sequences run the split kernels when a workspace is given (the
-    binding allocates one) and the on-chip chunked kernel without one;
+    binding allocates one) and the on-chip chunked kernel without one -- with
+    few enough pairs from 80 tokens per sequence on average;
     sequences of a few dozen tokens run the on-chip chunked kernel either
     way; short ones, or a call with per-token states, the per-tile kernel."""
     long_w = problem([200, 150, 300], seed=21)                 # 24 pairs, mean 217
@@ -170,6 +171,11 @@ def test_auto_schedule_picks_by_length_and_pairs():
     assert _bits_equal(auto_nows, chunked)
     per_tile, _, _ = run_gpu(long_w, schedule=binding.SCHEDULE_PER_TILE)
     assert not _bits_equal(auto, per_tile) and not _bits_equal(auto, chunked)
+
+    two_cta_w = problem([70, 90, 110], seed=24)               # 24 pairs, mean 90: two state CTAs a pair
+    auto, _, _ = run_gpu(two_cta_w)
+    split, _, _ = run_gpu(two_cta_w, schedule=SPLIT)
+    assert _bits_equal(auto, split)
 
     mid_w = problem([30, 60, 10, 45], seed=23)                # 32 pairs, mean 36
     auto, _, _ = run_gpu(mid_w)

@@ -77,9 +77,9 @@ def test_auto_with_intermediates_long_sequences():
 
 
 def test_auto_without_workspace_short_mean_long_sequence():
-    """Without a workspace AUTO keeps the per-token kernel below 128 tokens
-    per sequence on average, so one 2,048-token sequence among short ones
-    runs there."""
+    """Without a workspace AUTO never runs the split kernels: one 2,048-token
+    sequence among 30 short ones (124 pairs, 78 tokens per sequence on
+    average) runs on the on-chip chunked kernel, chunk after chunk."""
     lens = [2048] + [3, 9, 17, 1, 30] * 6
     w = random_workload(lens, H=2, HV=4, seed=103, weak_heads=(1, 3), pad=(4,))
     check_whole(w, "auto_no_workspace_per_tile", workspace=None)
