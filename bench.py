@@ -464,6 +464,8 @@ def main():
     ap.add_argument("--tile-rows", type=int, default=0)
     ap.add_argument("--schedule", default="auto", choices=["auto", "per_tile", "pipelined", "chunked", "split"])
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--e2e-depth", type=int, default=3,
+                    help="host-fed steps in flight in the pipelined e2e loop (staging slots)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-per-config", action="store_true",
@@ -616,7 +618,7 @@ def main():
                 dist.all_reduce(te, op=dist.ReduceOp.MAX)
             return float(te.item()) / args.e2e_steps
 
-        pipe = binding.PipelinedHostDecode(*staged_args, stream=stream, **staged_kw)
+        pipe = binding.PipelinedHostDecode(*staged_args, stream=stream, depth=args.e2e_depth, **staged_kw)
         for slot in pipe.slots:
             fill(slot)
         for _ in range(4):
