@@ -97,7 +97,7 @@ struct Smem {
     int failed;
 };
 
-static_assert(offsetof(Smem, ua) % 16 == 0, "ua is read as 16-byte vectors");
+static_assert(offsetof(Smem, ua) % 16 == 0 && offsetof(Smem, wc) % 16 == 0, "ua and wc are read as 16-byte vectors");
 
 template <bool L2NORM>
 __global__ void __launch_bounds__(THREADS, 2) gdn_chunk_local_kernel(const __grid_constant__ DecodeParams p)
@@ -411,14 +411,15 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_chunk_local_kernel(const __gri
         if (!ok)
             break;
 
-        // ---- A by columns (lanes 0..63: K K^T is symmetric, so lane c holds
-        // column c; A[j][c] is nonzero for c < j < n) into k1, and P by rows
-        // (lanes 64..127: row j of Q K^T; P[j][i] for i <= j < n) as hi / lo
-        // tiles into k0.  Each lane's two threads take half of the columns.
+        // ---- A by columns into k1 (lanes 0..63: lane c holds row c of K K^T;
+        // A[c][j] is nonzero for j < c < n, stored at column j, row c, so the
+        // lanes' stores are consecutive words), and P by rows (lanes 64..127:
+        // row j of Q K^T; P[j][i] for i <= j < n) as hi / lo tiles into k0.
+        // Each lane's two threads take half of the columns.
         float *const At = reinterpret_cast<float *>(k1);
         if ((warp & 3) < 2) {
             const int c = v;
-            const float w = sm.wc[c];
+            const float uc = sm.ua[c];
 #pragma unroll
             for (int jb = ib; jb < ib + 32; jb += 16) {
                 float kk16[16];
@@ -427,13 +428,13 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_chunk_local_kernel(const __gri
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const int j0 = jb + 4 * e4;
-                    const float4 u4 = *reinterpret_cast<const float4 *>(sm.ua + j0);
-                    float4 a4;
-                    a4.x = (j0 > c && j0 < n) ? kk16[4 * e4] * ex2_approx(u4.x - w) : 0.f;
-                    a4.y = (j0 + 1 > c && j0 + 1 < n) ? kk16[4 * e4 + 1] * ex2_approx(u4.y - w) : 0.f;
-                    a4.z = (j0 + 2 > c && j0 + 2 < n) ? kk16[4 * e4 + 2] * ex2_approx(u4.z - w) : 0.f;
-                    a4.w = (j0 + 3 > c && j0 + 3 < n) ? kk16[4 * e4 + 3] * ex2_approx(u4.w - w) : 0.f;
-                    *reinterpret_cast<float4 *>(At + c * 64 + j0) = a4;
+                    const float4 w4 = *reinterpret_cast<const float4 *>(sm.wc + j0);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = j0 + e;
+                        At[j * 64 + c] = (j < c && c < n) ? kk16[4 * e4 + e] * ex2_approx(uc - wv[e]) : 0.f;
+                    }
                 }
             }
         } else {

@@ -552,31 +552,35 @@ __global__ void __launch_bounds__(THREADS, 4) gdn_chunk_wy_kernel(const __grid_c
     float t8[4][8];     // rows of T, kept for the two T diag() tile pairs
     if (ok) {
         // ---- step 3: A and P^T by columns of K [K;Q]^T (warps 0, 1) and the
-        // K' rows (warps 2, 3).  K K^T is symmetric, so TMEM lane c (row c)
-        // holds column c of it: thread c writes column c of A into At as
-        // contiguous 16-byte vectors, and row c of P^T (K Q^T row c) to the
-        // record.  A[j][c] is nonzero for c < j in the same segment, i.e.
-        // c < j < se_c; P[j][c] for c <= j < se_c.
+        // K' rows (warps 2, 3).  TMEM lane c holds row c of K K^T and of
+        // K Q^T: thread c writes row c of A into At (column j, row c: the
+        // lanes' stores are consecutive words; writing column c of the
+        // symmetric K K^T as 16-byte vectors instead was a 32-way bank
+        // conflict) and row c of P^T to the record.  A[c][j] is nonzero for
+        // j < c in the same segment, i.e. ss_c <= j < c; P[j][c] for
+        // c <= j < se_c.
         if (tid < 64) {
-            const int c = tid, ce = sm.se[c];
-            const float w = sm.wc[c];
+            const int c = tid, cs0 = sm.ss[c], ce = sm.se[c];
+            const float uc = sm.ua[c], w = sm.wc[c];
 #pragma unroll 1
             for (int jb = 0; jb < 64; jb += 16) {
                 float kk16[16];
                 tc::tmem_ld16(my_lane + WY_COL_KQ + jb, kk16);
                 tc::tmem_wait_ld();
+                // A[c][j] = 2^(ua_c - wc_j) (K K^T)[c][j]
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const int j0 = jb + 4 * e4;
-                    const float4 u4 = *reinterpret_cast<const float4 *>(sm.ua + j0);
-                    float4 a4;
-                    a4.x = (j0 > c && j0 < ce) ? kk16[4 * e4] * ex2_approx(u4.x - w) : 0.f;
-                    a4.y = (j0 + 1 > c && j0 + 1 < ce) ? kk16[4 * e4 + 1] * ex2_approx(u4.y - w) : 0.f;
-                    a4.z = (j0 + 2 > c && j0 + 2 < ce) ? kk16[4 * e4 + 2] * ex2_approx(u4.z - w) : 0.f;
-                    a4.w = (j0 + 3 > c && j0 + 3 < ce) ? kk16[4 * e4 + 3] * ex2_approx(u4.w - w) : 0.f;
-                    *reinterpret_cast<float4 *>(At + at_idx(c, j0)) = a4;
+                    const float4 w4 = *reinterpret_cast<const float4 *>(sm.wc + j0);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = j0 + e;
+                        At[at_idx(j, c)] = (j < c && j >= cs0) ? kk16[4 * e4 + e] * ex2_approx(uc - wv[e]) : 0.f;
+                    }
                 }
             }
+
 #pragma unroll 1
             for (int jb = 0; jb < 64; jb += 16) {
                 float pt[16];
