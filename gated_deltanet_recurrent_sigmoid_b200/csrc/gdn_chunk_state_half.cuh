@@ -50,8 +50,8 @@ constexpr uint32_t SH_COL_DQ = 256;            // [D | O1], hi and lo halves: 12
 enum { SH_BAR_A, SH_BAR_B, SH_BAR_R, SH_BAR_D, SH_BAR_S, SH_BAR_O, SH_BAR_DR, SH_BAR_TR, SH_NBAR };
 
 struct ShSmem {
-    // [S~hi | S~lo] [k][v' | v'], the MN-major B operand of product 1 (64 KB
-    // of state columns split: 128 rows of 2 x 64 columns)
+    // [S~hi | S~lo] [k][v' | v'], the MN-major B operand of product 1 (32 KB:
+    // 128 rows k, this CTA's 64 columns as hi parts, then as lo parts)
     alignas(1024) unsigned char st[128 * 128 * 2];
     alignas(1024) unsigned char rec_a[REC_A_BYTES];     // [W^T hi | Q^T], W^T lo of the piece
     alignas(1024) unsigned char rec_b[2][REC_B_BYTES];  // [K' | P^T] hi, lo by piece parity (follows rec_a)
