@@ -161,8 +161,10 @@ extern "C" {
                                     masked q.k matrix) for every 64-token block
                                     of the packed token range at once, written to
                                     the caller's workspace; then the recurrence
-                                    through the state, one CTA per (sequence,
-                                    value head).  Same restrictions as
+                                    through the state: two CTAs per (sequence,
+                                    value head), each on half of the state's
+                                    columns, while 2 P <= the SM count; else
+                                    one per pair.  Same restrictions as
                                     GDN_SCHEDULE_CHUNKED, plus a workspace of
                                     gdn_chunked_workspace_bytes(T_tot, HV) bytes
                                     in gdn_extra */
