@@ -20,7 +20,10 @@
 //                           (row by row, as the block kernel produces them).
 //   gdn_chunk_state_kernel  one 544-thread CTA per (sequence, value head) (or, for
 //                           many short sequences, gdn_chunk_state_compact_kernel:
-//                           256 threads, two CTAs per SM): walks the
+//                           256 threads, two CTAs per SM; for few pairs,
+//                           gdn_chunk_state_half_kernel in
+//                           gdn_chunk_state_half.cuh: two CTAs per pair, each
+//                           on half of the state's columns): walks the
 //                           blocks the sequence covers, fetching each block's
 //                           tiles with bulk copies one step ahead, and runs
 //                           only the state-dependent products.
