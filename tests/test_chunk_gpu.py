@@ -176,6 +176,10 @@ def test_auto_schedule_picks_by_length_and_pairs():
     auto, _, _ = run_gpu(two_cta_w)
     split, _, _ = run_gpu(two_cta_w, schedule=SPLIT)
     assert _bits_equal(auto, split)
+    below_w = problem([60, 70, 80], seed=25)                  # 24 pairs, mean 70: below the split range
+    auto, _, _ = run_gpu(below_w)
+    chunked, _, _ = run_gpu(below_w, schedule=CHUNKED)
+    assert _bits_equal(auto, chunked)
 
     mid_w = problem([30, 60, 10, 45], seed=23)                # 32 pairs, mean 36
     auto, _, _ = run_gpu(mid_w)
