@@ -72,6 +72,26 @@ NCU_TRAFFIC = {"kernel_sha256": "56a5bd6fd0f772dbd0de9456b16af0c872fa8c6c4137184
                "workload": "decode_b512_hv8", "bytes_per_launch": 257377792 + 202355968}
 
 
+def h2d_link_gbs(nbytes, device, reps=40):
+    """Pinned host -> device copy rate (GB/s) for a copy of `nbytes`: a warm-up
+    copy, then `reps` copies back to back on one stream, timed with events."""
+    import torch
+    if nbytes <= 0:
+        return None
+    host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dev = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    s = torch.cuda.Stream(device)
+    with torch.cuda.stream(s):
+        dev.copy_(host, non_blocking=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            dev.copy_(host, non_blocking=True)
+        e1.record()
+    s.synchronize()
+    return round(nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9, 1)
+
+
 def kernel_source_hash() -> str:
     """Hash of the per-tile kernel's device code (the kernel the traffic figure
     belongs to)."""
@@ -636,10 +656,15 @@ def main():
         torch.cuda.nvtx.range_push("e2e: pipelined host-fed steps")
         e2e_ms = timed(run_pipe)
         torch.cuda.nvtx.range_pop()
+        link = h2d_link_gbs(int(pipe.h2d_bytes), device)
         e2e = {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                "us_per_call": round(e2e_ms * 1e3, 3), "h2d_bytes_per_step": int(pipe.h2d_bytes),
                "d2h_bytes_per_step": int(pipe.d2h_bytes), "api": "binding.PipelinedHostDecode",
                "pipeline_depth": pipe.depth,
+               # the host link's pinned host -> device rate, right after the loop:
+               # a step cannot take less than h2d_bytes_per_step / this
+               "h2d_link_gbs": link,
+               "h2d_floor_us": round(pipe.h2d_bytes / (link * 1e3), 3) if link else None,
                "how": "each step: pinned host inputs -> device, update, output -> pinned host; the host "
                       "receives every step's output; copies overlap the neighbouring steps' kernels"}
         del pipe
